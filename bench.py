@@ -1,0 +1,419 @@
+"""Benchmark of one QSA (c4) layer decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: decode, batch 64 per GPU, one query token per request, contexts
+uniform in [120000, 131072], 16 query / 2 KV heads, d = 128, paged BF16 K/V
+(64-token pages, seeded page permutation), 4 x 128 indexer heads; synthetic
+inputs from qsa_gen.  One step = one qsa_decode call (ring append and
+compression, query rotation, scoring of every complete block, top-512,
+expansion, sparse GQA).  Every step streams ~650 MB (5x the L2), and the L2
+is also flushed (512 MiB write) between timed steps, outside the timed
+events.  Several GPUs run independent replicas (requests shard with no
+exchange): weak scaling, time = max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QSA decode query-tok/s/layer at 128K ctx; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "query-tok/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--batch", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_src_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+SCORER_SRC = ["block_sparse_attention_c4_b200/csrc/qsa_score.cu", "block_sparse_attention_c4_b200/csrc/qsa_common.cuh"]
+
+
+def committed_traffic(src_hash: str):
+    """DRAM bytes per launch of the scorer from a committed ncu summary, if it matches this source."""
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.txt")):
+        txt = open(path).read()
+        m_h = re.search(r"^kernel_src_sha256_16:\s*(\w+)", txt, re.M)
+        m_k = re.search(r"^kernel:\s*(\S+)", txt, re.M)
+        m_b = re.search(r"^dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt, re.M)
+        if m_h and m_k and m_b and m_k.group(1) == "k_score_topk" and m_h.group(1) == src_hash:
+            return float(m_b.group(1)), os.path.relpath(path, ROOT)
+    return None, None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu, self.proc, self.lines = gpu_index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_bytes(lens):
+    """Bytes a decode step must move at minimum, per kernel (see the design notes):
+    scorer: every complete block's compressed key (256 B) + query/weights + page-table entries + kept ids;
+    gqa: K and V of both KV heads at every kept position (1 KiB) + query + output + kept ids."""
+    score = gqa = 0
+    for L in lens:
+        nb = L // 4
+        npos = 4 * min(nb, 512) + L % 4
+        score += nb * 256 + 4 * 128 * 2 + 16 + 4 * ((nb + 15) // 16) + 4 * min(nb, 512)
+        gqa += npos * 1024 + 16 * 128 * 2 * 2 + 4 * min(nb, 512)
+    return score, gqa
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+    import qsa_gen as G
+    from block_sparse_attention_c4_b200 import build
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=300))
+
+    wl = G.decode_128k(seed=2 + 1000 * rank, batch=args.batch)
+    lens = [int(x) for x in wl.lens]
+    t0 = time.time()
+    cache = W.build_cache(wl, device=dev)
+    inp = W.decode_inputs(wl, device=dev)
+    torch.cuda.synchronize()
+    setup_s = time.time() - t0
+    B, max_len = wl.batch, max(lens)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_DECODE, B, max_len), device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    nk = Q.decode_kernel_count()
+
+    def step():
+        Q.decode(cache, inp["idx_k_new"], inp["idx_q"], inp["w"], inp["q"], inp["seq_len"], max_len, ws, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if ws.device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    K = args.steps
+    st = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nk + 2)] for _ in range(K)]
+    for e in ev:
+        for x in e:
+            x.record(st)  # materialise the events before handing them to the library
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.15)
+    wall0 = time.perf_counter()
+    for k in range(K):
+        flush.zero_()
+        ev[k][0].record(st)
+        Q.set_profile_events(ev[k][2:])
+        step()
+        ev[k][1].record(st)
+    Q.set_profile_events(None)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    step_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    kern_ms = [[ev[k][2 + 2 * i].elapsed_time(ev[k][3 + 2 * i]) for k in range(K)] for i in range(nk)]
+    mean_ms = float(np.mean(step_ms))
+
+    # ---- end to end through the host-buffer API ----
+    sess = Q.DecodeSession(cache, max_len, device=dev)
+    host_in = Q.DecodeSession.pinned_inputs(inp)
+    for _ in range(3):
+        sess.step(host_in)
+    torch.cuda.synchronize()
+    K2 = max(10, min(K, 500))
+    e2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
+    for k in range(K2):
+        flush.zero_()
+        e2[k][0].record(st)
+        sess.step(host_in)
+        e2[k][1].record(st)
+    torch.cuda.synchronize()
+    e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in e2]))
+    # the device-timed and host-fed results agree bit for bit
+    if not torch.equal(sess.host_out.view(torch.int16), out.cpu().view(torch.int16)):
+        raise RuntimeError("host-fed decode differs from the device-fed one")
+
+    t = torch.tensor([mean_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    mean_ms_max, e2e_ms_max = float(t[0]), float(t[1])
+
+    score_b, gqa_b = algorithmic_bytes(lens)
+    hbm_peak, peak_kind = measured_peaks()
+    score_ms = float(np.mean(kern_ms[1]))
+    src_hash = kernel_src_hash(SCORER_SRC)
+    traffic, traffic_src = committed_traffic(src_hash)
+    res = None
+    if rank == 0:
+        achieved = score_b / (score_ms * 1e-3) / 1e9
+        total_b = score_b + gqa_b
+        res = {
+            "metric": METRIC,
+            "value": round(B * world / (mean_ms_max * 1e-3), 1),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": max(args.warmup, 3),
+            "ms_per_step": round(mean_ms_max, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (qsa_gen seeded generator; N(0,1) bf16 K/V, q, index keys with 5% planted blocks)",
+            "config": {
+                "workload": f"decode_b{B}_ctx120000-131072",
+                "batch_per_gpu": B,
+                "global_batch": B * world,
+                "ctx_min": min(lens), "ctx_max": max(lens), "ctx_mean": round(float(np.mean(lens)), 1),
+                "heads": "16q/2kv d128, indexer 4x128, top-512 of c4 blocks",
+                "page_size": 64,
+                "l2": "inputs 5x larger than L2 per step, plus a 512 MiB flush between timed steps (untimed)",
+                "parallelism": f"replicas x{world} (requests sharded, no exchange)",
+            },
+            "gpu_launches": K * nk,
+            "kernels_ms_mean": {n: round(float(np.mean(v)), 5) for n, v in
+                                zip(["prologue", "score_topk", "sparse_gqa"], kern_ms)},
+            "step_bytes_algorithmic": int(total_b),
+            "step_hbm_gbs": round(total_b / (mean_ms * 1e-3) / 1e9, 1),
+            "step_frac_of_hbm": round(total_b / (mean_ms * 1e-3) / 1e9 / hbm_peak, 4),
+            "roofline": {
+                "kernel": "k_score_topk",
+                "bound": "hbm",
+                "achieved": round(achieved, 1),
+                "peak": hbm_peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else
+                "fallback 6.65 TB/s",
+                "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4),
+                "traffic": None if traffic is None else int(traffic),
+                "traffic_source": traffic_src,
+                "algorithmic_bytes_per_launch": int(score_b),
+                "kernel_src_sha256_16": src_hash,
+            },
+            "e2e": {"value": round(B * world / (e2e_ms_max * 1e-3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": sess.h2d_bytes(), "d2h_bytes_per_step": sess.d2h_bytes()},
+            "clocks": clocks,
+            "wall_s_timed_region": round(wall, 3),
+            "setup_s": round(setup_s, 1),
+        }
+    # free device memory before the CPU baseline
+    del cache, ws, flush, sess
+    torch.cuda.empty_cache()
+    if world > 1:
+        dist.destroy_process_group()
+    return res, wl
+
+
+def oracle_sample_step(wl, reqs, nthreads):
+    """Prepare oracle state for requests `reqs` of a decode workload; return a callable running one
+    decode step of those requests on the CPU oracle, plus its input size."""
+    import oracle as O
+
+    st = {"L": [], "ring": [], "comp": [], "knew": [], "iq": [], "w": [], "q": [], "K": [], "V": []}
+    for r in reqs:
+        L = int(wl.lens[r])
+        raw = wl.idx_keys(r, 0, L)
+        nb0 = (L - 1) // 4
+        comp = np.zeros((max(L // 4, 1), 128), dtype=np.uint16)
+        comp[:nb0] = O.compress(raw[:4 * nb0], nthreads=nthreads)
+        ring = np.zeros((4, 128), dtype=np.uint16)
+        for p in range(4 * nb0, L - 1):
+            ring[p % 4] = raw[p]
+        st["L"].append(L)
+        st["ring"].append(ring)
+        st["comp"].append(comp)
+        st["knew"].append(np.ascontiguousarray(raw[L - 1]))
+        st["iq"].append(wl.idx_q(r)[0])
+        st["w"].append(wl.w(r)[0])
+        st["q"].append(wl.q(r)[0])
+        st["K"].append(wl.k(r, 0, L))
+        st["V"].append(wl.v(r, 0, L))
+
+    def run():
+        O.decode_batch(st["L"], st["ring"], st["comp"], st["knew"], st["iq"], st["w"], st["q"], st["K"], st["V"],
+                       theta=wl.rope_theta, nthreads=nthreads)
+
+    return run
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, seconds: float):
+    nthreads = cpu_threads()
+    n = min(wl.batch, max(nthreads, 8), 32)
+    reqs = list(range(n))
+    run = oracle_sample_step(wl, reqs, nthreads)
+    t0 = time.perf_counter()
+    run()
+    one = time.perf_counter() - t0
+    reps = max(1, int(seconds / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = time.perf_counter() - t0
+    return {"value": round(n * reps / dt, 2), "unit": UNIT, "cores": min(nthreads, n), "kind": "oracle",
+            "sample": f"decode steps of {n} of the {wl.batch} requests (contexts {min(wl.lens[:n])}-"
+                      f"{max(wl.lens[:n])}), {reps} repetitions after one warm-up, FP64 C++ oracle, "
+                      f"one std::thread per request"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    import qsa_gen as G
+
+    wl = G.decode_128k(seed=2, batch=args.batch)
+    nthreads = cpu_threads()
+    n = min(wl.batch, nthreads, 32)
+    run = oracle_sample_step(wl, list(range(n)), nthreads)
+    for _ in range(max(args.warmup, 3)):
+        run()
+    # bound the run: at most ~120 s of timed work whatever --steps says
+    t0 = time.perf_counter()
+    run()
+    one = time.perf_counter() - t0
+    K = max(1, min(args.steps, int(120.0 / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(K):
+        run()
+    dt = time.perf_counter() - t0
+    value = round(n * K / dt, 2)
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(dt / K * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (qsa_gen)", "impl": "reference",
+        "config": {"workload": f"decode_b{wl.batch}_ctx120000-131072", "sample_requests_per_step": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(nthreads, n), "kind": "oracle",
+                         "sample": f"each step: decode of {n} of the {wl.batch} requests on the FP64 C++ oracle"
+                                   f" ({K} steps; --steps {args.steps} bounded to ~120 s)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    res, wl = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

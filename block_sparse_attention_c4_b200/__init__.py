@@ -1,0 +1,305 @@
+"""Python binding of ``libqsa.so``: one Qwen Sparse Attention (c4) layer on B200.
+
+Thin argument marshalling over the C ABI in ``include/qsa.h`` (same names,
+``qsa_`` prefix dropped).  Every step of the layer runs in the library's CUDA
+kernels; PyTorch only provides device memory and the current stream.  There
+is no fallback: if the library is missing or a call fails, an exception says
+so.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa.so")
+
+HEAD_DIM = 128
+INDEX_HEADS = 4
+Q_HEADS = 16
+KV_HEADS = 2
+BLOCK = 4
+TOPK = 512
+MAX_SEL = 2051
+PAGE_SIZE = 64
+MAX_DRAFT = 8
+
+OP_INDEX_SCORE_TOPK, OP_SPARSE_GQA, OP_DECODE, OP_DECODE_INDEXSHARE, OP_COMPRESS_APPEND = 1, 2, 3, 4, 5
+
+DEVERR_BITS = {1: "page", 2: "length", 4: "position", 8: "request", 16: "selection", 32: "timeout"}
+
+
+class QsaError(RuntimeError):
+    pass
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("cidx", ctypes.c_void_p), ("ring", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p), ("num_slots", ctypes.c_int64), ("page_size", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32), ("batch", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("rope_theta", ctypes.c_double),
+    ]
+
+
+_lib = None
+EXPORTS = [
+    "qsa_workspace_bytes", "qsa_workspace_init", "qsa_compress_append", "qsa_index_score_topk",
+    "qsa_expand_indices", "qsa_sparse_gqa", "qsa_decode", "qsa_decode_indexshare", "qsa_device_error",
+    "qsa_set_profile_events", "qsa_decode_kernel_count", "qsa_status_string", "qsa_version",
+]
+
+
+def lib():
+    """Load libqsa.so (building it first if the sources are newer is the caller's job: see build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise QsaError(f"{LIB_PATH} is missing: run `python -m block_sparse_attention_c4_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    cp = ctypes.POINTER(CacheStruct)
+    L.qsa_workspace_bytes.argtypes = [i32, i32, i32]
+    L.qsa_workspace_bytes.restype = sz
+    L.qsa_workspace_init.argtypes = [vp, sz, vp]
+    L.qsa_compress_append.argtypes = [cp, vp, vp, vp, i32, i32, vp]
+    L.qsa_index_score_topk.argtypes = [cp, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
+    L.qsa_expand_indices.argtypes = [vp, vp, vp, i32, vp, vp, vp]
+    L.qsa_sparse_gqa.argtypes = [cp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.qsa_decode.argtypes = [cp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]
+    L.qsa_decode_indexshare.argtypes = [cp, vp, vp, i32, vp, i32, vp, f32, vp, vp, sz, vp]
+    L.qsa_device_error.argtypes = [vp, i32, vp]
+    L.qsa_device_error.restype = i32
+    L.qsa_set_profile_events.argtypes = [ctypes.POINTER(vp), i32]
+    L.qsa_set_profile_events.restype = None
+    L.qsa_decode_kernel_count.restype = i32
+    L.qsa_status_string.argtypes = [ctypes.c_int]
+    L.qsa_status_string.restype = ctypes.c_char_p
+    L.qsa_version.restype = ctypes.c_char_p
+    for name in ("qsa_workspace_init", "qsa_compress_append", "qsa_index_score_topk", "qsa_expand_indices",
+                 "qsa_sparse_gqa", "qsa_decode", "qsa_decode_indexshare"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise QsaError(f"{what} failed: {lib().qsa_status_string(status).decode()} (status {status})")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise QsaError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise QsaError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise QsaError(f"{name} must be contiguous")
+    return t
+
+
+def version() -> str:
+    return lib().qsa_version().decode()
+
+
+def workspace_bytes(op: int, rows: int, max_len: int) -> int:
+    return int(lib().qsa_workspace_bytes(op, rows, max_len))
+
+
+class Workspace:
+    """Caller-owned scratch memory (a torch uint8 CUDA tensor), zeroed once."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self.t = self.buf[off:off + self.nbytes]
+        _check(lib().qsa_workspace_init(_ptr(self.t), self.nbytes, _stream()), "qsa_workspace_init")
+
+    @property
+    def ptr(self):
+        return _ptr(self.t)
+
+    def device_error(self, clear: bool = True) -> int:
+        return int(lib().qsa_device_error(self.ptr, 1 if clear else 0, _stream()))
+
+
+class LayerCache:
+    """The layer's paged cache: raw K/V pool, compressed index keys, ring and page table.
+
+    k, v: bf16 [num_slots, 2, 128]; cidx: bf16 [num_slots/4, 128]; ring: bf16 [batch, 4, 128];
+    page_table: int32 [batch, max_pages].
+    """
+
+    def __init__(self, num_slots: int, batch: int, max_pages: int, rope_theta: float = 1.0e7, device="cuda",
+                 page_table: torch.Tensor | None = None):
+        if num_slots % PAGE_SIZE:
+            raise QsaError("num_slots must be a multiple of 64")
+        self.num_slots, self.batch, self.max_pages, self.rope_theta = num_slots, batch, max_pages, rope_theta
+        self.k = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.cidx = torch.zeros(num_slots // BLOCK, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.ring = torch.zeros(max(batch, 1), BLOCK, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        if page_table is None:
+            page_table = torch.full((max(batch, 1), max_pages), -1, dtype=torch.int32, device=device)
+        self.page_table = _dev(page_table, torch.int32, "page_table")
+
+    def struct(self, batch: int | None = None) -> CacheStruct:
+        return CacheStruct(self.k.data_ptr(), self.v.data_ptr(), self.cidx.data_ptr(), self.ring.data_ptr(),
+                           self.page_table.data_ptr(), self.num_slots, PAGE_SIZE, self.max_pages,
+                           self.batch if batch is None else batch, 0, self.rope_theta)
+
+
+def compress_append(cache: LayerCache, idx_k_new, cu_new, len_before, max_new: int, stream=None):
+    c = cache.struct()
+    total = int(idx_k_new.shape[0]) if idx_k_new is not None else 0
+    if total:
+        _dev(idx_k_new, torch.bfloat16, "idx_k_new")
+    _dev(cu_new, torch.int32, "cu_new")
+    _dev(len_before, torch.int32, "len_before")
+    _check(lib().qsa_compress_append(ctypes.byref(c), _ptr(idx_k_new) if total else None, _ptr(cu_new),
+                                     _ptr(len_before), total, int(max_new), _stream(stream)), "qsa_compress_append")
+
+
+def index_score_topk(cache: LayerCache, idx_q, w, q_req, q_pos, max_len: int, ws: Workspace, blocks=None,
+                     nblocks=None, stream=None):
+    nq = int(q_pos.shape[0])
+    dev = q_pos.device
+    if blocks is None:
+        blocks = torch.full((nq, TOPK), -1, dtype=torch.int32, device=dev)
+    if nblocks is None:
+        nblocks = torch.zeros(nq, dtype=torch.int32, device=dev)
+    c = cache.struct()
+    _check(lib().qsa_index_score_topk(ctypes.byref(c), _ptr(_dev(idx_q, torch.bfloat16, "idx_q")),
+                                      _ptr(_dev(w, torch.float32, "w")), _ptr(_dev(q_req, torch.int32, "q_req")),
+                                      _ptr(_dev(q_pos, torch.int32, "q_pos")), nq, int(max_len), _ptr(blocks),
+                                      _ptr(nblocks), ws.ptr, ws.nbytes, _stream(stream)), "qsa_index_score_topk")
+    return blocks, nblocks
+
+
+def expand_indices(blocks, nblocks, q_pos, pos=None, npos=None, stream=None):
+    nq = int(q_pos.shape[0])
+    dev = q_pos.device
+    if pos is None:
+        pos = torch.full((nq, MAX_SEL), -1, dtype=torch.int32, device=dev)
+    if npos is None:
+        npos = torch.zeros(nq, dtype=torch.int32, device=dev)
+    _check(lib().qsa_expand_indices(_ptr(blocks), _ptr(nblocks), _ptr(q_pos), nq, _ptr(pos), _ptr(npos),
+                                    _stream(stream)), "qsa_expand_indices")
+    return pos, npos
+
+
+def sparse_gqa(cache: LayerCache, q, q_req, pos, npos, max_pos: int, ws: Workspace, scale: float | None = None,
+               out=None, lse=None, stream=None):
+    nq = int(q.shape[0])
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty(nq, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
+    c = cache.struct()
+    _check(lib().qsa_sparse_gqa(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q")),
+                                _ptr(_dev(q_req, torch.int32, "q_req")), _ptr(_dev(pos, torch.int32, "pos")),
+                                _ptr(_dev(npos, torch.int32, "npos")), int(pos.shape[1]), int(max_pos), nq,
+                                float(scale), _ptr(out), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)),
+           "qsa_sparse_gqa")
+    return out
+
+
+def decode(cache: LayerCache, idx_k_new, idx_q, w, q, seq_len, max_len: int, ws: Workspace,
+           scale: float | None = None, out=None, lse=None, blocks_out=None, nblocks_out=None, stream=None):
+    B = cache.batch
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
+    c = cache.struct()
+    _check(lib().qsa_decode(ctypes.byref(c), _ptr(_dev(idx_k_new, torch.bfloat16, "idx_k_new")),
+                            _ptr(_dev(idx_q, torch.bfloat16, "idx_q")), _ptr(_dev(w, torch.float32, "w")),
+                            _ptr(_dev(q, torch.bfloat16, "q")), _ptr(_dev(seq_len, torch.int32, "seq_len")),
+                            int(max_len), float(scale), _ptr(out), _ptr(lse), _ptr(blocks_out), _ptr(nblocks_out),
+                            ws.ptr, ws.nbytes, _stream(stream)), "qsa_decode")
+    return out
+
+
+def decode_indexshare(cache: LayerCache, frozen_pos, frozen_n, len0, q, ws: Workspace, scale: float | None = None,
+                      out=None, stream=None):
+    B, n_plus_1 = int(q.shape[0]), int(q.shape[1])
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty(B, n_plus_1, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
+    c = cache.struct()
+    _check(lib().qsa_decode_indexshare(ctypes.byref(c), _ptr(_dev(frozen_pos, torch.int32, "frozen_pos")),
+                                       _ptr(_dev(frozen_n, torch.int32, "frozen_n")), int(frozen_pos.shape[1]),
+                                       _ptr(_dev(len0, torch.int32, "len0")), n_plus_1,
+                                       _ptr(_dev(q, torch.bfloat16, "q")), float(scale), _ptr(out), ws.ptr,
+                                       ws.nbytes, _stream(stream)), "qsa_decode_indexshare")
+    return out
+
+
+def set_profile_events(events):
+    """events: list of torch.cuda.Event (2 per kernel: start, end), or None to switch off."""
+    if not events:
+        lib().qsa_set_profile_events(None, 0)
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    lib().qsa_set_profile_events(arr, len(events) // 2)
+
+
+def decode_kernel_count() -> int:
+    return int(lib().qsa_decode_kernel_count())
+
+
+class DecodeSession:
+    """Decode steps fed from host memory: the call a serving loop makes once per step.
+
+    step() copies the step's inputs from (pinned) host tensors to device staging buffers, runs
+    qsa_decode, and copies the attention output back to a pinned host tensor, all on one stream.
+    """
+
+    INPUTS = ("idx_k_new", "idx_q", "w", "q", "seq_len")
+
+    def __init__(self, cache: LayerCache, max_len: int, device="cuda"):
+        B = cache.batch
+        self.cache, self.max_len = cache, int(max_len)
+        self.ws = Workspace(workspace_bytes(OP_DECODE, B, self.max_len), device=device)
+        bf = torch.bfloat16
+        self.dev = {
+            "idx_k_new": torch.empty(B, HEAD_DIM, dtype=bf, device=device),
+            "idx_q": torch.empty(B, INDEX_HEADS, HEAD_DIM, dtype=bf, device=device),
+            "w": torch.empty(B, INDEX_HEADS, dtype=torch.float32, device=device),
+            "q": torch.empty(B, Q_HEADS, HEAD_DIM, dtype=bf, device=device),
+            "seq_len": torch.empty(B, dtype=torch.int32, device=device),
+        }
+        self.out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=bf, device=device)
+        self.host_out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=bf, pin_memory=True)
+
+    @staticmethod
+    def pinned_inputs(device_inputs: dict) -> dict:
+        return {k: device_inputs[k].cpu().pin_memory() for k in DecodeSession.INPUTS}
+
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self.dev.values())
+
+    def d2h_bytes(self) -> int:
+        return self.host_out.numel() * self.host_out.element_size()
+
+    def step(self, host_inputs: dict, stream=None) -> torch.Tensor:
+        for k, t in self.dev.items():
+            t.copy_(host_inputs[k], non_blocking=True)
+        decode(self.cache, self.dev["idx_k_new"], self.dev["idx_q"], self.dev["w"], self.dev["q"],
+               self.dev["seq_len"], self.max_len, self.ws, out=self.out, stream=stream)
+        self.host_out.copy_(self.out, non_blocking=True)
+        return self.host_out

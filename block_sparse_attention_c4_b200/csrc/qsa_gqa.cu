@@ -1,0 +1,363 @@
+// Sparse GQA over the raw paged K/V at the kept positions (decode, IndexShare
+// draft steps, explicit position lists).
+//
+// Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
+// (SGLang day-0 blog for Qwen3.8-Flash-Next): the compressed keys are only an
+// index; the softmax and the value sum use the original, uncompressed K/V at
+// the (at most 2051) selected positions.  Section "IndexShare MTP: Reusing the
+// QSA Selection Across Draft Steps": draft query i also sees the positions
+// drafted since the capture, up to its own.
+//
+// Design (B200): one CTA covers every query head of a row (16 heads x up to 8
+// queries sharing one position list) for a contiguous range of positions
+// (split-K), so each K/V row crosses HBM once.  16-position tiles of K and V
+// (both KV heads, 1 KiB per position) are gathered with 16-byte cp.async
+// into a 4-deep, XOR-swizzled shared-memory ring.  Warp (g, d-half, m-tile):
+// S = Q_g K_g^T with m16n8k16 bf16 MMAs (rows = query heads of KV group g),
+// an online softmax in the log2 domain, and O += P V_g for its 64 output
+// dims.  Splits write (O, m, l) partials; the last CTA of the row (atomic
+// ticket, no waiting) merges them.
+#include "qsa_common.cuh"
+#include "qsa_kernels.h"
+
+namespace qsa {
+
+constexpr int GQ_TILE = 16;
+constexpr int GQ_STAGES = 4;
+constexpr int GQ_ROW_BYTES = D * 2;                             // 256 B: one head of one position
+constexpr int GQ_KV_BYTES = GQ_TILE * HKV * GQ_ROW_BYTES;       // 8 KiB: K (or V) of a tile
+constexpr int GQ_STAGE_BYTES = 2 * GQ_KV_BYTES;                 // 16 KiB
+
+template <int MT>
+struct GqaSmem {
+  alignas(128) uint8_t q[HKV][MT * 16][GQ_ROW_BYTES];
+  alignas(128) uint8_t kv[GQ_STAGES][GQ_STAGE_BYTES];  // [K|V][group][pos][256 B], swizzled
+  float ml[HKV][MT * 16][2];
+  int is_last;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(((chunk ^ (row & 7)) << 4)); }
+
+template <int MT>
+__global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
+  constexpr int THREADS = MT * 128;
+  extern __shared__ uint8_t smem_raw[];
+  GqaSmem<MT>& S = *reinterpret_cast<GqaSmem<MT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int row = blockIdx.y, split = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nq = p.nq_row;
+  const int req = p.row_req ? __ldg(p.row_req + row) : row;
+  bool bad = req < 0 || req >= p.c.batch;
+  if (bad && split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_REQUEST);
+
+  // ---- the row's position list ----
+  int nbase = 0, nsel4 = 0, tail0 = 0;
+  const int32_t* sel = nullptr;
+  const int32_t* list = nullptr;
+  if (!bad) {
+    if (p.mode == 0) {
+      const int L = __ldg(p.row_len + row) + p.len_offset;
+      const int nsel = __ldg(p.sel_n + row);
+      if (L < 1 || L > p.max_len || nsel < 0 || nsel > TOPK || nsel > (L >> 2)) {
+        if (split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_SELECTION);
+        bad = true;
+      } else {
+        sel = p.sel + (int64_t)row * TOPK;
+        nsel4 = 4 * nsel;
+        tail0 = (L >> 2) << 2;
+        nbase = nsel4 + (L & 3);
+      }
+    } else {
+      const int n = __ldg(p.list_n + row);
+      if (n < 0 || n > p.list_stride) {
+        if (split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_SELECTION);
+        bad = true;
+      } else {
+        list = p.list + (int64_t)row * p.list_stride;
+        nbase = n;
+      }
+    }
+  }
+  const int ext0 = (!bad && p.extra_base) ? __ldg(p.extra_base + row) : 0;
+  const int ntot = bad ? 0 : nbase + (p.extra_base ? p.n_extra : 0);
+  const int tiles = ceil_div(ntot, GQ_TILE);
+  const int tps = ceil_div(tiles, p.splits);
+  const int t_begin = min(tiles, split * tps), t_end = min(tiles, t_begin + tps);
+  const int ntl = t_end - t_begin;
+
+  auto position = [&](int j) -> int {
+    if (j < nbase) {
+      if (list) return __ldg(list + j);
+      return j < nsel4 ? __ldg(sel + (j >> 2)) * CBLK + (j & 3) : tail0 + (j - nsel4);
+    }
+    return ext0 + (j - nbase);
+  };
+
+  // ---- load the queries of both KV groups: row rho = query*8 + head-in-group ----
+  {
+    const __nv_bfloat16* qrow = p.q + (int64_t)row * nq * HQ * D;
+    constexpr int CHUNKS = HKV * MT * 16 * (GQ_ROW_BYTES / 16);
+    for (int c = tid; c < CHUNKS; c += THREADS) {
+      const int g = c / (MT * 16 * 16);
+      const int rho = (c / 16) % (MT * 16);
+      const int ch = c % 16;
+      const int qi = rho >> 3, h = g * GROUP + (rho & 7);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (qi < nq) v = __ldg(reinterpret_cast<const uint4*>(qrow + ((int64_t)qi * HQ + h) * D) + ch);
+      *reinterpret_cast<uint4*>(&S.q[g][rho][swz(rho, ch)]) = v;
+    }
+  }
+
+  // ---- async gather of one tile into a stage ----
+  // chunk id c in [0, 1024): kv = c >> 9, pos j = (c >> 5) & 15, group = (c >> 4) & 1, 16 B chunk = c & 15
+  auto issue_tile = [&](int t, int stage) {
+    uint8_t* dst0 = S.kv[stage];
+    constexpr int PER = 1024 / THREADS;  // chunks per thread
+    constexpr int POS_PER = 512 / THREADS > 0 ? 512 / THREADS : 1;
+    int64_t slot[(PER + 1) / 2 > 0 ? (PER + 1) / 2 : 1];
+#pragma unroll
+    for (int k = 0; k < (PER + 1) / 2; ++k) {
+      const int c = tid + k * THREADS;
+      const int j = (c >> 5) & 15;
+      const int jj = t * GQ_TILE + j;
+      slot[k] = jj < ntot ? slot_of(p.c, req, position(jj), p.err) : -1;
+    }
+    (void)POS_PER;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      const int c = tid + k * THREADS;
+      const int kvsel = c >> 9, j = (c >> 5) & 15, g = (c >> 4) & 1, ch = c & 15;
+      const int64_t sl = slot[k % ((PER + 1) / 2)];
+      const __nv_bfloat16* base = kvsel ? p.c.v : p.c.k;
+      const __nv_bfloat16* src = sl >= 0 ? base + (sl * HKV + g) * D + ch * 8 : base;
+      uint8_t* dst = dst0 + kvsel * GQ_KV_BYTES + g * (GQ_TILE * GQ_ROW_BYTES) + j * GQ_ROW_BYTES + swz(j, ch);
+      cp_async_16(dst, src, sl >= 0 ? 16 : 0);
+    }
+  };
+
+  // prologue of the pipeline
+#pragma unroll
+  for (int k = 0; k < GQ_STAGES - 1; ++k) {
+    if (k < ntl) issue_tile(t_begin + k, k);
+    cp_async_commit();
+  }
+  __syncthreads();  // queries in shared memory
+
+  // ---- warp role and its query fragments ----
+  const int g = warp & 1, dh = (warp >> 1) & 1, mt = warp >> 2;
+  const int gq = lane >> 2, cq = lane & 3;
+  uint32_t qa[8][4];
+  {
+    const int mtx = lane >> 3;
+    const int rho = mt * 16 + (lane & 7) + ((mtx & 1) << 3);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      ldmatrix_x4(qa[j][0], qa[j][1], qa[j][2], qa[j][3], smem_u32(&S.q[g][rho][swz(rho, 2 * j + (mtx >> 1))]));
+  }
+  const int qi0 = (mt * 16 + gq) >> 3, qi1 = (mt * 16 + gq + 8) >> 3;  // query of rows gq, gq+8
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[8][4];
+#pragma unroll
+  for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+  for (int it = 0; it < ntl; ++it) {
+    cp_async_wait<GQ_STAGES - 2>();
+    __syncthreads();
+    if (it + GQ_STAGES - 1 < ntl) issue_tile(t_begin + it + GQ_STAGES - 1, (it + GQ_STAGES - 1) % GQ_STAGES);
+    cp_async_commit();
+
+    const int stage = it % GQ_STAGES;
+    const int t = t_begin + it;
+    const uint8_t* kbase = S.kv[stage] + g * (GQ_TILE * GQ_ROW_BYTES);
+    const uint8_t* vbase = S.kv[stage] + GQ_KV_BYTES + g * (GQ_TILE * GQ_ROW_BYTES);
+
+    // S = Q K^T : 16 rows x 16 positions
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int mtx = lane >> 3;
+      const int pj = (lane & 7) + ((mtx >> 1) << 3);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(b0, b1, b2, b3, smem_u32(kbase + pj * GQ_ROW_BYTES + swz(pj, 2 * j + (mtx & 1))));
+        mma_bf16_16816(s[0], qa[j], b0, b1);
+        mma_bf16_16816(s[1], qa[j], b2, b3);
+      }
+    }
+    // mask, scale (log2 domain), online softmax
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int jj = t * GQ_TILE + 8 * n + 2 * cq + e;
+        const int ex = jj - nbase;  // >= 0: a drafted position, seen by queries ex..
+        const bool ok0 = jj < ntot && (ex < 0 || ex <= qi0);
+        const bool ok1 = jj < ntot && (ex < 0 || ex <= qi1);
+        s[n][e] = ok0 ? s[n][e] * p.scale_log2 : -INFINITY;
+        s[n][2 + e] = ok1 ? s[n][2 + e] * p.scale_log2 : -INFINITY;
+        mx0 = fmaxf(mx0, s[n][e]);
+        mx1 = fmaxf(mx1, s[n][2 + e]);
+      }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float base0 = mn0 == -INFINITY ? 0.f : mn0, base1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float c0 = exp2f(m0 - base0), c1 = exp2f(m1 - base1);
+    m0 = mn0;
+    m1 = mn1;
+    float pr[2][4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+      pr[n][0] = exp2f(s[n][0] - base0);
+      pr[n][1] = exp2f(s[n][1] - base0);
+      pr[n][2] = exp2f(s[n][2] - base1);
+      pr[n][3] = exp2f(s[n][3] - base1);
+    }
+    l0 = l0 * c0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
+    l1 = l1 * c1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      o[n][0] *= c0;
+      o[n][1] *= c0;
+      o[n][2] *= c1;
+      o[n][3] *= c1;
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+    pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+    pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+    pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+    // O += P V over this warp's 64 dims
+    {
+      const int mtx = lane >> 3;
+      const int pj = (lane & 7) + ((mtx & 1) << 3);
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) {
+        const int ch = (dh * 64 + pp * 16) / 8 + (mtx >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(vbase + pj * GQ_ROW_BYTES + swz(pj, ch)));
+        mma_bf16_16816(o[2 * pp], pa, b0, b1);
+        mma_bf16_16816(o[2 * pp + 1], pa, b2, b3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  // ---- finish: full row sums, then write the result or a partial ----
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  const int rho0 = mt * 16 + gq, rho1 = rho0 + 8;
+  const int h0 = g * GROUP + (rho0 & 7), h1 = g * GROUP + (rho1 & 7);
+  const int nh = nq * HQ;
+  if (p.splits == 1) {
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    __nv_bfloat16* out = p.out + (int64_t)row * nh * D;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int d = dh * 64 + 8 * n + 2 * cq;
+      if (qi0 < nq)
+        *reinterpret_cast<uint32_t*>(out + ((int64_t)qi0 * HQ + h0) * D + d) = pack_bf16x2(o[n][0] * i0, o[n][1] * i0);
+      if (qi1 < nq)
+        *reinterpret_cast<uint32_t*>(out + ((int64_t)qi1 * HQ + h1) * D + d) = pack_bf16x2(o[n][2] * i1, o[n][3] * i1);
+    }
+    if (p.lse && dh == 0 && cq == 0) {
+      constexpr float LN2 = 0.69314718055994530942f;
+      if (qi0 < nq) p.lse[(int64_t)row * nh + qi0 * HQ + h0] = l0 > 0.f ? (m0 + log2f(l0)) * LN2 : -INFINITY;
+      if (qi1 < nq) p.lse[(int64_t)row * nh + qi1 * HQ + h1] = l1 > 0.f ? (m1 + log2f(l1)) * LN2 : -INFINITY;
+    }
+    return;
+  }
+  float* po = p.part_o + ((int64_t)row * p.splits + split) * nh * D;
+  float* pml = p.part_ml + ((int64_t)row * p.splits + split) * nh * 2;
+#pragma unroll
+  for (int n = 0; n < 8; ++n) {
+    const int d = dh * 64 + 8 * n + 2 * cq;
+    if (qi0 < nq) *reinterpret_cast<float2*>(po + ((int64_t)qi0 * HQ + h0) * D + d) = make_float2(o[n][0], o[n][1]);
+    if (qi1 < nq) *reinterpret_cast<float2*>(po + ((int64_t)qi1 * HQ + h1) * D + d) = make_float2(o[n][2], o[n][3]);
+  }
+  if (dh == 0 && cq == 0) {
+    if (qi0 < nq) *reinterpret_cast<float2*>(pml + (qi0 * HQ + h0) * 2) = make_float2(m0, l0);
+    if (qi1 < nq) *reinterpret_cast<float2*>(pml + (qi1 * HQ + h1) * 2) = make_float2(m1, l1);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) S.is_last = atomicAdd(p.counters + row, 1) == p.splits - 1;
+  __syncthreads();
+  if (!S.is_last) return;
+  __threadfence();
+  // merge: thread handles (head, 4-dim group)
+  const float* pob = p.part_o + (int64_t)row * p.splits * nh * D;
+  const float* pmb = p.part_ml + (int64_t)row * p.splits * nh * 2;
+  __nv_bfloat16* out = p.out + (int64_t)row * nh * D;
+  for (int idx = tid; idx < nh * (D / 4); idx += THREADS) {
+    const int hh = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < p.splits; ++s2) M = fmaxf(M, __ldcg(pmb + ((int64_t)s2 * nh + hh) * 2));
+    const float base = M == -INFINITY ? 0.f : M;
+    float den = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int s2 = 0; s2 < p.splits; ++s2) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(pmb + ((int64_t)s2 * nh + hh) * 2));
+      const float f = exp2f(ml.x - base);
+      den += f * ml.y;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(pob + ((int64_t)s2 * nh + hh) * D + d4));
+      a0 += f * v.x;
+      a1 += f * v.y;
+      a2 += f * v.z;
+      a3 += f * v.w;
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint2 pk;
+    pk.x = pack_bf16x2(a0 * inv, a1 * inv);
+    pk.y = pack_bf16x2(a2 * inv, a3 * inv);
+    *reinterpret_cast<uint2*>(out + (int64_t)hh * D + d4) = pk;
+    if (p.lse && d4 == 0) {
+      constexpr float LN2 = 0.69314718055994530942f;
+      p.lse[(int64_t)row * nh + hh] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+    }
+  }
+  if (tid == 0) p.counters[row] = 0;
+}
+
+int gqa_splits_for(int rows, int max_pos, int nq_row, int num_sms) {
+  const int tiles = ceil_div(max_pos, GQ_TILE);
+  // aim for ~3 resident CTAs per SM over the whole grid, at least 2 tiles per split
+  int s = ceil_div(3 * num_sms, rows > 0 ? rows : 1);
+  s = min(s, max(1, tiles / 2));
+  s = max(1, min(s, GQ_MAX_SPLITS));
+  (void)nq_row;
+  return s;
+}
+
+template <int MT>
+static cudaError_t launch_mt(const GqaParams& p, int rows, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const size_t smem = sizeof(GqaSmem<MT>) + 128;
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(p.splits, rows);
+  k_sparse_gqa<MT><<<grid, MT * 128, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gqa(const GqaParams& p, int rows, cudaStream_t st) {
+  const int mt = ceil_div(p.nq_row * GROUP, 16);
+  switch (mt) {
+    case 1: return launch_mt<1>(p, rows, st);
+    case 2: return launch_mt<2>(p, rows, st);
+    case 3:
+    case 4: return launch_mt<4>(p, rows, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qsa

@@ -1,0 +1,258 @@
+/*
+ * qsa.h -- C ABI of a B200 (sm_100a) implementation of one Qwen Sparse
+ * Attention layer with compression ratio 4 (QSA c4).
+ *
+ * The method is the one the SGLang day-0 blog for Qwen3.8-Flash-Next describes
+ * in its sections "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
+ * and "IndexShare MTP: Reusing the QSA Selection Across Draft Steps":
+ *
+ *   indexer  every 4 raw 128-d index keys -> one compressed key (FP32 mean,
+ *            L2-normalised, RoPE-rotated at the block's first position, BF16);
+ *            the raw keys of an unfinished block wait in a 4-slot ring;
+ *            a query's 4 index heads score every complete block,
+ *            score_b = sum_h w_h * max(0, q~_h . k^_b), and the best 512 blocks
+ *            are kept (ties: lower block index first);
+ *   expand   512 blocks -> 2048 token positions, plus the 0..3 tokens of the
+ *            unfinished block: at most 2051 positions;
+ *   attend   GQA (16 query heads, 2 KV heads, d = 128) over the raw, paged BF16
+ *            K/V at exactly those positions.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates nothing, never synchronises the stream (except
+ *     qsa_device_error, which says so) and only enqueues work on `stream`
+ *     (a cudaStream_t; NULL = the legacy default stream).
+ *   - bf16 tensors are passed as void* holding IEEE bfloat16 values.
+ *   - Row-major layouts; shapes are given in brackets, innermost last.
+ *   - Host-checkable errors (null pointers, bad sizes, a workspace that is too
+ *     small, unsupported shapes) return an error status before anything is
+ *     enqueued.  Data-dependent errors found on the device (a page id outside
+ *     the pool, a length beyond the stated maximum, a position past the pages
+ *     of its request) set bits of the device error word in the workspace and
+ *     the offending rows are skipped; read it with qsa_device_error.
+ *   - Positions are logical token indices of a request.  Logical position p of
+ *     request r lives in physical slot page_table[r][p / 64] * 64 + p % 64.
+ *   - Lengths: L is a context length INCLUDING the query token, whose position
+ *     is L - 1.  A query sees floor(L/4) complete blocks and L mod 4 tail tokens.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QSA_HEAD_DIM 128    /* dims of every index head and attention head       */
+#define QSA_INDEX_HEADS 4   /* index query heads (one shared index key head)     */
+#define QSA_Q_HEADS 16      /* attention query heads                              */
+#define QSA_KV_HEADS 2      /* attention KV heads; head h reads KV head h / 8    */
+#define QSA_BLOCK 4         /* compression ratio c4                              */
+#define QSA_TOPK 512        /* kept blocks                                        */
+#define QSA_MAX_SEL 2051    /* 512 * 4 + 3 positions                              */
+#define QSA_PAGE_SIZE 64    /* tokens per K/V page (16 compressed entries)        */
+#define QSA_MAX_DRAFT 8     /* largest n_plus_1 of qsa_decode_indexshare          */
+#define QSA_MAX_CONTEXT (1 << 24) /* largest context length accepted              */
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size          */
+  QSA_ERR_UNSUPPORTED = 2, /* shape or configuration this build does not handle   */
+  QSA_ERR_WORKSPACE = 3,   /* workspace null, misaligned or smaller than required */
+  QSA_ERR_CUDA = 4         /* a CUDA launch or driver call failed                 */
+} qsa_status;
+
+/* Device error word bits (qsa_device_error). */
+#define QSA_DEVERR_PAGE 1       /* page id outside [0, num_slots / 64)           */
+#define QSA_DEVERR_LENGTH 2     /* length < 1, beyond max_len or past the pages  */
+#define QSA_DEVERR_POSITION 4   /* an explicit position outside its request      */
+#define QSA_DEVERR_REQUEST 8    /* a request index outside [0, batch)            */
+#define QSA_DEVERR_SELECTION 16 /* a selection count outside [0, 512]            */
+#define QSA_DEVERR_TIMEOUT 32   /* a bounded wait inside a kernel gave up        */
+
+/*
+ * The layer's cache.  All pointers are device pointers owned by the caller.
+ *   k, v        bf16 [num_slots][2][128]  raw attention keys / values (paged pool)
+ *   cidx        bf16 [num_slots / 4][128] compressed index keys; block b of request r
+ *               lives at entry (page_table[r][4b / 64] * 64 + 4b % 64) / 4, so one
+ *               page's 16 entries are contiguous (page-aligned full_slot / 4 rule)
+ *   ring        bf16 [batch][4][128]      raw index keys of each request's
+ *               unfinished block, slot = position mod 4
+ *   page_table  int32 [batch][max_pages]  physical page of each logical page
+ *   num_slots   multiple of page_size; page_size must be 64
+ *   rope_theta  RoPE base of the index keys/queries (1e7 for the workloads here)
+ * Alignment: k, v, cidx, ring 16-byte aligned; page_table 4-byte aligned.
+ */
+typedef struct {
+  void* k;
+  void* v;
+  void* cidx;
+  void* ring;
+  const int32_t* page_table;
+  int64_t num_slots;
+  int32_t page_size;
+  int32_t max_pages;
+  int32_t batch;
+  int32_t reserved;
+  double rope_theta;
+} qsa_cache;
+
+/* Operation ids for qsa_workspace_bytes. */
+typedef enum {
+  QSA_OP_INDEX_SCORE_TOPK = 1,
+  QSA_OP_SPARSE_GQA = 2,
+  QSA_OP_DECODE = 3,
+  QSA_OP_DECODE_INDEXSHARE = 4,
+  QSA_OP_COMPRESS_APPEND = 5
+} qsa_op;
+
+/*
+ * Workspace bytes an operation needs for `rows` rows (queries for
+ * QSA_OP_INDEX_SCORE_TOPK / QSA_OP_SPARSE_GQA, requests for the decode ops)
+ * whose contexts are at most `max_len` tokens (for QSA_OP_SPARSE_GQA:
+ * positions per query; for QSA_OP_DECODE_INDEXSHARE pass the capture length
+ * L0).  Returns 0 for invalid arguments.  The workspace must be 256-byte
+ * aligned and must be zeroed once with qsa_workspace_init before its first
+ * use; the kernels leave it ready for the next call.  Calls that share one
+ * workspace must be ordered on the GPU (same stream or synchronised).
+ */
+size_t qsa_workspace_bytes(int32_t op, int32_t rows, int32_t max_len);
+
+/* Zero a workspace (enqueued on `stream`). */
+qsa_status qsa_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Append new raw index keys to the cache (prefill / chunked prefill / decode).
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely":
+ * each group of 4 raw index keys becomes one compressed key (FP32 mean,
+ * normalised, rotated at its first token's position, stored BF16); the keys
+ * of the unfinished block wait in the 4-slot ring.
+ *   idx_k_new   bf16 [total_new][128]  raw index keys, request r's keys in rows
+ *               cu_new[r] .. cu_new[r+1]-1, at positions len_before[r] + j
+ *   cu_new      int32 [batch + 1]      prefix offsets (device)
+ *   len_before  int32 [batch]          tokens already appended per request (device)
+ *   max_new     upper bound of cu_new[r+1]-cu_new[r] over r (host), >= 0
+ * Completed blocks are written to cidx; the ring ends up holding the keys of
+ * each request's unfinished block (slots of positions past the last appended
+ * token keep whatever they held).  Appending a prefix in one call, token by
+ * token, or in chunks gives bit-identical caches.
+ */
+qsa_status qsa_compress_append(const qsa_cache* cache, const void* idx_k_new, const int32_t* cu_new,
+                               const int32_t* len_before, int32_t total_new, int32_t max_new, void* stream);
+
+/*
+ * Score the visible compressed blocks of each query and keep the top 512.
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
+ * (score formula as stated in this header's preamble; the text's own formula
+ * is lost).  Query i belongs to request q_req[i] and sits at position
+ * q_pos[i]; it scores blocks b < floor((q_pos[i]+1)/4).
+ *   idx_q     bf16 [nq][4][128]  unrotated index queries (rotated here at q_pos)
+ *   w         f32  [nq][4]       per-query head weights
+ *   q_req     int32 [nq], q_pos int32 [nq]   (device)
+ *   max_len   host bound of q_pos[i] + 1
+ *   blocks    int32 [nq][512]  out: kept block ids, ascending; unused tail untouched
+ *   nblocks   int32 [nq]       out: min(512, floor((q_pos+1)/4))
+ *   ws        workspace of qsa_workspace_bytes(QSA_OP_INDEX_SCORE_TOPK, nq, max_len)
+ */
+qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, const int32_t* q_req,
+                                const int32_t* q_pos, int32_t nq, int32_t max_len, int32_t* blocks,
+                                int32_t* nblocks, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Expand kept blocks to token positions: block b -> 4b..4b+3 in block order,
+ * then the tail 4*floor(L/4) .. L-1 with L = q_pos[i] + 1.
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely".
+ *   blocks  int32 [nq][512], nblocks int32 [nq], q_pos int32 [nq] (device)
+ *   pos     int32 [nq][2051] out, npos int32 [nq] out (= 4*nblocks + L mod 4)
+ */
+qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, const int32_t* q_pos, int32_t nq,
+                              int32_t* pos, int32_t* npos, void* stream);
+
+/*
+ * Sparse GQA of nq query tokens, each over its own list of positions.
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely":
+ * softmax and value sum run over the raw, uncompressed K/V of the cache.
+ *   q        bf16 [nq][16][128]
+ *   q_req    int32 [nq] request of each query (device)
+ *   pos      int32 [nq][pos_stride] positions (device); npos int32 [nq]
+ *   max_pos  host bound of npos[i] (<= pos_stride)
+ *   scale    softmax scale (1/sqrt(128) for the layer)
+ *   out      bf16 [nq][16][128] out; lse f32 [nq][16] out (natural log) or NULL
+ *   ws       workspace of qsa_workspace_bytes(QSA_OP_SPARSE_GQA, nq, max_pos)
+ * A query with no positions gets zeros (lse = -inf).
+ */
+qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* q_req, const int32_t* pos,
+                          const int32_t* npos, int32_t pos_stride, int32_t max_pos, int32_t nq, float scale,
+                          void* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One decode step of the whole layer for every request of the cache:
+ * append the new index key (ring; compress when it completes a block), rotate
+ * the index query at seq_len[r]-1, score the complete blocks, keep the top
+ * 512, and attend over the kept positions plus the tail.
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely".
+ *   idx_k_new  bf16 [batch][128]     index key of each request's new token
+ *   idx_q      bf16 [batch][4][128]  unrotated index queries
+ *   w          f32  [batch][4]       index head weights
+ *   q          bf16 [batch][16][128] attention queries
+ *   seq_len    int32 [batch] context length including the new token (device);
+ *              the new token's K/V must already be in the pool
+ *   max_len    host bound of seq_len
+ *   out        bf16 [batch][16][128] out; lse f32 [batch][16] out or NULL
+ *   blocks_out int32 [batch][512], nblocks_out int32 [batch]: the kept blocks
+ *              (out, may both be NULL; IndexShare captures them from here)
+ *   ws         workspace of qsa_workspace_bytes(QSA_OP_DECODE, batch, max_len)
+ * Calling it twice with the same inputs gives the same result (the append is
+ * idempotent).
+ */
+qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
+                      const void* q, const int32_t* seq_len, int32_t max_len, float scale, void* out, float* lse,
+                      int32_t* blocks_out, int32_t* nblocks_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * IndexShare draft step: attention only, the indexer is skipped.
+ * Blog section "IndexShare MTP: Reusing the QSA Selection Across Draft Steps":
+ * the selection captured at the last accepted token (position len0[r]-1) is
+ * frozen; draft query i (i = 0 .. n_plus_1-1, position len0[r]+i) attends to
+ * the frozen positions plus the drafted positions len0[r] .. len0[r]+i.
+ *   frozen_pos  int32 [batch][frozen_stride] frozen positions (e.g. from
+ *               qsa_expand_indices on qsa_decode's blocks_out), all < len0[r]
+ *   frozen_n    int32 [batch]
+ *   len0        int32 [batch] context length at capture (device)
+ *   n_plus_1    drafted positions per request, 1 .. QSA_MAX_DRAFT (host)
+ *   q           bf16 [batch][n_plus_1][16][128]
+ *   out         bf16 [batch][n_plus_1][16][128] out
+ *   ws          workspace of qsa_workspace_bytes(QSA_OP_DECODE_INDEXSHARE, batch, max_len0)
+ */
+qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_pos, const int32_t* frozen_n,
+                                 int32_t frozen_stride, const int32_t* len0, int32_t n_plus_1, const void* q,
+                                 float scale, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Read (and optionally clear) the device error word of a workspace.  This
+ * call synchronises `stream`.  Returns the QSA_DEVERR_* bits, or -1 if the
+ * copy failed.
+ */
+int32_t qsa_device_error(void* ws, int32_t clear, void* stream);
+
+/*
+ * Measurement hook: when `events` is non-NULL, qsa_decode records
+ * events[2*i] before and events[2*i+1] after its i-th kernel (i < n_pairs)
+ * on its stream.  Each entry is a cudaEvent_t.  Pass NULL to switch it off.
+ * Not thread-safe with concurrent qsa_decode calls from several host threads.
+ */
+void qsa_set_profile_events(void* const* events, int32_t n_pairs);
+
+/* Number of kernels qsa_decode launches per call. */
+int32_t qsa_decode_kernel_count(void);
+
+const char* qsa_status_string(qsa_status s);
+const char* qsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H */
