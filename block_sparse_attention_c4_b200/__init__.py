@@ -71,6 +71,8 @@ def lib():
     L.qsa_sparse_gqa.argtypes = [cp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.qsa_decode.argtypes = [cp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]
     L.qsa_decode_indexshare.argtypes = [cp, vp, vp, i32, vp, i32, vp, f32, vp, vp, sz, vp]
+    L.qsa_sparse_gqa_noalloc.argtypes = [cp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp]
+    L.qsa_sparse_gqa_noalloc.restype = ctypes.c_int
     L.qsa_device_error.argtypes = [vp, i32, vp]
     L.qsa_device_error.restype = i32
     L.qsa_set_profile_events.argtypes = [ctypes.POINTER(vp), i32]
@@ -216,6 +218,25 @@ def sparse_gqa(cache: LayerCache, q, q_req, pos, npos, max_pos: int, ws: Workspa
                                 _ptr(_dev(npos, torch.int32, "npos")), int(pos.shape[1]), int(max_pos), nq,
                                 float(scale), _ptr(out), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)),
            "qsa_sparse_gqa")
+    return out
+
+
+def sparse_gqa_noalloc(cache: LayerCache, q, q_req, pos, npos, max_pos: int, scale: float | None = None,
+                       out=None, lse=None, stream=None):
+    """qsa_sparse_gqa without a workspace, for callers that cannot allocate device memory (a plugin that
+    is handed only its input and output buffers, code running during CUDA-graph capture, a fixed
+    device-memory budget).  Scratch is the library's own static device array (about 4.1 MiB per GPU);
+    nq is limited to 4096; calls that overlap on the GPU share that array and race."""
+    nq = int(q.shape[0])
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty(nq, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
+    c = cache.struct()
+    _check(lib().qsa_sparse_gqa_noalloc(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q")),
+                                        _ptr(_dev(q_req, torch.int32, "q_req")), _ptr(_dev(pos, torch.int32, "pos")),
+                                        _ptr(_dev(npos, torch.int32, "npos")), int(pos.shape[1]), int(max_pos), nq,
+                                        float(scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "qsa_sparse_gqa_noalloc")
     return out
 
 

@@ -231,6 +231,39 @@ qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_p
                                  float scale, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Sparse GQA without a workspace: the same computation as qsa_sparse_gqa
+ * (same arguments minus ws / ws_bytes), for callers that cannot allocate
+ * device memory or pass the library scratch space -- e.g. a plugin whose host
+ * hands it only input and output buffers, code running during CUDA-graph
+ * capture where cudaMalloc is not allowed, or a deployment whose device memory
+ * is fixed at start-up.  The QSA description has no counterpart: this is an
+ * interface convenience of this library, not a step of the method.
+ *   Scratch: a file-scope device array of QSA_NOALLOC_SCRATCH_BYTES (about
+ *   4.1 MiB) that every GPU which loads the library keeps until the process
+ *   exits.  It holds split-K partials for at most QSA_NOALLOC_ROW_SPLITS
+ *   (query, split) pairs, so fewer splits are used for large nq.
+ *   Limit: nq <= QSA_NOALLOC_MAX_QUERIES, else QSA_ERR_UNSUPPORTED is returned
+ *   before anything is enqueued.
+ *   The entry point allocates nothing (no cudaMalloc / cudaFree, no allocating
+ *   library call).  Its first call on a device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.  Each call zeroes the arrival counters it
+ *   uses (cudaMemsetAsync on `stream`).
+ *   All calls share the one array, which keeps the last call's contents: calls
+ *   that overlap on the GPU (different streams, no ordering) race and give
+ *   wrong results.  Device-side data errors are not reported (there is no
+ *   error word): positions outside their request are skipped.
+ */
+#define QSA_NOALLOC_MAX_QUERIES 4096
+#define QSA_NOALLOC_ROW_SPLITS 512
+#define QSA_NOALLOC_SCRATCH_BYTES                                          \
+  (256 + 4 * QSA_NOALLOC_MAX_QUERIES + 4 * QSA_NOALLOC_ROW_SPLITS * 16 * 2 + \
+   4 * QSA_NOALLOC_ROW_SPLITS * 16 * 128)
+qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void* q, const int32_t* q_req, const int32_t* pos,
+                                  const int32_t* npos, int32_t pos_stride, int32_t max_pos, int32_t nq, float scale,
+                                  void* out, float* lse, void* stream);
+
+/*
  * Read (and optionally clear) the device error word of a workspace.  This
  * call synchronises `stream`.  Returns the QSA_DEVERR_* bits, or -1 if the
  * copy failed.
