@@ -22,11 +22,26 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t cnt_score = 0, cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, cand_key = 0, cand_id = 0, part_o = 0,
-         part_ml = 0, total = 0;
-  int max_chunks_bound = 0;
+  size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, seg_cnt = 0, cand_cnt = 0,
+         pages_done = 0, seg_tab = 0, cand_key = 0, cand_id = 0, part_o = 0, part_ml = 0, total = 0;
+  int ppc_min = 0;
+  int seg_cap = 0;
   int splits_bound = 0;
 };
+
+constexpr size_t WS_ERR = 0;     // int: device error word
+constexpr size_t WS_TICKET = 64;  // int: prologue arrival ticket
+
+// Scorer range sizing from the longest context: ranges of at least ppc_min
+// pages keep the segments of one row at or below seg_cap (16 up to ~1.8M
+// tokens, so a row's candidates fit the merge buffer in shared memory).
+// A row of np pages meets at most ceil(np / ppc) + 1 ranges, and each range
+// piece is cut every SC_MAX_SEG_PAGES pages.
+void scorer_sizing(int max_len, int& ppc_min, int& seg_cap) {
+  const int np_max = std::max(1, ceil_div(max_len / QSA_BLOCK, PAGE_BLOCKS));
+  ppc_min = std::max(SC_MIN_PPC, ceil_div(np_max, 14));
+  seg_cap = ceil_div(np_max, ppc_min) + ceil_div(np_max, SC_MAX_SEG_PAGES) + 2;
+}
 
 int positions_bound(int op, int max_len) {
   if (op == QSA_OP_SPARSE_GQA) return max_len;
@@ -40,33 +55,36 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
   const bool scorer = op == QSA_OP_INDEX_SCORE_TOPK || op == QSA_OP_DECODE;
   const bool gqa = op == QSA_OP_SPARSE_GQA || op == QSA_OP_DECODE || op == QSA_OP_DECODE_INDEXSHARE;
   if (!scorer && !gqa && op != QSA_OP_COMPRESS_APPEND) return false;
-  size_t off = 256;  // error word and spare
-  w.cnt_score = off;
-  off += align256(sizeof(int) * (size_t)rows);
-  w.cnt_gqa = off;
-  off += align256(sizeof(int) * (size_t)rows);
+  size_t off = 256;  // error word, prologue ticket, spare
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  w.cnt_gqa = take(sizeof(int) * (size_t)rows);
   if (scorer) {
-    const int nb = max_len / QSA_BLOCK;
-    w.max_chunks_bound = std::max(1, ceil_div(nb, SC_MIN_CHUNK));
-    w.qrot = off;
-    off += align256((size_t)rows * HI * D * 2);
-    w.sel = off;
-    off += align256((size_t)rows * TOPK * 4);
-    w.sel_n = off;
-    off += align256((size_t)rows * 4);
-    w.cand_key = off;
-    off += align256((size_t)rows * w.max_chunks_bound * TOPK * 4);
-    w.cand_id = off;
-    off += align256((size_t)rows * w.max_chunks_bound * TOPK * 4);
+    scorer_sizing(max_len, w.ppc_min, w.seg_cap);
+    if (w.seg_cap > SC_MAX_SEGS) return false;
+    const int np_max = ceil_div(max_len / QSA_BLOCK, PAGE_BLOCKS);
+    if ((int64_t)rows * np_max >= (int64_t)INT32_MAX) return false;
+    w.qrot = take((size_t)rows * HI * D * 2);
+    w.sel = take((size_t)rows * TOPK * 4);
+    w.sel_n = take((size_t)rows * 4);
+    w.row_pages = take((size_t)rows * 4);
+    w.page_off = take((size_t)(rows + 1) * 4);
+    w.seg_cnt = take((size_t)rows * 4);
+    w.cand_cnt = take((size_t)rows * 4);
+    w.pages_done = take((size_t)rows * 4);
+    w.seg_tab = take((size_t)rows * w.seg_cap * 16);
+    w.cand_key = take((size_t)rows * w.seg_cap * TOPK * 4);
+    w.cand_id = take((size_t)rows * w.seg_cap * TOPK * 4);
   }
   if (gqa) {
     const int nq_row = op == QSA_OP_DECODE_INDEXSHARE ? QSA_MAX_DRAFT : 1;
-    w.splits_bound = gqa_splits_for(rows, positions_bound(op, max_len), nq_row, SIZING_SMS);
+    w.splits_bound = gqa_split_bound(rows, positions_bound(op, max_len));
     const size_t heads = (size_t)nq_row * HQ;
-    w.part_o = off;
-    off += align256((size_t)rows * w.splits_bound * heads * D * 4);
-    w.part_ml = off;
-    off += align256((size_t)rows * w.splits_bound * heads * 2 * 4);
+    w.part_o = take((size_t)rows * w.splits_bound * heads * D * 4);
+    w.part_ml = take((size_t)rows * w.splits_bound * heads * 2 * 4);
   }
   w.total = off;
   return true;
@@ -128,36 +146,6 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-// ---- TMA descriptor of the compressed cache: [num_slots/4 rows][128 bf16] ----
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-bool make_cidx_map(const qsa_cache* c, CUtensorMap* map) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(c->num_slots / QSA_BLOCK)};
-  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)PAGE_BLOCKS};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->cidx, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // ---- measurement hook ----
 std::mutex g_prof_mu;
 cudaEvent_t g_prof[16];
@@ -176,30 +164,45 @@ struct ProfScope {
 
 qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
 
-// Scorer pass shared by qsa_decode and qsa_index_score_topk (after the prologue).
-qsa_status run_scorer(const qsa_cache* cache, const CacheView& cv, const int32_t* row_req, const int32_t* row_len,
-                      int len_offset, int rows, int max_len, const __nv_bfloat16* qrot, const float* w, int32_t* sel,
-                      int32_t* sel_n, void* ws, const WsLayout& L, int* err, cudaStream_t st) {
-  CUtensorMap map;
-  if (!make_cidx_map(cache, &map)) return QSA_ERR_CUDA;
+// Prologue (rotation, decode append, page offsets) and scorer, shared by
+// qsa_decode and qsa_index_score_topk.
+qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_bfloat16* knew,
+                       const __nv_bfloat16* idx_q, const int32_t* row_req, const int32_t* row_len, int len_offset,
+                       int rows, int max_len, const float* w, int32_t* sel, int32_t* sel_n, void* ws,
+                       const WsLayout& L, cudaStream_t st) {
+  const RopeFreqs fr = make_freqs(cache->rope_theta);
+  int* err = at<int>(ws, WS_ERR);
+  __nv_bfloat16* qrot = at<__nv_bfloat16>(ws, L.qrot);
+  {
+    ProfScope ps(st, 0);
+    cudaError_t e = launch_index_prologue(cv, knew, idx_q, row_req, row_len, len_offset, rows, max_len, fr, qrot,
+                                          at<int32_t>(ws, L.row_pages), at<int32_t>(ws, L.page_off),
+                                          at<int>(ws, WS_TICKET), err, st);
+    if (e != cudaSuccess) return QSA_ERR_CUDA;
+  }
   ScoreParams p;
   p.c = cv;
   p.row_req = row_req;
   p.row_len = row_len;
   p.len_offset = len_offset;
   p.max_len = max_len;
+  p.rows = rows;
   p.qrot = qrot;
   p.w = w;
-  p.chunk = score_chunk_for(rows, max_len, num_sms());
-  p.max_chunks = std::max(1, ceil_div(max_len / QSA_BLOCK, p.chunk));
-  if (p.max_chunks > L.max_chunks_bound) return QSA_ERR_WORKSPACE;
+  p.page_off = at<int32_t>(ws, L.page_off);
+  p.ppc_min = L.ppc_min;
+  p.seg_cap = L.seg_cap;
+  p.seg_tab = at<int4>(ws, L.seg_tab);
+  p.seg_cnt = at<int>(ws, L.seg_cnt);
+  p.cand_cnt = at<int>(ws, L.cand_cnt);
+  p.pages_done = at<int>(ws, L.pages_done);
   p.cand_key = at<uint32_t>(ws, L.cand_key);
   p.cand_id = at<int32_t>(ws, L.cand_id);
-  p.counters = at<int>(ws, L.cnt_score);
   p.sel = sel;
   p.sel_n = sel_n;
   p.err = err;
-  return cuda_status(launch_score_topk(p, rows, &map, st));
+  ProfScope ps(st, 1);
+  return cuda_status(launch_score_topk(p, score_grid(num_sms()), st));
 }
 
 }  // namespace
@@ -279,15 +282,8 @@ qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const
   WsLayout L;
   if (!layout(QSA_OP_INDEX_SCORE_TOPK, nq, max_len, L)) return QSA_ERR_INVALID_ARG;
   if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const CacheView cv = view_of(cache);
-  const RopeFreqs fr = make_freqs(cache->rope_theta);
-  int* err = at<int>(ws, 0);
-  __nv_bfloat16* qrot = at<__nv_bfloat16>(ws, L.qrot);
-  s = cuda_status(launch_index_prologue(cv, nullptr, static_cast<const __nv_bfloat16*>(idx_q), q_req, q_pos, 1, nq,
-                                        max_len, fr, qrot, err, st));
-  if (s != QSA_OK) return s;
-  return run_scorer(cache, cv, q_req, q_pos, 1, nq, max_len, qrot, w, blocks, nblocks, ws, L, err, st);
+  return run_indexer(cache, view_of(cache), nullptr, static_cast<const __nv_bfloat16*>(idx_q), q_req, q_pos, 1, nq,
+                     max_len, w, blocks, nblocks, ws, L, static_cast<cudaStream_t>(stream));
 }
 
 qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, const int32_t* q_pos, int32_t nq,
@@ -305,6 +301,7 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
   if (s != QSA_OK) return s;
   if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !(scale > 0.f) || !std::isfinite(scale))
     return QSA_ERR_INVALID_ARG;
+  if (max_pos > QSA_MAX_SEL) return QSA_ERR_UNSUPPORTED;
   if (nq == 0) return QSA_OK;
   if (!q || !q_req || !pos || !npos || !out) return QSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(out, 16) || (lse && !aligned(lse, 4))) return QSA_ERR_INVALID_ARG;
@@ -326,9 +323,8 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
   p.part_o = at<float>(ws, L.part_o);
   p.part_ml = at<float>(ws, L.part_ml);
   p.counters = at<int>(ws, L.cnt_gqa);
-  p.splits = std::min(L.splits_bound, gqa_splits_for(nq, max_pos, 1, num_sms()));
-  p.err = at<int>(ws, 0);
-  return cuda_status(launch_gqa(p, nq, static_cast<cudaStream_t>(stream)));
+  p.err = at<int>(ws, WS_ERR);
+  return cuda_status(launch_gqa(p, nq, max_pos, num_sms(), L.splits_bound, static_cast<cudaStream_t>(stream)));
 }
 
 qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
@@ -350,23 +346,12 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const CacheView cv = view_of(cache);
-  const RopeFreqs fr = make_freqs(cache->rope_theta);
-  int* err = at<int>(ws, 0);
-  __nv_bfloat16* qrot = at<__nv_bfloat16>(ws, L.qrot);
+  int* err = at<int>(ws, WS_ERR);
   int32_t* sel = blocks_out ? blocks_out : at<int32_t>(ws, L.sel);
   int32_t* sel_n = nblocks_out ? nblocks_out : at<int32_t>(ws, L.sel_n);
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  {
-    ProfScope ps(st, 0);
-    s = cuda_status(launch_index_prologue(cv, static_cast<const __nv_bfloat16*>(idx_k_new),
-                                          static_cast<const __nv_bfloat16*>(idx_q), nullptr, seq_len, 0, B, max_len,
-                                          fr, qrot, err, st));
-  }
-  if (s != QSA_OK) return s;
-  {
-    ProfScope ps(st, 1);
-    s = run_scorer(cache, cv, nullptr, seq_len, 0, B, max_len, qrot, w, sel, sel_n, ws, L, err, st);
-  }
+  s = run_indexer(cache, cv, static_cast<const __nv_bfloat16*>(idx_k_new), static_cast<const __nv_bfloat16*>(idx_q),
+                  nullptr, seq_len, 0, B, max_len, w, sel, sel_n, ws, L, st);
   if (s != QSA_OK) return s;
   GqaParams p{};
   p.c = cv;
@@ -384,10 +369,9 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   p.part_o = at<float>(ws, L.part_o);
   p.part_ml = at<float>(ws, L.part_ml);
   p.counters = at<int>(ws, L.cnt_gqa);
-  p.splits = std::min(L.splits_bound, gqa_splits_for(B, positions_bound(QSA_OP_DECODE, max_len), 1, num_sms()));
   p.err = err;
   ProfScope ps(st, 2);
-  return cuda_status(launch_gqa(p, B, st));
+  return cuda_status(launch_gqa(p, B, positions_bound(QSA_OP_DECODE, max_len), num_sms(), L.splits_bound, st));
 }
 
 qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_pos, const int32_t* frozen_n,
@@ -420,10 +404,9 @@ qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_p
   p.part_o = at<float>(ws, L.part_o);
   p.part_ml = at<float>(ws, L.part_ml);
   p.counters = at<int>(ws, L.cnt_gqa);
-  p.splits = std::min(L.splits_bound,
-                      gqa_splits_for(B, positions_bound(QSA_OP_DECODE_INDEXSHARE, 1), n_plus_1, num_sms()));
-  p.err = at<int>(ws, 0);
-  return cuda_status(launch_gqa(p, B, static_cast<cudaStream_t>(stream)));
+  p.err = at<int>(ws, WS_ERR);
+  return cuda_status(launch_gqa(p, B, frozen_stride + n_plus_1, num_sms(), L.splits_bound,
+                                static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -199,12 +199,29 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 
 // ---------------------------------------------------------------------------
-// Block-wide exclusive scan (any blockDim that is a multiple of 32, <= 1024).
-// `warp_tot` needs 33 ints of shared memory.  Returns the exclusive prefix of
-// `v` and writes the block total to *total.
+// Thread groups: the first NT threads of the block, synchronising on named
+// barrier BAR (BAR == 0: the whole block with __syncthreads).  Lets a subset of
+// warps (e.g. the consumer warps of a warp-specialised kernel) run the
+// collective helpers below while other warps keep working.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+template <int NT, int BAR>
+struct Group {
+  static constexpr int N = NT;
+  __device__ __forceinline__ static void sync() {
+    if constexpr (BAR == 0) {
+      __syncthreads();
+    } else {
+      asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+    }
+  }
+};
+
+// Exclusive scan over the group.  `warp_tot` needs 33 ints of shared memory.
+// Returns the exclusive prefix of `v`; *total gets the group total.
+template <class G>
+__device__ __forceinline__ int group_exclusive_scan(int v, int* warp_tot, int* total) {
+  constexpr int NW = G::N / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -212,39 +229,48 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
     if (lane >= o) x += y;
   }
   if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
+  G::sync();
   if (warp == 0) {
-    int t = lane < nwarps ? warp_tot[lane] : 0;
+    int t = lane < NW ? warp_tot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, t, o);
       if (lane >= o) t += y;
     }
-    if (lane < nwarps) warp_tot[lane] = t;  // inclusive warp prefix
+    if (lane < NW) warp_tot[lane] = t;  // inclusive warp prefix
     if (lane == 31) warp_tot[32] = t;
   }
-  __syncthreads();
+  G::sync();
   const int before = warp > 0 ? warp_tot[warp - 1] : 0;
   const int res = before + x - v;
   *total = warp_tot[32];
-  __syncthreads();
+  G::sync();
   return res;
 }
 
 // ---------------------------------------------------------------------------
-// CTA-wide exact top-k selection on 32-bit keys (larger key first, then lower
-// index first).  Step 1, radix_select: 8-bit digits from the top find the
-// masked prefix T such that count(key&mask > T) < k <= count(key&mask >= T);
-// `need` is how many elements with key&mask == T are still to be taken.
-// Step 2, select_compact: keeps every key&mask > T and the first `need`
-// elements with key&mask == T in index order, emitting them in index order.
-// KeyAt: int -> uint32 accessor; n may exceed blockDim.
+// Exact top-k selection on 32-bit keys over a group (larger key first, then
+// lower index first).
+//
+// radix_select: finds the masked prefix T with
+//   count(key & mask > T) < k <= count(key & mask >= T)
+// and `need`, how many elements with key & mask == T are still to be taken.
+// It first reduces min and max to skip the high bits every key shares, then
+// walks down in digits of up to 11 bits (2048-bin histograms, warp-aggregated
+// shared-memory atomics), stopping early once the threshold bin is taken whole.
+// select_compact: keeps every key & mask > T and the first `need` elements
+// with key & mask == T in index order, emitting them in index order.
+// KeyAt: int -> uint32 accessor; any n (the loops stride over the group).
 // ---------------------------------------------------------------------------
+constexpr int SEL_BINS = 2048;
+
 struct SelectScratch {
-  int hist[256];
+  int hist[SEL_BINS];
   int warp_tot[33];
   int digit;
   int above;
+  uint32_t kmin[32];
+  uint32_t kmax[32];
 };
 
 struct SelectResult {
@@ -253,62 +279,103 @@ struct SelectResult {
   int need;
 };
 
-template <typename KeyAt>
+template <class G, typename KeyAt>
 __device__ SelectResult radix_select(KeyAt key_at, int n, int k, SelectScratch* sc) {
-  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-  uint32_t prefix = 0, mask = 0;
+  constexpr int NT = G::N;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // common high bits of all keys
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int i = tid; i < n; i += NT) {
+    const uint32_t u = key_at(i);
+    mn = min(mn, u);
+    mx = max(mx, u);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    sc->kmin[warp] = mn;
+    sc->kmax[warp] = mx;
+  }
+  G::sync();
+  mn = sc->kmin[0];
+  mx = sc->kmax[0];
+  for (int w = 1; w < NT / 32; ++w) {
+    mn = min(mn, sc->kmin[w]);
+    mx = max(mx, sc->kmax[w]);
+  }
+  G::sync();
+  if (mn == mx) return SelectResult{mx, 0xFFFFFFFFu, k};  // all keys equal: the first k by index
+  int hb = 31 - __clz(mn ^ mx);                           // highest bit that differs
+  uint32_t mask = hb == 31 ? 0u : ~((2u << hb) - 1u);
+  uint32_t prefix = mx & mask;
   int remaining = k;
-  const int n_round = (n + nt - 1) / nt * nt;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += nt) sc->hist[i] = 0;
-    __syncthreads();
-    for (int i = tid; i < n_round; i += nt) {
+  const int n_round = (n + NT - 1) / NT * NT;
+  while (hb >= 0) {
+    const int lo = max(0, hb - 10);
+    const int bins = 1 << (hb - lo + 1);
+    for (int i = tid; i < bins; i += NT) sc->hist[i] = 0;
+    G::sync();
+    for (int i = tid; i < n_round; i += NT) {
       bool valid = false;
       uint32_t dg = 0xFFFFFFFFu;
       if (i < n) {
         const uint32_t u = key_at(i);
         if ((u & mask) == prefix) {
           valid = true;
-          dg = (u >> shift) & 255u;
+          dg = (u >> lo) & (uint32_t)(bins - 1);
         }
       }
       const unsigned peers = __match_any_sync(0xffffffffu, dg);
       if (valid && lane == __ffs(peers) - 1) atomicAdd(&sc->hist[dg], __popc(peers));
     }
-    __syncthreads();
-    // suffix sums over digits: thread t < 256 handles digit 255 - t
-    int cnt = 0, incl = 0;
-    if (tid < 256) cnt = sc->hist[255 - tid];
-    {
-      int tot;
-      // scan only the first 256 threads' values; others contribute zero
-      const int ex = block_exclusive_scan(tid < 256 ? cnt : 0, sc->warp_tot, &tot);
-      incl = ex + cnt;
-      // digit d = 255 - tid: count of digits > d is ex; count >= d is incl
-      if (tid < 256 && ex < remaining && incl >= remaining) {
-        sc->digit = 255 - tid;
-        sc->above = ex;
+    G::sync();
+    // thread t owns the digits bins-1-t*per .. bins-per-t*per (descending)
+    const int per = (bins + NT - 1) / NT;
+    int local = 0;
+    for (int j = 0; j < per; ++j) {
+      const int d = bins - 1 - (tid * per + j);
+      if (d >= 0) local += sc->hist[d];
+    }
+    int tot;
+    const int ex = group_exclusive_scan<G>(local, sc->warp_tot, &tot);
+    if (ex < remaining && ex + local >= remaining) {
+      int c = ex;
+      for (int j = 0; j < per; ++j) {
+        const int d = bins - 1 - (tid * per + j);
+        if (d < 0) break;
+        const int h = sc->hist[d];
+        if (c + h >= remaining) {
+          sc->digit = d;
+          sc->above = c;
+          break;
+        }
+        c += h;
       }
     }
-    __syncthreads();
+    G::sync();
     const uint32_t d = (uint32_t)sc->digit;
     const int above = sc->above;
     const int in_bin = sc->hist[d];
-    __syncthreads();
+    G::sync();
     remaining -= above;
-    prefix |= d << shift;
-    mask |= 255u << shift;
+    prefix |= d << lo;
+    mask |= (uint32_t)(bins - 1) << lo;
+    hb = lo - 1;
     if (in_bin == remaining) break;  // the whole bin is taken: no finer digit needed
   }
   return SelectResult{prefix, mask, remaining};
 }
 
 // Emit(i, out_index) is called for each kept element, out_index in [0, k).
-template <typename KeyAt, typename Emit>
+template <class G, typename KeyAt, typename Emit>
 __device__ void select_compact(KeyAt key_at, int n, SelectResult r, Emit emit, SelectScratch* sc) {
-  const int tid = threadIdx.x, nt = blockDim.x;
+  constexpr int NT = G::N;
+  const int tid = threadIdx.x;
   int base_gt = 0, base_eq = 0;
-  for (int t0 = 0; t0 < n; t0 += nt) {
+  for (int t0 = 0; t0 < n; t0 += NT) {
     const int i = t0 + tid;
     int gt = 0, eq = 0;
     if (i < n) {
@@ -317,14 +384,178 @@ __device__ void select_compact(KeyAt key_at, int n, SelectResult r, Emit emit, S
       eq = km == r.thresh;
     }
     int tot;
-    const int ex = block_exclusive_scan(gt | (eq << 16), sc->warp_tot, &tot);
-    const int ex_gt = ex & 0xFFFF, ex_eq = ex >> 16;
-    const int eq_before = base_eq + ex_eq;  // equal elements before i
-    const int taken_eq_before = min(eq_before, r.need) - min(base_eq, r.need);
-    if (gt || (eq && eq_before < r.need)) emit(i, base_gt + min(base_eq, r.need) + ex_gt + taken_eq_before);
+    const int ex = group_exclusive_scan<G>(gt | (eq << 16), sc->warp_tot, &tot);
+    const int eq_before = base_eq + (ex >> 16);  // equal elements before i (in index order)
+    if (gt || (eq && eq_before < r.need)) emit(i, base_gt + (ex & 0xFFFF) + min(eq_before, r.need));
     base_gt += tot & 0xFFFF;
     base_eq += tot >> 16;
   }
+}
+
+// ---------------------------------------------------------------------------
+// Fast exact top-k (k <= n) for keys held in shared memory, in a few light
+// passes: (1) min/max, to skip the high bits every key shares; (2) one
+// histogram of the next <= 11 bits, which finds the bin D holding the k-th
+// key; (3) the elements of bin D are gathered and ranked among themselves by
+// (key desc, index asc), which gives the exact cut (key T, index I) of the
+// k-th element; (4) an order-preserving compaction (warp ballots, one barrier
+// round) emits every element above the cut in index order.  Falls back to
+// radix_select/select_compact when bin D holds more than FT_BIN_CAP keys
+// (heavily tied keys).  Emit(i, out_index), out_index in [0, k).
+// ---------------------------------------------------------------------------
+constexpr int FT_BIN_CAP = 1024;
+
+struct FastTopScratch {
+  SelectScratch sel;
+  uint32_t bin_key[FT_BIN_CAP];
+  int bin_idx[FT_BIN_CAP];
+  int bin_cnt;
+  uint32_t cut_key;
+  int cut_idx;
+  int warp_cnt[33];
+};
+
+template <class G, typename KeyAt, typename Emit>
+__device__ void fast_topk(KeyAt key_at, int n, int k, Emit emit, FastTopScratch* fs) {
+  constexpr int NT = G::N, NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  SelectScratch* sc = &fs->sel;
+  // (1) min / max
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int i = tid; i < n; i += NT) {
+    const uint32_t u = key_at(i);
+    mn = min(mn, u);
+    mx = max(mx, u);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    sc->kmin[warp] = mn;
+    sc->kmax[warp] = mx;
+  }
+  if (tid == 0) fs->bin_cnt = 0;
+  G::sync();
+  mn = sc->kmin[0];
+  mx = sc->kmax[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) {
+    mn = min(mn, sc->kmin[w]);
+    mx = max(mx, sc->kmax[w]);
+  }
+  // cut: elements with (key > T) or (key == T and index <= I) are kept
+  uint32_t T;
+  int I;
+  if (mn == mx) {  // all keys equal: the first k by index
+    T = mx;
+    I = k - 1;
+  } else {
+    // (2) histogram over linear bins of the score range.  bin() is monotone
+    // (IEEE subtraction, multiplication and floor are), so a larger key never
+    // lands in a lower bin; scores spread over the bins far better than the
+    // raw bits of their encoding do.
+    const float smin = key_score(mn), smax = key_score(mx);
+    const float span = smax - smin;
+    if (!(span > 1e-30f) || !(span < 3.0e38f)) {  // degenerate range: exact radix refinement
+      const SelectResult r = radix_select<G>(key_at, n, k, sc);
+      select_compact<G>(key_at, n, r, emit, sc);
+      return;
+    }
+    const float scale = (float)SEL_BINS / span;
+    auto bin_of = [&](uint32_t u) { return min(SEL_BINS - 1, (int)((key_score(u) - smin) * scale)); };
+    constexpr int bins = SEL_BINS;
+    for (int i = tid; i < bins; i += NT) sc->hist[i] = 0;
+    G::sync();
+    for (int i = tid; i < n; i += NT) atomicAdd(&sc->hist[bin_of(key_at(i))], 1);
+    G::sync();
+    constexpr int per = (bins + NT - 1) / NT;  // thread t owns bins bins-1-t*per .. (descending)
+    int local = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+      const int d = bins - 1 - (tid * per + j);
+      if (d >= 0) local += sc->hist[d];
+    }
+    int tot;
+    const int ex = group_exclusive_scan<G>(local, sc->warp_tot, &tot);
+    if (ex < k && ex + local >= k) {
+      int c = ex;
+      for (int j = 0; j < per; ++j) {
+        const int d = bins - 1 - (tid * per + j);
+        if (d < 0) break;
+        const int h = sc->hist[d];
+        if (c + h >= k) {
+          sc->digit = d;
+          sc->above = c;
+          break;
+        }
+        c += h;
+      }
+    }
+    G::sync();
+    const int D = sc->digit;
+    const int need = k - sc->above;  // elements still to take from bin D (>= 1)
+    const int inbin = sc->hist[D];
+    G::sync();
+    if (inbin > FT_BIN_CAP) {  // heavily tied keys: exact radix refinement
+      const SelectResult r = radix_select<G>(key_at, n, k, sc);
+      select_compact<G>(key_at, n, r, emit, sc);
+      return;
+    }
+    // (3) gather bin D and rank its elements
+    for (int i = tid; i < n; i += NT) {
+      const uint32_t u = key_at(i);
+      if (bin_of(u) == D) {
+        const int slot = atomicAdd(&fs->bin_cnt, 1);
+        fs->bin_key[slot] = u;
+        fs->bin_idx[slot] = i;
+      }
+    }
+    G::sync();
+    const int cnt = fs->bin_cnt;
+    for (int j = tid; j < cnt; j += NT) {
+      const uint32_t kj = fs->bin_key[j];
+      const int ij = fs->bin_idx[j];
+      int rank = 0;
+      for (int m = 0; m < cnt; ++m) {
+        const uint32_t km = fs->bin_key[m];
+        rank += (km > kj) || (km == kj && fs->bin_idx[m] < ij);
+      }
+      if (rank == need - 1) {
+        fs->cut_key = kj;
+        fs->cut_idx = ij;
+      }
+    }
+    G::sync();
+    T = fs->cut_key;
+    I = fs->cut_idx;
+    G::sync();
+  }
+  // (4) order-preserving compaction: warp w owns [w*chunk, (w+1)*chunk)
+  const int chunk = ((n + NW - 1) / NW + 31) & ~31;
+  const int w0 = min(n, warp * chunk), w1 = min(n, w0 + chunk);
+  auto kept = [&](int i) {
+    const uint32_t u = key_at(i);
+    return u > T || (u == T && i <= I);
+  };
+  int count = 0;
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    count += __popc(__ballot_sync(0xffffffffu, i < w1 && kept(i)));
+  }
+  if (lane == 0) fs->warp_cnt[warp] = count;
+  G::sync();
+  int out = 0;
+  for (int w = 0; w < warp; ++w) out += fs->warp_cnt[w];
+  for (int base = w0; base < w1; base += 32) {
+    const int i = base + lane;
+    const bool kp = i < w1 && kept(i);
+    const unsigned m = __ballot_sync(0xffffffffu, kp);
+    if (kp) emit(i, out + __popc(m & ((1u << lane) - 1u)));
+    out += __popc(m);
+  }
+  G::sync();
 }
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }

@@ -17,6 +17,8 @@
 // an online softmax in the log2 domain, and O += P V_g for its 64 output
 // dims.  Splits write (O, m, l) partials; the last CTA of the row (atomic
 // ticket, no waiting) merges them.
+#include <cstdlib>
+
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 
@@ -28,12 +30,14 @@ constexpr int GQ_ROW_BYTES = D * 2;                             // 256 B: one he
 constexpr int GQ_KV_BYTES = GQ_TILE * HKV * GQ_ROW_BYTES;       // 8 KiB: K (or V) of a tile
 constexpr int GQ_STAGE_BYTES = 2 * GQ_KV_BYTES;                 // 16 KiB
 
+constexpr int GQ_MAX_TILES = (QSA_MAX_SEL + QSA_MAX_DRAFT + GQ_TILE - 1) / GQ_TILE;  // per row
+
 template <int MT>
 struct GqaSmem {
   alignas(128) uint8_t q[HKV][MT * 16][GQ_ROW_BYTES];
   alignas(128) uint8_t kv[GQ_STAGES][GQ_STAGE_BYTES];  // [K|V][group][pos][256 B], swizzled
-  float ml[HKV][MT * 16][2];
   int is_last;
+  int32_t slot[1];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(((chunk ^ (row & 7)) << 4)); }
@@ -69,7 +73,7 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
       }
     } else {
       const int n = __ldg(p.list_n + row);
-      if (n < 0 || n > p.list_stride) {
+      if (n < 0 || n > p.list_stride || n > MAX_SEL) {
         if (split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_SELECTION);
         bad = true;
       } else {
@@ -81,7 +85,11 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   const int ext0 = (!bad && p.extra_base) ? __ldg(p.extra_base + row) : 0;
   const int ntot = bad ? 0 : nbase + (p.extra_base ? p.n_extra : 0);
   const int tiles = ceil_div(ntot, GQ_TILE);
-  const int tps = ceil_div(tiles, p.splits);
+  int tps = ceil_div(tiles, p.splits);
+  if (tps > p.tiles_per_split) {  // more positions than the host bound it was sized for
+    if (split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_SELECTION);
+    tps = p.tiles_per_split;
+  }
   const int t_begin = min(tiles, split * tps), t_end = min(tiles, t_begin + tps);
   const int ntl = t_end - t_begin;
 
@@ -108,26 +116,24 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
     }
   }
 
+  // ---- physical slots of this CTA's positions, resolved once up front ----
+  for (int j = tid; j < ntl * GQ_TILE; j += THREADS) {
+    const int jj = t_begin * GQ_TILE + j;
+    S.slot[j] = jj < ntot ? (int32_t)slot_of(p.c, req, position(jj), p.err) : -1;
+  }
+  __syncthreads();
+
   // ---- async gather of one tile into a stage ----
   // chunk id c in [0, 1024): kv = c >> 9, pos j = (c >> 5) & 15, group = (c >> 4) & 1, 16 B chunk = c & 15
   auto issue_tile = [&](int t, int stage) {
     uint8_t* dst0 = S.kv[stage];
     constexpr int PER = 1024 / THREADS;  // chunks per thread
-    constexpr int POS_PER = 512 / THREADS > 0 ? 512 / THREADS : 1;
-    int64_t slot[(PER + 1) / 2 > 0 ? (PER + 1) / 2 : 1];
-#pragma unroll
-    for (int k = 0; k < (PER + 1) / 2; ++k) {
-      const int c = tid + k * THREADS;
-      const int j = (c >> 5) & 15;
-      const int jj = t * GQ_TILE + j;
-      slot[k] = jj < ntot ? slot_of(p.c, req, position(jj), p.err) : -1;
-    }
-    (void)POS_PER;
+    const int32_t* tslot = S.slot + (t - t_begin) * GQ_TILE;
 #pragma unroll
     for (int k = 0; k < PER; ++k) {
       const int c = tid + k * THREADS;
       const int kvsel = c >> 9, j = (c >> 5) & 15, g = (c >> 4) & 1, ch = c & 15;
-      const int64_t sl = slot[k % ((PER + 1) / 2)];
+      const int64_t sl = tslot[j];
       const __nv_bfloat16* base = kvsel ? p.c.v : p.c.k;
       const __nv_bfloat16* src = sl >= 0 ? base + (sl * HKV + g) * D + ch * 8 : base;
       uint8_t* dst = dst0 + kvsel * GQ_KV_BYTES + g * (GQ_TILE * GQ_ROW_BYTES) + j * GQ_ROW_BYTES + swz(j, ch);
@@ -323,39 +329,78 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   if (tid == 0) p.counters[row] = 0;
 }
 
-int gqa_splits_for(int rows, int max_pos, int nq_row, int num_sms) {
-  const int tiles = ceil_div(max_pos, GQ_TILE);
-  // aim for ~3 resident CTAs per SM over the whole grid, at least 2 tiles per split
-  int s = ceil_div(3 * num_sms, rows > 0 ? rows : 1);
+// Workspace bound on the split count (no device needed): at most 8 resident
+// CTAs per SM on at most 256 SMs.
+int gqa_split_bound(int rows, int max_pos) {
+  const int tiles = ceil_div(max(max_pos, 1), GQ_TILE);
+  int s = ceil_div(8 * 256, rows > 0 ? rows : 1);
   s = min(s, max(1, tiles / 2));
-  s = max(1, min(s, GQ_MAX_SPLITS));
-  (void)nq_row;
-  return s;
+  return max(1, min(s, GQ_MAX_SPLITS));
 }
 
 template <int MT>
-static cudaError_t launch_mt(const GqaParams& p, int rows, cudaStream_t st) {
+static size_t gqa_smem_bytes(int tiles_per_split) {
+  return sizeof(GqaSmem<MT>) + sizeof(int32_t) * (size_t)tiles_per_split * GQ_TILE + 128;
+}
+
+template <int MT>
+static int occupancy(size_t smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_sparse_gqa<MT>, MT * 128, smem) != cudaSuccess) return 1;
+  return max(n, 1);
+}
+
+// Splits so that the grid is one wave of resident CTAs (rows x splits <=
+// resident CTAs per SM x SMs), each split at least two tiles.
+template <int MT>
+static void choose_splits(int rows, int max_pos, int num_sms, int bound, int& splits, int& tps) {
+  static const int forced = [] {  // tuning override: QSA_GQA_CTAS_PER_SM=1..8 (resident CTAs to plan for)
+    const char* e = getenv("QSA_GQA_CTAS_PER_SM");
+    const int v = e ? atoi(e) : 0;
+    return (v >= 1 && v <= 8) ? v : 0;
+  }();
+  const int tiles = ceil_div(max(max_pos, 1), GQ_TILE);
+  rows = max(rows, 1);
+  for (int occ_try = 8; occ_try >= 1; --occ_try) {
+    if (forced && occ_try != forced) continue;
+    int s = (occ_try * num_sms) / rows;
+    s = max(1, min(s, min(max(1, tiles / 2), min(bound, GQ_MAX_SPLITS))));
+    const int t = ceil_div(tiles, s);
+    if (forced || occupancy<MT>(gqa_smem_bytes<MT>(t)) >= occ_try || occ_try == 1) {
+      splits = s;
+      tps = t;
+      return;
+    }
+  }
+  splits = 1;
+  tps = tiles;
+}
+
+template <int MT>
+static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, int bound, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  const size_t smem = sizeof(GqaSmem<MT>) + 128;
+  const size_t smem_max = gqa_smem_bytes<MT>(GQ_MAX_TILES);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  choose_splits<MT>(rows, max_pos, num_sms, bound, p.splits, p.tiles_per_split);
   dim3 grid(p.splits, rows);
-  k_sparse_gqa<MT><<<grid, MT * 128, smem, st>>>(p);
+  k_sparse_gqa<MT><<<grid, MT * 128, gqa_smem_bytes<MT>(p.tiles_per_split), st>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gqa(const GqaParams& p, int rows, cudaStream_t st) {
+cudaError_t launch_gqa(const GqaParams& p, int rows, int max_pos, int num_sms, int split_bound, cudaStream_t st) {
   const int mt = ceil_div(p.nq_row * GROUP, 16);
   switch (mt) {
-    case 1: return launch_mt<1>(p, rows, st);
-    case 2: return launch_mt<2>(p, rows, st);
+    case 1: return launch_mt<1>(p, rows, max_pos, num_sms, split_bound, st);
+    case 2: return launch_mt<2>(p, rows, max_pos, num_sms, split_bound, st);
     case 3:
-    case 4: return launch_mt<4>(p, rows, st);
+    case 4: return launch_mt<4>(p, rows, max_pos, num_sms, split_bound, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -123,52 +123,82 @@ __global__ void __launch_bounds__(128) k_compress_append(CacheView c, const __nv
 // ring slot (L-1) mod 4, and when it completes block b = L/4 - 1 that block is
 // compressed from the ring slots 0..2 and the new key.  Always: the 4 index
 // query heads are rotated at position L-1 (L = row_len[row] + len_offset) and
-// stored as bf16 in qrot [rows][4][128].
+// stored as bf16 in qrot [rows][4][128]; row_pages[row] gets the number of
+// 64-token pages the scorer streams for the row (0 when it keeps every block
+// or the row is invalid), and the last CTA to finish (atomic ticket) writes
+// their exclusive prefix to page_off[0..rows].
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_index_prologue(CacheView c, const __nv_bfloat16* __restrict__ knew,
                                                         const __nv_bfloat16* __restrict__ idx_q,
                                                         const int32_t* __restrict__ row_req,
                                                         const int32_t* __restrict__ row_len, int len_offset,
-                                                        int max_len, RopeFreqs fr, __nv_bfloat16* __restrict__ qrot,
-                                                        int* err) {
+                                                        int max_len, int rows, RopeFreqs fr,
+                                                        __nv_bfloat16* __restrict__ qrot, int32_t* row_pages,
+                                                        int32_t* page_off, int* ticket, int* err) {
   const int row = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int req = row_req ? row_req[row] : row;
   const int L = row_len[row] + len_offset;
-  if (req < 0 || req >= c.batch || L < 1 || L > max_len) {
-    if (tid == 0) set_error(err, (req < 0 || req >= c.batch) ? QSA_DEVERR_REQUEST : QSA_DEVERR_LENGTH);
-    return;
-  }
-  const int pos = L - 1;
+  const bool valid = req >= 0 && req < c.batch && L >= 1 && L <= max_len;
   __shared__ double cs_s[D / 2], sn_s[D / 2];
-  if (tid < D / 2) sincos((double)pos * fr.f[tid], &sn_s[tid], &cs_s[tid]);
-
-  if (knew != nullptr && warp == 0) {
-    __nv_bfloat16* ring = c.ring + (int64_t)req * CBLK * D;
-    const __nv_bfloat16* key = knew + (int64_t)row * D;
-    if ((pos & 3) == 3) {
-      const __nv_bfloat16* k4[4] = {ring, ring + D, ring + 2 * D, key};
-      const int64_t b = pos >> 2;
-      const int64_t e = cidx_entry(c, req, b, err);
-      if (e >= 0) warp_compress_block(k4, b, fr, c.cidx + e * D);
-      __syncwarp();
+  __shared__ int warp_tot[33];
+  __shared__ int is_last;
+  if (!valid) {
+    if (tid == 0) set_error(err, (req < 0 || req >= c.batch) ? QSA_DEVERR_REQUEST : QSA_DEVERR_LENGTH);
+  } else {
+    const int pos = L - 1;
+    if (tid < D / 2) sincos((double)pos * fr.f[tid], &sn_s[tid], &cs_s[tid]);
+    if (knew != nullptr && warp == 0) {
+      __nv_bfloat16* ring = c.ring + (int64_t)req * CBLK * D;
+      const __nv_bfloat16* key = knew + (int64_t)row * D;
+      if ((pos & 3) == 3) {
+        const __nv_bfloat16* k4[4] = {ring, ring + D, ring + 2 * D, key};
+        const int64_t b = pos >> 2;
+        const int64_t e = cidx_entry(c, req, b, err);
+        if (e >= 0) warp_compress_block(k4, b, fr, c.cidx + e * D);
+        __syncwarp();
+      }
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(key);
+      uint32_t* dst = reinterpret_cast<uint32_t*>(ring + (pos & 3) * D);
+      for (int i = tid; i < D / 2; i += 32) dst[i] = src[i];
     }
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(key);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(ring + (pos & 3) * D);
-    for (int i = tid; i < D / 2; i += 32) dst[i] = src[i];
   }
   __syncthreads();
-  // rotate: thread t handles head t / 32 and pairs i = t % 32, t % 32 + 32
-  const int h = tid >> 5, lane = tid & 31;
-  const uint16_t* qin = reinterpret_cast<const uint16_t*>(idx_q + ((int64_t)row * HI + h) * D);
-  uint16_t* qo = reinterpret_cast<uint16_t*>(qrot + ((int64_t)row * HI + h) * D);
+  if (valid) {
+    // rotate: thread t handles head t / 32 and pairs i = t % 32, t % 32 + 32
+    const int h = tid >> 5, lane = tid & 31;
+    const uint16_t* qin = reinterpret_cast<const uint16_t*>(idx_q + ((int64_t)row * HI + h) * D);
+    uint16_t* qo = reinterpret_cast<uint16_t*>(qrot + ((int64_t)row * HI + h) * D);
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int i = lane + 32 * e;
-    const double x0 = (double)bf16_bits_to_f32(qin[i]);
-    const double x1 = (double)bf16_bits_to_f32(qin[i + D / 2]);
-    qo[i] = f64_to_bf16_bits(x0 * cs_s[i] - x1 * sn_s[i]);
-    qo[i + D / 2] = f64_to_bf16_bits(x0 * sn_s[i] + x1 * cs_s[i]);
+    for (int e = 0; e < 2; ++e) {
+      const int i = lane + 32 * e;
+      const double x0 = (double)bf16_bits_to_f32(qin[i]);
+      const double x1 = (double)bf16_bits_to_f32(qin[i + D / 2]);
+      qo[i] = f64_to_bf16_bits(x0 * cs_s[i] - x1 * sn_s[i]);
+      qo[i + D / 2] = f64_to_bf16_bits(x0 * sn_s[i] + x1 * cs_s[i]);
+    }
+  }
+  if (row_pages == nullptr) return;
+  const int nb = valid ? (L >> 2) : 0;
+  if (tid == 0) row_pages[row] = nb > TOPK ? ceil_div(nb, PAGE_BLOCKS) : 0;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(ticket, 1) == rows - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  using All = Group<128, 0>;
+  int running = 0;
+  for (int base = 0; base < rows; base += 128) {
+    const int v = base + tid < rows ? __ldcg(row_pages + base + tid) : 0;
+    int tot;
+    const int ex = group_exclusive_scan<All>(v, warp_tot, &tot);
+    if (base + tid < rows) page_off[base + tid] = running + ex;
+    running += tot;
+  }
+  if (tid == 0) {
+    page_off[rows] = running;
+    *ticket = 0;  // ready for the next call
   }
 }
 
@@ -208,9 +238,10 @@ cudaError_t launch_compress_append(const CacheView& c, const __nv_bfloat16* knew
 
 cudaError_t launch_index_prologue(const CacheView& c, const __nv_bfloat16* knew, const __nv_bfloat16* idx_q,
                                   const int32_t* row_req, const int32_t* row_len, int len_offset, int rows,
-                                  int max_len, const RopeFreqs& fr, __nv_bfloat16* qrot, int* err,
-                                  cudaStream_t st) {
-  k_index_prologue<<<rows, 128, 0, st>>>(c, knew, idx_q, row_req, row_len, len_offset, max_len, fr, qrot, err);
+                                  int max_len, const RopeFreqs& fr, __nv_bfloat16* qrot, int32_t* row_pages,
+                                  int32_t* page_off, int* ticket, int* err, cudaStream_t st) {
+  k_index_prologue<<<rows, 128, 0, st>>>(c, knew, idx_q, row_req, row_len, len_offset, max_len, rows, fr, qrot,
+                                         row_pages, page_off, ticket, err);
   return cudaGetLastError();
 }
 

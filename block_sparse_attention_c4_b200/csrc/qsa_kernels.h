@@ -10,15 +10,20 @@ namespace qsa {
 cudaError_t launch_compress_append(const CacheView& c, const __nv_bfloat16* knew, const int32_t* cu_new,
                                    const int32_t* len_before, int total_new, int max_new, const RopeFreqs& fr,
                                    int* err, cudaStream_t st);
+// Rotates each row's index query (and, for decode, appends the new index key),
+// writes the row's number of pages to score, and -- in the CTA that finishes
+// last -- the exclusive prefix of those page counts (page_off[rows + 1]).
 cudaError_t launch_index_prologue(const CacheView& c, const __nv_bfloat16* knew, const __nv_bfloat16* idx_q,
                                   const int32_t* row_req, const int32_t* row_len, int len_offset, int rows,
-                                  int max_len, const RopeFreqs& fr, __nv_bfloat16* qrot, int* err, cudaStream_t st);
+                                  int max_len, const RopeFreqs& fr, __nv_bfloat16* qrot, int32_t* row_pages,
+                                  int32_t* page_off, int* ticket, int* err, cudaStream_t st);
 cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblocks, const int32_t* q_pos, int nq, int32_t* pos,
                           int32_t* npos, int* err, cudaStream_t st);
 
 // ---- streaming scorer + top-512 (qsa_score.cu) ----
-constexpr int SC_MIN_CHUNK = 1024;  // blocks per CTA, lower bound (workspace sizing)
-constexpr int SC_MAX_CHUNK = 4096;  // upper bound (shared memory sizing)
+constexpr int SC_MAX_SEG_PAGES = 512;  // pages of one segment (8192 blocks of score keys in shared memory)
+constexpr int SC_MAX_SEGS = 64;        // segments per row a merge can order
+constexpr int SC_MIN_PPC = 32;         // pages per CTA range, lower bound
 
 struct ScoreParams {
   CacheView c;
@@ -26,20 +31,25 @@ struct ScoreParams {
   const int32_t* row_len;  // L = row_len[row] + len_offset
   int len_offset;
   int max_len;
+  int rows;
   const __nv_bfloat16* qrot;  // [rows][4][128] rotated index queries
   const float* w;             // [rows][4]
-  int chunk;                  // blocks per CTA (multiple of 16, SC_MIN_CHUNK..SC_MAX_CHUNK)
-  int max_chunks;             // grid.x; candidate buffer stride
-  uint32_t* cand_key;         // [rows][max_chunks][512]
-  int32_t* cand_id;           // [rows][max_chunks][512]
-  int* counters;              // [rows], zero between calls
+  const int32_t* page_off;    // [rows + 1] exclusive prefix of pages to score per row
+  int ppc_min;                // pages per CTA range, lower bound
+  int seg_cap;                // segment slots per row
+  int4* seg_tab;              // [rows][seg_cap] (first block, candidate offset, count, -)
+  int* seg_cnt;               // [rows], zero between calls
+  int* cand_cnt;              // [rows], zero between calls
+  int* pages_done;            // [rows], zero between calls
+  uint32_t* cand_key;         // [rows][seg_cap * 512]
+  int32_t* cand_id;           // [rows][seg_cap * 512]
   int32_t* sel;               // [rows][512] out
   int32_t* sel_n;             // [rows] out
   int* err;
 };
 
-int score_chunk_for(int rows, int max_len, int num_sms);
-cudaError_t launch_score_topk(const ScoreParams& p, int rows, const CUtensorMap* tmap, cudaStream_t st);
+int score_grid(int num_sms);
+cudaError_t launch_score_topk(const ScoreParams& p, int grid, cudaStream_t st);
 
 // ---- sparse GQA (qsa_gqa.cu) ----
 constexpr int GQ_MAX_SPLITS = 16;
@@ -66,11 +76,14 @@ struct GqaParams {
   float* part_o;              // [rows][splits][nq_row*16][128]
   float* part_ml;             // [rows][splits][nq_row*16][2]
   int* counters;              // [rows]
-  int splits;
+  int splits;                 // set by launch_gqa
+  int tiles_per_split;        // set by launch_gqa
   int* err;
 };
 
-int gqa_splits_for(int rows, int max_pos, int nq_row, int num_sms);
-cudaError_t launch_gqa(const GqaParams& p, int rows, cudaStream_t st);
+// Upper bound of the split count launch_gqa may choose (workspace sizing).
+int gqa_split_bound(int rows, int max_pos);
+// Chooses the split count (one wave of resident CTAs, at most split_bound) and launches.
+cudaError_t launch_gqa(const GqaParams& p, int rows, int max_pos, int num_sms, int split_bound, cudaStream_t st);
 
 }  // namespace qsa

@@ -80,6 +80,7 @@ extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void*
     return QSA_ERR_INVALID_ARG;
   if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !(scale > 0.f)) return QSA_ERR_INVALID_ARG;
   if (nq > QSA_NOALLOC_MAX_QUERIES) return QSA_ERR_UNSUPPORTED;  // beyond the array's stated capacity
+  if (max_pos > QSA_MAX_SEL) return QSA_ERR_UNSUPPORTED;
   if (nq == 0) return QSA_OK;
   if (!q || !q_req || !pos || !npos || !out) return QSA_ERR_INVALID_ARG;
   if (!is_aligned(q, 16) || !is_aligned(out, 16) || (lse && !is_aligned(lse, 4))) return QSA_ERR_INVALID_ARG;
@@ -110,9 +111,7 @@ extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void*
   p.part_o = reinterpret_cast<float*>(base + OFF_O);
   p.part_ml = reinterpret_cast<float*>(base + OFF_ML);
   p.counters = reinterpret_cast<int*>(base + OFF_COUNTERS);
-  const int cap = ROW_SPLITS / nq > 0 ? ROW_SPLITS / nq : 1;
-  int splits = gqa_splits_for(nq, max_pos, 1, sm_count());
-  p.splits = splits < cap ? splits : cap;
+  const int cap = ROW_SPLITS / nq > 0 ? ROW_SPLITS / nq : 1;  // partials that fit the array
   p.err = nullptr;  // no error word: positions outside their request are skipped silently
-  return launch_gqa(p, nq, st) == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
+  return launch_gqa(p, nq, max_pos, sm_count(), cap, st) == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }

@@ -7,205 +7,355 @@
 // lost; this is the stated reading): s_b = sum_h w_h * max(0, q~_h . k^_b);
 // ties keep the lower block index.
 //
-// Design (B200): the pass is HBM-bound -- 256 bytes of compressed key per
-// block against 4 dot products of 128.  Each CTA owns a chunk of one row's
-// blocks.  A producer warp streams whole 64-token pages (16 compressed keys =
-// 4 KiB, contiguous because the cache is page aligned) with 2-D TMA into a
-// 16-deep shared-memory ring, 128-byte swizzled so that ldmatrix reads are
-// conflict free.  Eight consumer warps each turn a page into 16 scores with
-// eight m16n8k16 bf16 MMAs (A = 16 keys x 16 dims, B = the 4 rotated query
-// heads padded to 8 columns) -- this keeps the FP32 pipes free, the tensor
-// pipe is nowhere near busy.  Scores never leave the SM: they become
-// order-preserving 32-bit keys in shared memory, a CTA-wide radix select keeps
-// the chunk's best 512, and the last CTA of the row to finish (atomic ticket,
-// no waiting) merges the chunks' candidates from L2 into the final 512.
+// Design (B200).  The pass is HBM-bound: 256 bytes of compressed key per block
+// against 4 dot products of 128.  Work is balanced exactly, whatever the mix
+// of context lengths: all pages to score (64 tokens = 16 compressed keys =
+// 4 KiB, contiguous because the cache is page aligned) are laid end to end
+// over the rows, and each persistent CTA (two per SM) owns equal contiguous
+// ranges of that list.  A range crosses at most a few rows; its piece of one
+// row is a "segment".
+//   * Pages sit at random places in HBM, so what bounds the pass is how many
+//     independent 4 KiB reads are in flight; a measured probe of this access
+//     pattern peaks with many warps each holding whole pages, not with one
+//     TMA producer per CTA.  So every warp reads its own pages with coalesced
+//     16-byte loads straight into registers (each load instruction covers
+//     eight keys x 64 contiguous bytes), U pages at a time.
+//   * The loaded registers ARE the A fragments of m16n8k16 bf16 MMAs (A = 16
+//     keys x 16 dims, B = the 4 rotated query heads padded to 8 columns):
+//     because a dot product does not care about the order of its terms, the
+//     query's B fragments are built with the same permutation of dims that
+//     the loads produce, and no shuffle or shared-memory staging is needed.
+//     The FP32 pipes stay free; the tensor pipe is far from busy.
+//   * Scores become order-preserving 32-bit keys in shared memory.  At the
+//     end of a segment the CTA radix-selects its best 512 (the other CTAs on
+//     the SM keep streaming).  A segment that is a whole row gives the answer
+//     directly; otherwise its candidates go to the row's list in global
+//     memory, and the CTA that completes the row's last segment (atomic page
+//     count, no waiting) merges them: it orders the row's segments by block,
+//     stages their candidates in shared memory and selects the final 512,
+//     ascending.  Scores never travel to HBM.
+#include <cstdlib>
+
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 
 namespace qsa {
 
-constexpr int SC_CONS = 8;                      // consumer warps
-constexpr int SC_THREADS = (SC_CONS + 1) * 32;  // + one producer warp
-constexpr int SC_STAGES = 16;                   // pages in flight per CTA
-constexpr int SC_PAGE_BYTES = PAGE_BLOCKS * D * 2;  // 4096
+#ifndef QSA_SC_PAGES_PER_LOAD
+#define QSA_SC_PAGES_PER_LOAD 1
+#endif
+#ifndef QSA_SC_CTAS_PER_SM
+#define QSA_SC_CTAS_PER_SM 2
+#endif
+constexpr int SC_WARPS = 8;
+constexpr int SC_THREADS = SC_WARPS * 32;
+constexpr int SC_U = QSA_SC_PAGES_PER_LOAD;  // pages a warp loads before computing
+constexpr int SC_SEG_KEYS = SC_MAX_SEG_PAGES * PAGE_BLOCKS;  // 8192
+constexpr int SC_ROWS_SMEM = 512;  // rows whose page offsets are staged in shared memory
 
-struct __align__(1024) ScoreSmem {
-  uint8_t stage[SC_STAGES][SC_PAGE_BYTES];  // each page: two 16 x 128 B halves (dims 0-63, 64-127)
-  uint32_t keys[SC_MAX_CHUNK];
-  uint64_t full[SC_STAGES];
-  uint64_t empty[SC_STAGES];
-  SelectScratch sel;
-  int is_last;
+using Cta = Group<SC_THREADS, 0>;
+
+struct ScoreSmem {
+  uint32_t keys[SC_SEG_KEYS];     // a segment's score keys; a merge's candidates
+  int32_t pid[SC_MAX_SEG_PAGES];  // physical pages of the current segment (-1: invalid)
+  int32_t off[SC_ROWS_SMEM + 1];  // exclusive prefix of pages per row
+  int4 segs[SC_MAX_SEGS];         // merge: the row's segments (start block, cand offset, count, -)
+  int vstart[SC_MAX_SEGS + 1];    // merge: prefix of the ordered segments' counts
+  FastTopScratch ft;
+  int bcast[4];
 };
 
-__global__ void __launch_bounds__(SC_THREADS, 2) k_score_topk(ScoreParams p, const __grid_constant__ CUtensorMap tmap) {
+struct Segment {
+  int row, p0, np;  // row, first page within the row, pages
+};
+
+// Largest row r with off[r] <= g (off is non-decreasing; rows without pages
+// have empty intervals and are never returned for g < off[rows]).
+__device__ __forceinline__ int row_of_page(const int32_t* off_s, const int32_t* off_g, int rows, int g) {
+  int lo = 0, hi = rows - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    const int v = off_s ? off_s[mid] : __ldg(off_g + mid);
+    if (v <= g) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// One page of 16 keys: lane (g, c) holds 16-byte chunks c, c+4, c+8, c+12 of
+// keys g and g+8.  Chunk u of key g, read as four bf16 pairs x, y, z, w,
+// supplies the A fragment of k-steps 2u (pairs x, y) and 2u+1 (pairs z, w):
+// logical k {2c, 2c+1} -> first pair, {2c+8, 2c+9} -> second pair.
+struct PageRegs {
+  uint4 lo[4], hi[4];  // keys g and g + 8
+};
+
+__device__ __forceinline__ void load_page(PageRegs& r, const uint4* page, int g, int c) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    r.lo[u] = ldg_stream(page + g * 16 + c + 4 * u);
+    r.hi[u] = ldg_stream(page + (g + 8) * 16 + c + 4 * u);
+  }
+}
+
+__device__ __forceinline__ void score_page(const PageRegs& r, const uint32_t (&bq)[8][2], float wa, float wb,
+                                           float& lo_score, float& hi_score) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int u = j >> 1;
+    uint32_t a[4];
+    a[0] = (j & 1) ? r.lo[u].z : r.lo[u].x;
+    a[1] = (j & 1) ? r.hi[u].z : r.hi[u].x;
+    a[2] = (j & 1) ? r.lo[u].w : r.lo[u].y;
+    a[3] = (j & 1) ? r.hi[u].w : r.hi[u].y;
+    mma_bf16_16816(acc, a, bq[j][0], bq[j][1]);
+  }
+  // acc: rows g / g+8 (keys), columns 2c, 2c+1 (heads); sum the heads over the quad
+  float lo = wa * fmaxf(acc[0], 0.f) + wb * fmaxf(acc[1], 0.f);
+  float hi = wa * fmaxf(acc[2], 0.f) + wb * fmaxf(acc[3], 0.f);
+  lo += __shfl_xor_sync(0xffffffffu, lo, 1);
+  hi += __shfl_xor_sync(0xffffffffu, hi, 1);
+  lo += __shfl_xor_sync(0xffffffffu, lo, 2);
+  hi += __shfl_xor_sync(0xffffffffu, hi, 2);
+  lo_score = lo;
+  hi_score = hi;
+}
+
+__global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(ScoreParams p) {
   extern __shared__ uint8_t smem_raw[];
-  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int row = blockIdx.y, chunk = blockIdx.x;
+  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int req = p.row_req ? __ldg(p.row_req + row) : row;
-  const int L = __ldg(p.row_len + row) + p.len_offset;
-  int32_t* sel = p.sel + (int64_t)row * TOPK;
-  if (req < 0 || req >= p.c.batch || L < 1 || L > p.max_len) {
-    if (chunk == 0 && tid == 0) {
-      set_error(p.err, (req < 0 || req >= p.c.batch) ? QSA_DEVERR_REQUEST : QSA_DEVERR_LENGTH);
-      p.sel_n[row] = 0;
-    }
-    return;
-  }
-  const int nb = L >> 2;
-  if (nb <= TOPK) {  // every complete block is kept
-    if (chunk == 0) {
-      for (int i = tid; i < nb; i += blockDim.x) sel[i] = i;
-      if (tid == 0) p.sel_n[row] = nb;
-    }
-    return;
-  }
-  const int nchunks = ceil_div(nb, p.chunk);
-  if (chunk >= nchunks) return;
-  const int b0 = chunk * p.chunk;
-  const int nvalid = min(p.chunk, nb - b0);
-  const int npages = ceil_div(nvalid, PAGE_BLOCKS);
-  const int page0 = b0 / PAGE_BLOCKS;
+  const int rows = p.rows;
 
-  if (tid == 0) {
-    for (int s = 0; s < SC_STAGES; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);
+  // ---- rows with at most 512 complete blocks keep them all; bad rows keep none ----
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int req = p.row_req ? __ldg(p.row_req + r) : r;
+    const int L = __ldg(p.row_len + r) + p.len_offset;
+    const bool bad = req < 0 || req >= p.c.batch || L < 1 || L > p.max_len;
+    const int nb = bad ? 0 : (L >> 2);
+    if (nb > TOPK) continue;
+    int32_t* sel = p.sel + (int64_t)r * TOPK;
+    for (int i = tid; i < nb; i += SC_THREADS) sel[i] = i;
+    if (tid == 0) {
+      p.sel_n[r] = nb;
+      if (bad) set_error(p.err, (req < 0 || req >= p.c.batch) ? QSA_DEVERR_REQUEST : QSA_DEVERR_LENGTH);
     }
-    fence_mbar_init();
   }
+
+  // ---- the page list ----
+  const bool off_in_smem = rows <= SC_ROWS_SMEM;
+  if (off_in_smem)
+    for (int i = tid; i <= rows; i += SC_THREADS) S.off[i] = __ldg(p.page_off + i);
   __syncthreads();
+  const int32_t* off_s = off_in_smem ? S.off : nullptr;
+  auto off_at = [&](int r) { return off_in_smem ? S.off[r] : __ldg(p.page_off + r); };
+  const int P = off_at(rows);
+  if (P == 0) return;
+  int ppc = ceil_div(P, gridDim.x);  // pages per range
+  ppc = max(ppc, p.ppc_min);
+  const int nranges = ceil_div(P, ppc);
 
-  if (warp == SC_CONS) {
-    // ---------------- producer: one lane issues the page loads ----------------
-    if (lane == 0) {
-      prefetch_tmap(&tmap);
+  const int g8 = lane >> 2, cq = lane & 3;
+  const uint4* cidx = reinterpret_cast<const uint4*>(p.c.cidx);
+  int range = -1, g = 0, gend = 0;
+  int cur_row = -1;
+  uint32_t bq[8][2];
+  float wa = 0.f, wb = 0.f;
+  auto skey = [&](int i) { return S.keys[i]; };
+  while (true) {
+    // ---- next segment: ranges blockIdx.x, +gridDim.x, ..., cut at row boundaries and every 512 pages ----
+    if (g >= gend) {
+      range = range < 0 ? (int)blockIdx.x : range + (int)gridDim.x;
+      if (range >= nranges) break;
+      g = range * ppc;
+      gend = min(P, g + ppc);
+    }
+    Segment sg;
+    sg.row = row_of_page(off_s, p.page_off, rows, g);
+    const int rend = off_at(sg.row + 1);
+    sg.p0 = g - off_at(sg.row);
+    sg.np = min(min(gend, rend), g + SC_MAX_SEG_PAGES) - g;
+    g += sg.np;
+    if (sg.np <= 0) continue;
+    const int r = sg.row;
+    const int req = p.row_req ? __ldg(p.row_req + r) : r;
+    {  // the segment's physical pages
       const int32_t* pt = p.c.page_table + (int64_t)req * p.c.max_pages;
-      for (int i = 0; i < npages; ++i) {
-        const int s = i % SC_STAGES;
-        if (i >= SC_STAGES) mbar_wait(&S.empty[s], ((i / SC_STAGES) - 1) & 1, p.err);
-        const int lp = page0 + i;
-        const int phys = lp < p.c.max_pages ? __ldg(pt + lp) : -1;
+      for (int k = tid; k < sg.np; k += SC_THREADS) {
+        const int lp = sg.p0 + k;
+        int phys = lp < p.c.max_pages ? __ldg(pt + lp) : -1;
         if (phys < 0 || phys >= p.c.num_pages) {
           set_error(p.err, QSA_DEVERR_PAGE);
-          mbar_arrive(&S.full[s]);  // complete the phase without data
-          continue;
+          phys = -1;
         }
-        mbar_arrive_expect_tx(&S.full[s], SC_PAGE_BYTES);
-        tma_load_2d(S.stage[s], &tmap, 0, phys * PAGE_BLOCKS, &S.full[s]);
-        tma_load_2d(S.stage[s] + SC_PAGE_BYTES / 2, &tmap, 64, phys * PAGE_BLOCKS, &S.full[s]);
+        S.pid[k] = phys;
       }
     }
-  } else {
-    // ---------------- consumers: 16 scores per page on the tensor pipe --------
-    const int g = lane >> 2, cq = lane & 3;
-    // B operand: column n = index head n (n < 4), k = dim; padded heads are 0.
-    uint32_t bq[8][2];
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.qrot + (int64_t)row * HI * D);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      bq[j][0] = g < HI ? __ldg(q32 + ((g * D + 16 * j + 2 * cq) >> 1)) : 0u;
-      bq[j][1] = g < HI ? __ldg(q32 + ((g * D + 16 * j + 2 * cq + 8) >> 1)) : 0u;
-    }
-    const float wa = cq < 2 ? __ldg(p.w + (int64_t)row * HI + 2 * cq) : 0.f;
-    const float wb = cq < 2 ? __ldg(p.w + (int64_t)row * HI + 2 * cq + 1) : 0.f;
-    // ldmatrix lane geometry: matrix mtx = lane/8 covers rows (mtx&1)*8.., dims (mtx>>1)*8..
-    const int mtx = lane >> 3;
-    const int rr = (lane & 7) + ((mtx & 1) << 3);
-    const uint32_t lane_off = rr * 128;
-    for (int i = warp; i < npages; i += SC_CONS) {
-      const int s = i % SC_STAGES;
-      mbar_wait(&S.full[s], (i / SC_STAGES) & 1, p.err);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t base = smem_u32(S.stage[s]) + lane_off;
+    if (r != cur_row) {
+      // B operand, permuted like the loads: column n = index head n (zero for n >= 4); for k-step
+      // j = 2u + h, lane (n, c) holds dims 8(c+4u) + 4h + {0,1} (b0) and + {2,3} (b1).
+      cur_row = r;
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.qrot + (int64_t)r * HI * D);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int c16 = ((j & 3) << 1) + (mtx >> 1);
-        uint32_t a[4];
-        ldmatrix_x4(a[0], a[1], a[2], a[3], base + (j >> 2) * (SC_PAGE_BYTES / 2) + ((c16 ^ (rr & 7)) << 4));
-        mma_bf16_16816(acc, a, bq[j][0], bq[j][1]);
+        const int d0 = 8 * (cq + 4 * (j >> 1)) + 4 * (j & 1);
+        bq[j][0] = g8 < HI ? __ldg(q32 + ((g8 * D + d0) >> 1)) : 0u;
+        bq[j][1] = g8 < HI ? __ldg(q32 + ((g8 * D + d0 + 2) >> 1)) : 0u;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.empty[s]);
-      // acc: rows g / g+8 (keys), columns 2cq, 2cq+1 (heads)
-      float lo = wa * fmaxf(acc[0], 0.f) + wb * fmaxf(acc[1], 0.f);
-      float hi = wa * fmaxf(acc[2], 0.f) + wb * fmaxf(acc[3], 0.f);
-      lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-      hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-      lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-      hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-      if (cq < 2) {
-        const int local = i * PAGE_BLOCKS + g + 8 * cq;
-        if (local < nvalid) S.keys[local] = score_key(cq ? hi : lo);
+      wa = cq < 2 ? __ldg(p.w + (int64_t)r * HI + 2 * cq) : 0.f;
+      wb = cq < 2 ? __ldg(p.w + (int64_t)r * HI + 2 * cq + 1) : 0.f;
+    }
+    const int L = __ldg(p.row_len + r) + p.len_offset;
+    const int nb = L >> 2;
+    const int b0 = sg.p0 * PAGE_BLOCKS;
+    const int nvalid = min(sg.np * PAGE_BLOCKS, nb - b0);
+    Cta::sync();
+
+    // ---- stream: warp w scores pages w, w+8, ... (SC_U at a time) ----
+    for (int k0 = warp * SC_U; k0 < sg.np; k0 += SC_WARPS * SC_U) {
+      PageRegs pr[SC_U];
+#pragma unroll
+      for (int u = 0; u < SC_U; ++u) {
+        const int k = k0 + u;
+        const int phys = k < sg.np ? S.pid[k] : -1;
+        if (phys >= 0) load_page(pr[u], cidx + (int64_t)phys * (PAGE_BLOCKS * D / 8), g8, cq);
+      }
+#pragma unroll
+      for (int u = 0; u < SC_U; ++u) {
+        const int k = k0 + u;
+        if (k >= sg.np) break;
+        float lo, hi;
+        score_page(pr[u], bq, wa, wb, lo, hi);
+        if (S.pid[k] < 0) lo = hi = 0.f;  // unreadable page (flagged above)
+        if (cq < 2) {
+          const int local = k * PAGE_BLOCKS + g8 + 8 * cq;
+          if (local < nvalid) S.keys[local] = score_key(cq ? hi : lo);
+        }
       }
     }
-  }
-  __syncthreads();
+    Cta::sync();
 
-  // ---------------- chunk top-512 ----------------
-  SelectResult r{0u, 0u, nvalid};  // nvalid <= 512: keep all (every key matches the empty mask)
-  auto skey = [&](int i) { return S.keys[i]; };
-  if (nvalid > TOPK) r = radix_select(skey, nvalid, TOPK, &S.sel);
-  if (nchunks == 1) {
-    select_compact(skey, nvalid, r, [&](int i, int o) { sel[o] = b0 + i; }, &S.sel);
-    if (tid == 0) p.sel_n[row] = TOPK;
-    return;
-  }
-  uint32_t* ck = p.cand_key + ((int64_t)row * p.max_chunks + chunk) * TOPK;
-  int32_t* ci = p.cand_id + ((int64_t)row * p.max_chunks + chunk) * TOPK;
-  select_compact(
-      skey, nvalid, r,
-      [&](int i, int o) {
+    // ---- the segment's best 512 ----
+    const int np_row = off_at(r + 1) - off_at(r);
+    int32_t* sel = p.sel + (int64_t)r * TOPK;
+    if (sg.np == np_row) {  // the whole row (nb > 512 here): this is the answer
+      fast_topk<Cta>(skey, nvalid, TOPK, [&](int i, int o) { sel[o] = b0 + i; }, &S.ft);
+      if (tid == 0) p.sel_n[r] = TOPK;
+      Cta::sync();
+      continue;
+    }
+    const int ncand = min(nvalid, TOPK);
+    if (tid == 0) {
+      const int slot = atomicAdd(p.seg_cnt + r, 1);
+      int coff = atomicAdd(p.cand_cnt + r, ncand);
+      const bool fits = slot < p.seg_cap && coff + ncand <= p.seg_cap * TOPK;
+      if (!fits) {  // more segments than the workspace was sized for: drop this one, flag it
+        set_error(p.err, QSA_DEVERR_SELECTION);
+        coff = -1;
+      }
+      if (slot < p.seg_cap) p.seg_tab[(int64_t)r * p.seg_cap + slot] = make_int4(b0, fits ? coff : 0, fits ? ncand : 0, 0);
+      S.bcast[0] = coff;
+    }
+    Cta::sync();
+    const int coff = S.bcast[0];
+    if (coff >= 0) {
+      uint32_t* ck = p.cand_key + (int64_t)r * p.seg_cap * TOPK + coff;
+      int32_t* ci = p.cand_id + (int64_t)r * p.seg_cap * TOPK + coff;
+      auto put = [&](int i, int o) {
         ck[o] = S.keys[i];
         ci[o] = b0 + i;
-      },
-      &S.sel);
-  for (int o = min(nvalid, TOPK) + tid; o < TOPK; o += blockDim.x) {  // pad: below every real key
-    ck[o] = 0u;
-    ci[o] = -1;
-  }
+      };
+      if (nvalid > TOPK) {
+        fast_topk<Cta>(skey, nvalid, TOPK, put, &S.ft);
+      } else {
+        for (int i = tid; i < nvalid; i += SC_THREADS) put(i, i);
+      }
+    }
+    __threadfence();
+    Cta::sync();
+    if (tid == 0) S.bcast[1] = atomicAdd(p.pages_done + r, sg.np) + sg.np == np_row;
+    Cta::sync();
+    if (!S.bcast[1]) continue;
 
-  // ---------------- last CTA of the row merges ----------------
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) S.is_last = atomicAdd(p.counters + row, 1) == nchunks - 1;
-  __syncthreads();
-  if (!S.is_last) return;
-  __threadfence();
-  const uint32_t* rk = p.cand_key + (int64_t)row * p.max_chunks * TOPK;
-  const int32_t* ri = p.cand_id + (int64_t)row * p.max_chunks * TOPK;
-  const int n = nchunks * TOPK;
-  auto gkey = [&](int i) { return __ldcg(rk + i); };
-  const SelectResult m = radix_select(gkey, n, TOPK, &S.sel);
-  select_compact(gkey, n, m, [&](int i, int o) { sel[o] = __ldcg(ri + i); }, &S.sel);
-  if (tid == 0) {
-    p.sel_n[row] = TOPK;
-    p.counters[row] = 0;  // ready for the next call
+    // ---- this CTA finished the row: merge its segments' candidates ----
+    __threadfence();
+    const int ns = min(__ldcg(p.seg_cnt + r), min(p.seg_cap, SC_MAX_SEGS));
+    const int4* tab = p.seg_tab + (int64_t)r * p.seg_cap;
+    // order the segments by first block (rank sort in shared memory; the starts are distinct)
+    int4* raw = reinterpret_cast<int4*>(S.keys);
+    for (int j = tid; j < ns; j += SC_THREADS) raw[j] = __ldcg(tab + j);
+    Cta::sync();
+    for (int j = tid; j < ns; j += SC_THREADS) {
+      const int4 e = raw[j];
+      int rank = 0;
+      for (int m = 0; m < ns; ++m) rank += raw[m].x < e.x;
+      S.segs[rank] = e;
+    }
+    Cta::sync();
+    if (tid == 0) {
+      int acc = 0;
+      for (int j = 0; j < ns; ++j) {
+        S.vstart[j] = acc;
+        acc += S.segs[j].z;
+      }
+      S.vstart[ns] = acc;
+    }
+    Cta::sync();
+    const uint32_t* rk = p.cand_key + (int64_t)r * p.seg_cap * TOPK;
+    const int32_t* ri = p.cand_id + (int64_t)r * p.seg_cap * TOPK;
+    // virtual index v (ascending block order) -> index into the row's candidate list
+    auto gidx = [&](int v) {
+      int lo = 0, hi = ns - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (S.vstart[mid] <= v) lo = mid;
+        else hi = mid - 1;
+      }
+      return S.segs[lo].y + (v - S.vstart[lo]);
+    };
+    const int nv = S.vstart[ns];
+    auto put = [&](int v, int o) { sel[o] = __ldcg(ri + gidx(v)); };
+    if (nv <= SC_SEG_KEYS) {
+      for (int v = tid; v < nv; v += SC_THREADS) S.keys[v] = __ldcg(rk + gidx(v));
+      Cta::sync();
+      fast_topk<Cta>(skey, nv, TOPK, put, &S.ft);
+    } else {  // long rows: read the candidates from L2 in place
+      auto gkey = [&](int v) { return __ldcg(rk + gidx(v)); };
+      const SelectResult m = radix_select<Cta>(gkey, nv, TOPK, &S.ft.sel);
+      select_compact<Cta>(gkey, nv, m, put, &S.ft.sel);
+    }
+    if (tid == 0) {
+      p.sel_n[r] = TOPK;
+      p.seg_cnt[r] = 0;  // ready for the next call
+      p.cand_cnt[r] = 0;
+      p.pages_done[r] = 0;
+    }
+    Cta::sync();
   }
 }
 
-int score_chunk_for(int rows, int max_len, int num_sms) {
-  const int nb = max_len / CBLK;
-  int chunk = 2048;
-  // prefer more CTAs when the batch is small, fewer (less merge work) when it is large
-  while (chunk > SC_MIN_CHUNK && (int64_t)rows * ceil_div(nb, chunk) < 4 * num_sms) chunk >>= 1;
-  while (chunk < SC_MAX_CHUNK && (int64_t)rows * ceil_div(nb, chunk) > 16 * num_sms) chunk <<= 1;
-  return chunk;
-}
+int score_grid(int num_sms) { return QSA_SC_CTAS_PER_SM * num_sms; }
 
-cudaError_t launch_score_topk(const ScoreParams& p, int rows, const CUtensorMap* tmap, cudaStream_t st) {
+cudaError_t launch_score_topk(const ScoreParams& p, int grid, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  const size_t smem = sizeof(ScoreSmem) + 1024;
+  const size_t smem = sizeof(ScoreSmem) + 128;
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k_score_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(p.max_chunks, rows);
-  k_score_topk<<<grid, SC_THREADS, smem, st>>>(p, *tmap);
+  k_score_topk<<<grid, SC_THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -54,7 +54,7 @@ extern "C" {
 #define QSA_MAX_SEL 2051    /* 512 * 4 + 3 positions                              */
 #define QSA_PAGE_SIZE 64    /* tokens per K/V page (16 compressed entries)        */
 #define QSA_MAX_DRAFT 8     /* largest n_plus_1 of qsa_decode_indexshare          */
-#define QSA_MAX_CONTEXT (1 << 24) /* largest context length accepted              */
+#define QSA_MAX_CONTEXT (1 << 20) /* largest context length accepted (1,048,576)    */
 
 typedef enum {
   QSA_OK = 0,
@@ -177,7 +177,9 @@ qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, con
  *   q        bf16 [nq][16][128]
  *   q_req    int32 [nq] request of each query (device)
  *   pos      int32 [nq][pos_stride] positions (device); npos int32 [nq]
- *   max_pos  host bound of npos[i] (<= pos_stride)
+ *   max_pos  host bound of npos[i] (<= pos_stride and <= QSA_MAX_SEL, else
+ *            QSA_ERR_UNSUPPORTED); a row whose npos exceeds 2051 is skipped
+ *            and flagged QSA_DEVERR_SELECTION
  *   scale    softmax scale (1/sqrt(128) for the layer)
  *   out      bf16 [nq][16][128] out; lse f32 [nq][16] out (natural log) or NULL
  *   ws       workspace of qsa_workspace_bytes(QSA_OP_SPARSE_GQA, nq, max_pos)

@@ -49,7 +49,7 @@ def test_workspace_bytes(qsa):
         assert n > 0 and n % 256 == 0
     assert qsa.workspace_bytes(99, 4, 100) == 0
     assert qsa.workspace_bytes(qsa.OP_DECODE, -1, 100) == 0
-    assert qsa.workspace_bytes(qsa.OP_DECODE, 4, (1 << 24) + 1) == 0
+    assert qsa.workspace_bytes(qsa.OP_DECODE, 4, (1 << 20) + 1) == 0
     # grows with the batch and with the context (candidate buffers)
     assert qsa.workspace_bytes(qsa.OP_DECODE, 64, 131072) > qsa.workspace_bytes(qsa.OP_DECODE, 4, 131072)
     assert qsa.workspace_bytes(qsa.OP_DECODE, 4, 262147) > qsa.workspace_bytes(qsa.OP_DECODE, 4, 8192)

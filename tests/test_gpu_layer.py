@@ -336,3 +336,38 @@ def test_indexshare_small(Q, W):
 def test_indexshare_full_config(Q, W):
     """Batch 16, capture context 65536 + U[0,3], 3 draft steps (4 drafted positions)."""
     _indexshare_case(Q, W, G.indexshare_64k())
+
+
+def test_topk_heavy_ties_across_segments(Q, W):
+    """Thousands of blocks with bit-identical compressed keys: the kept set must take the tied blocks
+    with the lowest indices, inside every scorer segment and in the merge of the segments."""
+    for nb in (3000, 20000):
+        L = 4 * nb
+        wl = G.custom_decode(29, [L])
+        cache = W.build_cache(wl, prefix_tokens=[0])
+        rng = np.random.default_rng(nb)
+        a = rng.standard_normal(128)
+        b = 0.3 * a + rng.standard_normal(128)
+        keys = np.empty((nb, 128), dtype=np.uint16)
+
+        def bits(v):  # unit vector -> bf16 bits
+            t = torch.from_numpy((v / np.linalg.norm(v)).astype(np.float32)).to(torch.bfloat16)
+            return t.view(torch.int16).numpy().view(np.uint16)
+
+        keys[:] = bits(b)
+        keys[::50] = bits(a)  # 400 (or 60) blocks tie at the top, the rest tie below
+        pt = wl.page_table()[0]
+        blk = np.arange(nb)
+        entries = (pt[(4 * blk) // 64].astype(np.int64) * 64 + (4 * blk) % 64) // 4
+        cache.cidx[torch.from_numpy(entries).cuda()] = W.bits_to_bf16(keys, "cuda")
+        idx_q = np.repeat(bits(a)[None, :], 4, axis=0)[None]  # every head looks along a
+        w = np.array([[0.5, 0.25, 0.125, 1.0]], dtype=np.float32)
+        ws = Q.Workspace(Q.workspace_bytes(Q.OP_INDEX_SCORE_TOPK, 1, L))
+        blocks, nblocks = Q.index_score_topk(cache, W.bits_to_bf16(idx_q, "cuda"), torch.from_numpy(w).cuda(),
+                                             torch.zeros(1, dtype=torch.int32).cuda(),
+                                             torch.tensor([L - 1], dtype=torch.int32).cuda(), L, ws)
+        torch.cuda.synchronize()
+        assert ws.device_error() == 0
+        ob, _, s = O.select_query(idx_q[0], w[0], keys, L)
+        assert len(np.unique(s)) <= 2 and nblocks.item() == 512
+        np.testing.assert_array_equal(blocks[0].cpu().numpy(), ob)
