@@ -27,6 +27,7 @@ PAGE_SIZE = 64
 MAX_DRAFT = 8
 
 OP_INDEX_SCORE_TOPK, OP_SPARSE_GQA, OP_DECODE, OP_DECODE_INDEXSHARE, OP_COMPRESS_APPEND = 1, 2, 3, 4, 5
+OP_PREFILL_SCORE_TOPK = 6
 
 DEVERR_BITS = {1: "page", 2: "length", 4: "position", 8: "request", 16: "selection", 32: "timeout"}
 
@@ -49,6 +50,7 @@ EXPORTS = [
     "qsa_workspace_bytes", "qsa_workspace_init", "qsa_compress_append", "qsa_index_score_topk",
     "qsa_expand_indices", "qsa_sparse_gqa", "qsa_decode", "qsa_decode_indexshare", "qsa_device_error",
     "qsa_set_profile_events", "qsa_decode_kernel_count", "qsa_status_string", "qsa_version",
+    "qsa_prefill_score_topk",
 ]
 
 
@@ -68,6 +70,8 @@ def lib():
     L.qsa_compress_append.argtypes = [cp, vp, vp, vp, i32, i32, vp]
     L.qsa_index_score_topk.argtypes = [cp, vp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]
     L.qsa_expand_indices.argtypes = [vp, vp, vp, i32, vp, vp, vp]
+    L.qsa_prefill_score_topk.argtypes = [cp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+    L.qsa_prefill_score_topk.restype = ctypes.c_int
     L.qsa_sparse_gqa.argtypes = [cp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
     L.qsa_decode.argtypes = [cp, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]
     L.qsa_decode_indexshare.argtypes = [cp, vp, vp, i32, vp, i32, vp, f32, vp, vp, sz, vp]
@@ -81,6 +85,7 @@ def lib():
     L.qsa_status_string.argtypes = [ctypes.c_int]
     L.qsa_status_string.restype = ctypes.c_char_p
     L.qsa_version.restype = ctypes.c_char_p
+    L.qsa_last_error_string.restype = ctypes.c_char_p
     for name in ("qsa_workspace_init", "qsa_compress_append", "qsa_index_score_topk", "qsa_expand_indices",
                  "qsa_sparse_gqa", "qsa_decode", "qsa_decode_indexshare"):
         getattr(L, name).restype = ctypes.c_int
@@ -90,7 +95,8 @@ def lib():
 
 def _check(status: int, what: str):
     if status != 0:
-        raise QsaError(f"{what} failed: {lib().qsa_status_string(status).decode()} (status {status})")
+        detail = f" [{lib().qsa_last_error_string().decode()}]" if status == 4 else ""
+        raise QsaError(f"{what} failed: {lib().qsa_status_string(status).decode()} (status {status}){detail}")
 
 
 def _ptr(t):
@@ -105,13 +111,15 @@ def _stream(stream=None):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _dev(t: torch.Tensor, dtype, name: str):
+def _dev(t: torch.Tensor, dtype, name: str, shape=None):
     if not t.is_cuda:
         raise QsaError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise QsaError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise QsaError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise QsaError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
 
 
@@ -171,9 +179,9 @@ def compress_append(cache: LayerCache, idx_k_new, cu_new, len_before, max_new: i
     c = cache.struct()
     total = int(idx_k_new.shape[0]) if idx_k_new is not None else 0
     if total:
-        _dev(idx_k_new, torch.bfloat16, "idx_k_new")
-    _dev(cu_new, torch.int32, "cu_new")
-    _dev(len_before, torch.int32, "len_before")
+        _dev(idx_k_new, torch.bfloat16, "idx_k_new", (total, HEAD_DIM))
+    _dev(cu_new, torch.int32, "cu_new", (cache.batch + 1,))
+    _dev(len_before, torch.int32, "len_before", (cache.batch,))
     _check(lib().qsa_compress_append(ctypes.byref(c), _ptr(idx_k_new) if total else None, _ptr(cu_new),
                                      _ptr(len_before), total, int(max_new), _stream(stream)), "qsa_compress_append")
 
@@ -187,10 +195,31 @@ def index_score_topk(cache: LayerCache, idx_q, w, q_req, q_pos, max_len: int, ws
     if nblocks is None:
         nblocks = torch.zeros(nq, dtype=torch.int32, device=dev)
     c = cache.struct()
-    _check(lib().qsa_index_score_topk(ctypes.byref(c), _ptr(_dev(idx_q, torch.bfloat16, "idx_q")),
-                                      _ptr(_dev(w, torch.float32, "w")), _ptr(_dev(q_req, torch.int32, "q_req")),
-                                      _ptr(_dev(q_pos, torch.int32, "q_pos")), nq, int(max_len), _ptr(blocks),
+    _dev(blocks, torch.int32, "blocks", (nq, TOPK))
+    _dev(nblocks, torch.int32, "nblocks", (nq,))
+    _check(lib().qsa_index_score_topk(ctypes.byref(c), _ptr(_dev(idx_q, torch.bfloat16, "idx_q", (nq, INDEX_HEADS, HEAD_DIM))),
+                                      _ptr(_dev(w, torch.float32, "w", (nq, INDEX_HEADS))),
+                                      _ptr(_dev(q_req, torch.int32, "q_req", (nq,))),
+                                      _ptr(_dev(q_pos, torch.int32, "q_pos", (nq,))), nq, int(max_len), _ptr(blocks),
                                       _ptr(nblocks), ws.ptr, ws.nbytes, _stream(stream)), "qsa_index_score_topk")
+    return blocks, nblocks
+
+
+def prefill_score_topk(cache: LayerCache, idx_q, w, req: int, pos0: int, ws: Workspace, blocks=None, nblocks=None,
+                       stream=None):
+    """Tensor-core scoring + top-512 of the causal chunk of queries at positions pos0 .. pos0+T-1."""
+    T = int(idx_q.shape[0])
+    dev = idx_q.device
+    if blocks is None:
+        blocks = torch.full((T, TOPK), -1, dtype=torch.int32, device=dev)
+    if nblocks is None:
+        nblocks = torch.zeros(T, dtype=torch.int32, device=dev)
+    c = cache.struct()
+    _dev(blocks, torch.int32, "blocks", (T, TOPK))
+    _dev(nblocks, torch.int32, "nblocks", (T,))
+    _check(lib().qsa_prefill_score_topk(ctypes.byref(c), _ptr(_dev(idx_q, torch.bfloat16, "idx_q", (T, INDEX_HEADS, HEAD_DIM))),
+                                        _ptr(_dev(w, torch.float32, "w", (T, INDEX_HEADS))), int(req), int(pos0), T, _ptr(blocks),
+                                        _ptr(nblocks), ws.ptr, ws.nbytes, _stream(stream)), "qsa_prefill_score_topk")
     return blocks, nblocks
 
 
@@ -201,6 +230,11 @@ def expand_indices(blocks, nblocks, q_pos, pos=None, npos=None, stream=None):
         pos = torch.full((nq, MAX_SEL), -1, dtype=torch.int32, device=dev)
     if npos is None:
         npos = torch.zeros(nq, dtype=torch.int32, device=dev)
+    _dev(blocks, torch.int32, "blocks", (nq, TOPK))
+    _dev(nblocks, torch.int32, "nblocks", (nq,))
+    _dev(q_pos, torch.int32, "q_pos", (nq,))
+    _dev(pos, torch.int32, "pos", (nq, MAX_SEL))
+    _dev(npos, torch.int32, "npos", (nq,))
     _check(lib().qsa_expand_indices(_ptr(blocks), _ptr(nblocks), _ptr(q_pos), nq, _ptr(pos), _ptr(npos),
                                     _stream(stream)), "qsa_expand_indices")
     return pos, npos
@@ -213,9 +247,12 @@ def sparse_gqa(cache: LayerCache, q, q_req, pos, npos, max_pos: int, ws: Workspa
     if out is None:
         out = torch.empty(nq, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
     c = cache.struct()
-    _check(lib().qsa_sparse_gqa(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q")),
-                                _ptr(_dev(q_req, torch.int32, "q_req")), _ptr(_dev(pos, torch.int32, "pos")),
-                                _ptr(_dev(npos, torch.int32, "npos")), int(pos.shape[1]), int(max_pos), nq,
+    _dev(out, torch.bfloat16, "out", (nq, Q_HEADS, HEAD_DIM))
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (nq, Q_HEADS))
+    _check(lib().qsa_sparse_gqa(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q", (nq, Q_HEADS, HEAD_DIM))),
+                                _ptr(_dev(q_req, torch.int32, "q_req", (nq,))), _ptr(_dev(pos, torch.int32, "pos")),
+                                _ptr(_dev(npos, torch.int32, "npos", (nq,))), int(pos.shape[1]), int(max_pos), nq,
                                 float(scale), _ptr(out), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)),
            "qsa_sparse_gqa")
     return out
@@ -232,9 +269,12 @@ def sparse_gqa_noalloc(cache: LayerCache, q, q_req, pos, npos, max_pos: int, sca
     if out is None:
         out = torch.empty(nq, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
     c = cache.struct()
-    _check(lib().qsa_sparse_gqa_noalloc(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q")),
-                                        _ptr(_dev(q_req, torch.int32, "q_req")), _ptr(_dev(pos, torch.int32, "pos")),
-                                        _ptr(_dev(npos, torch.int32, "npos")), int(pos.shape[1]), int(max_pos), nq,
+    _dev(out, torch.bfloat16, "out", (nq, Q_HEADS, HEAD_DIM))
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (nq, Q_HEADS))
+    _check(lib().qsa_sparse_gqa_noalloc(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q", (nq, Q_HEADS, HEAD_DIM))),
+                                        _ptr(_dev(q_req, torch.int32, "q_req", (nq,))), _ptr(_dev(pos, torch.int32, "pos")),
+                                        _ptr(_dev(npos, torch.int32, "npos", (nq,))), int(pos.shape[1]), int(max_pos), nq,
                                         float(scale), _ptr(out), _ptr(lse), _stream(stream)),
            "qsa_sparse_gqa_noalloc")
     return out
@@ -247,9 +287,17 @@ def decode(cache: LayerCache, idx_k_new, idx_q, w, q, seq_len, max_len: int, ws:
     if out is None:
         out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
     c = cache.struct()
-    _check(lib().qsa_decode(ctypes.byref(c), _ptr(_dev(idx_k_new, torch.bfloat16, "idx_k_new")),
-                            _ptr(_dev(idx_q, torch.bfloat16, "idx_q")), _ptr(_dev(w, torch.float32, "w")),
-                            _ptr(_dev(q, torch.bfloat16, "q")), _ptr(_dev(seq_len, torch.int32, "seq_len")),
+    _dev(out, torch.bfloat16, "out", (B, Q_HEADS, HEAD_DIM))
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (B, Q_HEADS))
+    if blocks_out is not None:
+        _dev(blocks_out, torch.int32, "blocks_out", (B, TOPK))
+        _dev(nblocks_out, torch.int32, "nblocks_out", (B,))
+    _check(lib().qsa_decode(ctypes.byref(c), _ptr(_dev(idx_k_new, torch.bfloat16, "idx_k_new", (B, HEAD_DIM))),
+                            _ptr(_dev(idx_q, torch.bfloat16, "idx_q", (B, INDEX_HEADS, HEAD_DIM))),
+                            _ptr(_dev(w, torch.float32, "w", (B, INDEX_HEADS))),
+                            _ptr(_dev(q, torch.bfloat16, "q", (B, Q_HEADS, HEAD_DIM))),
+                            _ptr(_dev(seq_len, torch.int32, "seq_len", (B,))),
                             int(max_len), float(scale), _ptr(out), _ptr(lse), _ptr(blocks_out), _ptr(nblocks_out),
                             ws.ptr, ws.nbytes, _stream(stream)), "qsa_decode")
     return out
@@ -262,9 +310,12 @@ def decode_indexshare(cache: LayerCache, frozen_pos, frozen_n, len0, q, ws: Work
     if out is None:
         out = torch.empty(B, n_plus_1, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
     c = cache.struct()
+    if B != cache.batch:
+        raise QsaError(f"q must have one row per request ({cache.batch}), got {B}")
+    _dev(out, torch.bfloat16, "out", (B, n_plus_1, Q_HEADS, HEAD_DIM))
     _check(lib().qsa_decode_indexshare(ctypes.byref(c), _ptr(_dev(frozen_pos, torch.int32, "frozen_pos")),
-                                       _ptr(_dev(frozen_n, torch.int32, "frozen_n")), int(frozen_pos.shape[1]),
-                                       _ptr(_dev(len0, torch.int32, "len0")), n_plus_1,
+                                       _ptr(_dev(frozen_n, torch.int32, "frozen_n", (B,))), int(frozen_pos.shape[1]),
+                                       _ptr(_dev(len0, torch.int32, "len0", (B,))), n_plus_1,
                                        _ptr(_dev(q, torch.bfloat16, "q")), float(scale), _ptr(out), ws.ptr,
                                        ws.nbytes, _stream(stream)), "qsa_decode_indexshare")
     return out

@@ -24,9 +24,11 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct WsLayout {
   size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, seg_cnt = 0, cand_cnt = 0,
          pages_done = 0, seg_tab = 0, cand_key = 0, cand_id = 0, part_o = 0, part_ml = 0, total = 0;
+  size_t pf_scale = 0, pf_cand_n = 0, pf_thr = 0, pf_ovf_n = 0, pf_ovf_list = 0;
   int ppc_min = 0;
   int seg_cap = 0;
   int splits_bound = 0;
+  int cap = 0;
 };
 
 constexpr size_t WS_ERR = 0;     // int: device error word
@@ -54,13 +56,27 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
   if (rows < 0 || max_len < 0 || max_len > QSA_MAX_CONTEXT) return false;
   const bool scorer = op == QSA_OP_INDEX_SCORE_TOPK || op == QSA_OP_DECODE;
   const bool gqa = op == QSA_OP_SPARSE_GQA || op == QSA_OP_DECODE || op == QSA_OP_DECODE_INDEXSHARE;
-  if (!scorer && !gqa && op != QSA_OP_COMPRESS_APPEND) return false;
+  const bool prefill = op == QSA_OP_PREFILL_SCORE_TOPK;
+  if (!scorer && !gqa && !prefill && op != QSA_OP_COMPRESS_APPEND) return false;
   size_t off = 256;  // error word, prologue ticket, spare
   auto take = [&](size_t bytes) {
     const size_t at = off;
     off += align256(bytes);
     return at;
   };
+  if (prefill) {
+    w.cap = std::max(1, max_len / QSA_BLOCK);
+    w.qrot = take((size_t)rows * HI * D * 2);
+    w.pf_scale = take((size_t)rows * 4);
+    w.pf_cand_n = take((size_t)rows * 4);
+    w.pf_thr = take((size_t)rows * 4);
+    w.pf_ovf_n = take(4);
+    w.pf_ovf_list = take((size_t)rows * 4);
+    w.cand_key = take((size_t)rows * w.cap * 4);
+    w.cand_id = take((size_t)rows * w.cap * 4);
+    w.total = off;
+    return true;
+  }
   w.cnt_gqa = take(sizeof(int) * (size_t)rows);
   if (scorer) {
     scorer_sizing(max_len, w.ppc_min, w.seg_cap);
@@ -162,7 +178,13 @@ struct ProfScope {
   }
 };
 
-qsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QSA_OK : QSA_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+qsa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QSA_OK;
+  g_last_cuda_error = e;
+  return QSA_ERR_CUDA;
+}
 
 // Prologue (rotation, decode append, page offsets) and scorer, shared by
 // qsa_decode and qsa_index_score_topk.
@@ -178,7 +200,7 @@ qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_b
     cudaError_t e = launch_index_prologue(cv, knew, idx_q, row_req, row_len, len_offset, rows, max_len, fr, qrot,
                                           at<int32_t>(ws, L.row_pages), at<int32_t>(ws, L.page_off),
                                           at<int>(ws, WS_TICKET), err, st);
-    if (e != cudaSuccess) return QSA_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
   }
   ScoreParams p;
   p.c = cv;
@@ -210,6 +232,10 @@ qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_b
 extern "C" {
 
 const char* qsa_version(void) { return "qsa-b200 0.1 (sm_100a)"; }
+
+const char* qsa_last_error_string(void) {
+  return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char* qsa_status_string(qsa_status s) {
   switch (s) {
@@ -284,6 +310,42 @@ qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const
   if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
   return run_indexer(cache, view_of(cache), nullptr, static_cast<const __nv_bfloat16*>(idx_q), q_req, q_pos, 1, nq,
                      max_len, w, blocks, nblocks, ws, L, static_cast<cudaStream_t>(stream));
+}
+
+qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, int32_t req,
+                                  int32_t pos0, int32_t T, int32_t* blocks, int32_t* nblocks, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  qsa_status s = check_cache(cache);
+  if (s != QSA_OK) return s;
+  if (T < 0 || pos0 < 0 || (int64_t)pos0 + T > QSA_MAX_CONTEXT) return QSA_ERR_INVALID_ARG;
+  if (T == 0) return QSA_OK;
+  if (req < 0 || req >= cache->batch) return QSA_ERR_INVALID_ARG;
+  if ((int64_t)pos0 + T > (int64_t)cache->max_pages * QSA_PAGE_SIZE) return QSA_ERR_INVALID_ARG;
+  if (!idx_q || !w || !blocks || !nblocks) return QSA_ERR_INVALID_ARG;
+  if (!aligned(idx_q, 16) || !aligned(w, 16)) return QSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!layout(QSA_OP_PREFILL_SCORE_TOPK, T, pos0 + T, L)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
+  PrefillParams p;
+  p.c = view_of(cache);
+  p.req = req;
+  p.pos0 = pos0;
+  p.T = T;
+  p.w = w;
+  p.qrot = at<__nv_bfloat16>(ws, L.qrot);
+  p.scale = at<float>(ws, L.pf_scale);
+  p.cand_key = at<uint32_t>(ws, L.cand_key);
+  p.cand_id = at<int32_t>(ws, L.cand_id);
+  p.cap = L.cap;
+  p.cand_n = at<int32_t>(ws, L.pf_cand_n);
+  p.thr_bin = at<int32_t>(ws, L.pf_thr);
+  p.sel = blocks;
+  p.sel_n = nblocks;
+  p.ovf_n = at<int>(ws, L.pf_ovf_n);
+  p.ovf_list = at<int32_t>(ws, L.pf_ovf_list);
+  p.err = at<int>(ws, WS_ERR);
+  return cuda_status(launch_prefill(p, static_cast<const __nv_bfloat16*>(idx_q), make_freqs(cache->rope_theta),
+                                    num_sms(), static_cast<cudaStream_t>(stream)));
 }
 
 qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, const int32_t* q_pos, int32_t nq,

@@ -86,4 +86,28 @@ int gqa_split_bound(int rows, int max_pos);
 // Chooses the split count (one wave of resident CTAs, at most split_bound) and launches.
 cudaError_t launch_gqa(const GqaParams& p, int rows, int max_pos, int num_sms, int split_bound, cudaStream_t st);
 
+// ---- prefill scorer on tcgen05 (qsa_prefill.cu) ----
+struct PrefillParams {
+  CacheView c;
+  int req;                 // request of the chunk
+  int pos0;                // position of the chunk's first query
+  int T;                   // queries (positions pos0 .. pos0+T-1)
+  const float* w;          // [T][4] head weights (16-byte aligned)
+  __nv_bfloat16* qrot;     // [T*4][128] rotated index queries (written by the rotation kernel)
+  float* scale;            // [T] histogram scale per query
+  uint32_t* cand_key;      // [T][cap]
+  int32_t* cand_id;        // [T][cap]
+  int cap;                 // candidates per query (>= visible blocks of the last query)
+  int32_t* cand_n;         // [T]
+  int32_t* thr_bin;        // [T]
+  int32_t* sel;            // [T][512] out
+  int32_t* sel_n;          // [T] out
+  int* ovf_n;              // overflow list length
+  int32_t* ovf_list;       // [T]
+  int* err;
+};
+
+cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,
+                           cudaStream_t st);
+
 }  // namespace qsa

@@ -105,7 +105,8 @@ typedef enum {
   QSA_OP_SPARSE_GQA = 2,
   QSA_OP_DECODE = 3,
   QSA_OP_DECODE_INDEXSHARE = 4,
-  QSA_OP_COMPRESS_APPEND = 5
+  QSA_OP_COMPRESS_APPEND = 5,
+  QSA_OP_PREFILL_SCORE_TOPK = 6
 } qsa_op;
 
 /*
@@ -159,6 +160,25 @@ qsa_status qsa_compress_append(const qsa_cache* cache, const void* idx_k_new, co
 qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, const int32_t* q_req,
                                 const int32_t* q_pos, int32_t nq, int32_t max_len, int32_t* blocks,
                                 int32_t* nblocks, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Prefill scoring of one causal chunk on the tensor cores: the queries at
+ * positions pos0 .. pos0+T-1 of request `req` each score their complete
+ * blocks b < floor((pos+1)/4) and keep the top 512.  Same result as
+ * qsa_index_score_topk on those queries; built for long chunks, where the
+ * chunk's queries share every compressed-key tile.
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
+ * (prefill: a GPU kernel computes the index scores, a fast top-k selects).
+ *   idx_q     bf16 [T][4][128] unrotated index queries
+ *   w         f32  [T][4] head weights, 16-byte aligned
+ *   req, pos0 host values; the cache must already hold the chunk's blocks
+ *             (qsa_compress_append of positions up to pos0+T-1)
+ *   blocks    int32 [T][512] out, ascending; nblocks int32 [T] out
+ *   ws        workspace of qsa_workspace_bytes(QSA_OP_PREFILL_SCORE_TOPK, T, pos0+T)
+ */
+qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, int32_t req,
+                                  int32_t pos0, int32_t T, int32_t* blocks, int32_t* nblocks, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * Expand kept blocks to token positions: block b -> 4b..4b+3 in block order,
@@ -284,6 +304,8 @@ void qsa_set_profile_events(void* const* events, int32_t n_pairs);
 int32_t qsa_decode_kernel_count(void);
 
 const char* qsa_status_string(qsa_status s);
+/* Text of the CUDA error behind the calling thread's last QSA_ERR_CUDA. */
+const char* qsa_last_error_string(void);
 const char* qsa_version(void);
 
 #ifdef __cplusplus
