@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--batch", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-scorer measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     return ap.parse_args()
 
@@ -300,12 +301,78 @@ def run_ours(args, rank, world, local_rank):
             "wall_s_timed_region": round(wall, 3),
             "setup_s": round(setup_s, 1),
         }
-    # free device memory before the CPU baseline
+    # free device memory before the secondary measurement and the CPU baseline
     del cache, ws, flush, sess
     torch.cuda.empty_cache()
+    if rank == 0 and not args.no_prefill:
+        res["prefill_scorer"] = run_prefill_scorer(dev)
+        torch.cuda.empty_cache()
     if world > 1:
         dist.destroy_process_group()
     return res, wl
+
+
+def prefill_flops(pos0: int, T: int) -> int:
+    """Algorithmic FLOPs of scoring a causal chunk: 4 heads x 128 dims x 2 per visible (query, block) pair."""
+    t = np.arange(pos0, pos0 + T, dtype=np.int64)
+    return int(((t + 1) // 4).sum()) * 4 * 128 * 2
+
+
+def run_prefill_scorer(dev, reps: int = 20):
+    """Time the tensor-core prefill scorer on the 32768-token causal chunk (every token a query)."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+    import qsa_gen as G
+
+    wl = G.prefill_32k()
+    T = 32768
+    cache = W.build_cache(wl, device=dev, prefix_tokens=[T])
+    idx_q = W.bits_to_bf16(wl.idx_q(0, 0, T), dev)
+    w = torch.from_numpy(wl.w(0, 0, T)).to(dev)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, T), device=dev)
+    blocks = torch.empty(T, 512, dtype=torch.int32, device=dev)
+    nblocks = torch.empty(T, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        Q.prefill_score_topk(cache, idx_q, w, 0, 0, ws, blocks, nblocks)
+    torch.cuda.synchronize()
+    if ws.device_error() != 0:
+        raise RuntimeError("device error word set in the prefill scorer")
+    st = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(reps)]
+    for e in ev:
+        for x in e:
+            x.record(st)
+    torch.cuda.synchronize()
+    for k in range(reps):
+        flush.zero_()
+        Q.set_profile_events(ev[k])
+        Q.prefill_score_topk(cache, idx_q, w, 0, 0, ws, blocks, nblocks)
+    Q.set_profile_events(None)
+    torch.cuda.synchronize()
+    ms = [[ev[k][2 * i].elapsed_time(ev[k][2 * i + 1]) for k in range(reps)] for i in range(3)]
+    total = [ev[k][0].elapsed_time(ev[k][5]) for k in range(reps)]
+    flops = prefill_flops(0, T)
+    score_s = float(np.mean(ms[1])) * 1e-3
+    peak = 1590.0
+    src = "fallback 1.59 PFLOP/s"
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        peak = float(json.load(open(pk))["bf16_tflops"])
+        src = "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+    ach = flops / score_s / 1e12
+    return {
+        "workload": "prefill_L32768 (one causal chunk of 32768 queries)",
+        "call_us": round(float(np.mean(total)) * 1e3, 2),
+        "kernels_us": {"rotate": round(float(np.mean(ms[0])) * 1e3, 2), "score_tcgen05": round(score_s * 1e6, 2),
+                       "finalize": round(float(np.mean(ms[2])) * 1e3, 2)},
+        "query_tok_per_s": round(T / (float(np.mean(total)) * 1e-3), 1),
+        "roofline": {"kernel": "k_prefill_score", "bound": "tensor", "achieved": round(ach, 1), "peak": peak,
+                     "peak_source": src, "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                     "algorithmic_flops_per_launch": flops},
+    }
 
 
 def oracle_sample_step(wl, reqs, nthreads):

@@ -344,8 +344,10 @@ qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, con
   p.ovf_n = at<int>(ws, L.pf_ovf_n);
   p.ovf_list = at<int32_t>(ws, L.pf_ovf_list);
   p.err = at<int>(ws, WS_ERR);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
   return cuda_status(launch_prefill(p, static_cast<const __nv_bfloat16*>(idx_q), make_freqs(cache->rope_theta),
-                                    num_sms(), static_cast<cudaStream_t>(stream)));
+                                    num_sms(), static_cast<cudaStream_t>(stream), g_prof_pairs ? g_prof : nullptr,
+                                    g_prof_pairs));
 }
 
 qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, const int32_t* q_pos, int32_t nq,

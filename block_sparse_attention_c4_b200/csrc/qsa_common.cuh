@@ -331,6 +331,10 @@ __device__ SelectResult radix_select(KeyAt key_at, int n, int k, SelectScratch* 
       const unsigned peers = __match_any_sync(0xffffffffu, dg);
       if (valid && lane == __ffs(peers) - 1) atomicAdd(&sc->hist[dg], __popc(peers));
     }
+    if (tid == 0) {  // defaults, in case no digit qualifies (k larger than the keys left)
+      sc->digit = 0;
+      sc->above = 0;
+    }
     G::sync();
     // thread t owns the digits bins-1-t*per .. bins-per-t*per (descending)
     const int per = (bins + NT - 1) / NT;
@@ -469,6 +473,10 @@ __device__ void fast_topk(KeyAt key_at, int n, int k, Emit emit, FastTopScratch*
     for (int i = tid; i < bins; i += NT) sc->hist[i] = 0;
     G::sync();
     for (int i = tid; i < n; i += NT) atomicAdd(&sc->hist[bin_of(key_at(i))], 1);
+    if (tid == 0) {  // defaults, in case no bin qualifies
+      sc->digit = 0;
+      sc->above = 0;
+    }
     G::sync();
     constexpr int per = (bins + NT - 1) / NT;  // thread t owns bins bins-1-t*per .. (descending)
     int local = 0;

@@ -107,7 +107,8 @@ struct PrefillParams {
   int* err;
 };
 
+// ev (nullable): n_ev event pairs recorded around the rotation, scoring and finalize kernels.
 cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,
-                           cudaStream_t st);
+                           cudaStream_t st, const cudaEvent_t* ev, int n_ev);
 
 }  // namespace qsa

@@ -50,8 +50,8 @@ constexpr int PF_A_BYTES = PF_M * D * 2;  // 32 KiB
 constexpr int PF_B_BYTES = PF_N * D * 2;  // 64 KiB
 constexpr uint32_t PF_TMEM_COLS = 512;
 
-struct PfQuery {
-  float w[4];
+struct __align__(16) PfQuery {
+  float4 w;     // head weights
   float theta;  // admit s > theta
   float scale;  // score -> histogram scale
   int nbv;      // visible complete blocks
@@ -66,7 +66,7 @@ struct __align__(1024) PfSmem {
   int count[2][PF_QT];
   int acnt[PF_QT];
   int new_ge[PF_QT];
-  uint32_t masks[2][32][4];
+  uint32_t masks[2][4][32];  // [half][quadrant][query of the half]
   uint64_t full_a[PF_STAGES], empty_a[PF_STAGES], full_b, empty_b, tfull[2], tempty[2];
   uint32_t tmem_base;
 };
@@ -109,7 +109,7 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 }
 
 // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major.
-constexpr uint32_t pf_idesc() {
+__host__ __device__ constexpr uint32_t pf_idesc() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PF_N >> 3) << 17) | ((uint32_t)(PF_M >> 4) << 24);
 }
 
@@ -272,15 +272,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int t = qt * PF_QT + etid;
         PfQuery qi;
         if (t < p.T) {
-          const float4 w4 = __ldg(reinterpret_cast<const float4*>(p.w) + t);
-          qi.w[0] = w4.x;
-          qi.w[1] = w4.y;
-          qi.w[2] = w4.z;
-          qi.w[3] = w4.w;
+          qi.w = __ldg(reinterpret_cast<const float4*>(p.w) + t);
           qi.scale = __ldg(p.scale + t);
           qi.nbv = sch.nbv_of(t);
         } else {
-          qi.w[0] = qi.w[1] = qi.w[2] = qi.w[3] = 0.f;
+          qi.w = make_float4(0.f, 0.f, 0.f, 0.f);
           qi.scale = 1.f;
           qi.nbv = 0;
         }
@@ -299,79 +295,117 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         tc_fence_after();
         const int b = mt * PF_M + quad * 32 + lane;  // this thread's block
         float sc[32];
-        uint32_t my_masks = 0;  // lane i: mask of query 32*half + i (for the leader's bookkeeping)
+        uint32_t my_masks = 0;  // lane i: this quadrant's admission mask of query 32*half + i
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint32_t r[32];
-          tc_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * PF_N + half * 128 + g * 32), r);
+        for (int g2 = 0; g2 < 2; ++g2) {
+          uint32_t r[2][32];
+          const uint32_t col = (uint32_t)(buf * PF_N + half * 128 + g2 * 64);
+          const uint32_t lanes = (uint32_t)(quad * 32) << 16;
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+              "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+              : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[0][4]), "=r"(r[0][5]),
+                "=r"(r[0][6]), "=r"(r[0][7]), "=r"(r[0][8]), "=r"(r[0][9]), "=r"(r[0][10]), "=r"(r[0][11]),
+                "=r"(r[0][12]), "=r"(r[0][13]), "=r"(r[0][14]), "=r"(r[0][15]), "=r"(r[0][16]), "=r"(r[0][17]),
+                "=r"(r[0][18]), "=r"(r[0][19]), "=r"(r[0][20]), "=r"(r[0][21]), "=r"(r[0][22]), "=r"(r[0][23]),
+                "=r"(r[0][24]), "=r"(r[0][25]), "=r"(r[0][26]), "=r"(r[0][27]), "=r"(r[0][28]), "=r"(r[0][29]),
+                "=r"(r[0][30]), "=r"(r[0][31])
+              : "r"(tmem + lanes + col));
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+              "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+              : "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]), "=r"(r[1][3]), "=r"(r[1][4]), "=r"(r[1][5]),
+                "=r"(r[1][6]), "=r"(r[1][7]), "=r"(r[1][8]), "=r"(r[1][9]), "=r"(r[1][10]), "=r"(r[1][11]),
+                "=r"(r[1][12]), "=r"(r[1][13]), "=r"(r[1][14]), "=r"(r[1][15]), "=r"(r[1][16]), "=r"(r[1][17]),
+                "=r"(r[1][18]), "=r"(r[1][19]), "=r"(r[1][20]), "=r"(r[1][21]), "=r"(r[1][22]), "=r"(r[1][23]),
+                "=r"(r[1][24]), "=r"(r[1][25]), "=r"(r[1][26]), "=r"(r[1][27]), "=r"(r[1][28]), "=r"(r[1][29]),
+                "=r"(r[1][30]), "=r"(r[1][31])
+              : "r"(tmem + lanes + col + 32u));
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int qq = 0; qq < 8; ++qq) {
-            const int jq = half * 32 + g * 8 + qq;
-            const PfQuery& qi = S.q[jq];
-            float s = qi.w[0] * fmaxf(__uint_as_float(r[4 * qq + 0]), 0.f);
-            s = fmaf(qi.w[1], fmaxf(__uint_as_float(r[4 * qq + 1]), 0.f), s);
-            s = fmaf(qi.w[2], fmaxf(__uint_as_float(r[4 * qq + 2]), 0.f), s);
-            s = fmaf(qi.w[3], fmaxf(__uint_as_float(r[4 * qq + 3]), 0.f), s);
-            sc[g * 8 + qq] = s;
-            const bool admit = s > qi.theta && b < qi.nbv;
+          for (int qq = 0; qq < 16; ++qq) {
+            const int jl = g2 * 16 + qq;  // query of the half
+            const PfQuery* qp = &S.q[half * 32 + jl];
+            const float4 w4 = qp->w;
+            const float4 tz = *reinterpret_cast<const float4*>(&qp->theta);  // theta, scale, nbv, D
+            const uint32_t* rr = &r[qq >> 3][4 * (qq & 7)];
+            float s = w4.x * fmaxf(__uint_as_float(rr[0]), 0.f);
+            s = fmaf(w4.y, fmaxf(__uint_as_float(rr[1]), 0.f), s);
+            s = fmaf(w4.z, fmaxf(__uint_as_float(rr[2]), 0.f), s);
+            s = fmaf(w4.w, fmaxf(__uint_as_float(rr[3]), 0.f), s);
+            sc[jl] = s;
+            const bool admit = s > tz.x && b < __float_as_int(tz.z);
             const uint32_t m = __ballot_sync(0xffffffffu, admit);
-            if (lane == g * 8 + qq) my_masks = m;
+            if (lane == jl) my_masks = m;
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.tempty[buf]);
-        S.masks[half][lane][quad] = my_masks;
+        S.masks[half][quad][lane] = my_masks;
         asm volatile("bar.sync %0, 128;" ::"r"(bar_half) : "memory");
 
         // ---- ordered append: quadrant q's blocks follow quadrants < q ----
+        // lane i prepares query 32*half + i: its masks, this warp's base offset, scale and D
         const int cur = mt & 1;
-        uint32_t any = 0, total_l = 0;
+        const int jq_l = half * 32 + lane;
+        uint32_t total_l, base_l;
         {
-          const uint32_t m0 = S.masks[half][lane][0], m1 = S.masks[half][lane][1];
-          const uint32_t m2 = S.masks[half][lane][2], m3 = S.masks[half][lane][3];
-          total_l = __popc(m0) + __popc(m1) + __popc(m2) + __popc(m3);
-          any = __ballot_sync(0xffffffffu, total_l != 0);
+          const uint32_t m0 = S.masks[half][0][lane], m1 = S.masks[half][1][lane];
+          const uint32_t m2 = S.masks[half][2][lane], m3 = S.masks[half][3][lane];
+          const uint32_t p0 = __popc(m0), p1 = __popc(m1), p2 = __popc(m2), p3 = __popc(m3);
+          total_l = p0 + p1 + p2 + p3;
+          base_l = (uint32_t)S.count[cur][jq_l] + (quad > 0 ? p0 : 0u) + (quad > 1 ? p1 : 0u) + (quad > 2 ? p2 : 0u);
         }
+        const float scale_l = S.q[jq_l].scale;
+        const int D_l = S.q[jq_l].D;
+        const uint32_t any = __ballot_sync(0xffffffffu, my_masks != 0);
+        const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (!(any & (1u << i))) continue;
+          const uint32_t mq = __shfl_sync(0xffffffffu, my_masks, i);
+          const int base = (int)__shfl_sync(0xffffffffu, base_l, i);
+          const float scale = __shfl_sync(0xffffffffu, scale_l, i);
+          const int Dq = __shfl_sync(0xffffffffu, D_l, i);
+          const bool mine = (mq >> lane) & 1u;
           const int jq = half * 32 + i;
-          const uint32_t mq = S.masks[half][i][quad];
-          if (!(mq & (1u << lane))) continue;
-          int before = 0;
-          for (int qd = 0; qd < quad; ++qd) before += __popc(S.masks[half][i][qd]);
-          const int pos = S.count[cur][jq] + before + __popc(mq & ((1u << lane) - 1u));
           const int t = qt * PF_QT + jq;
+          const int pos = base + __popc(mq & lt);
           const float s = sc[i];
-          if (t >= p.T || pos >= p.cap) {  // cannot happen: each visible block is admitted once per query
-            set_error(p.err, QSA_DEVERR_SELECTION);
-            continue;
+          int bin = -1;
+          if (mine) {
+            if (t < p.T && pos < p.cap) {
+              p.cand_key[(int64_t)t * p.cap + pos] = score_key(s);
+              p.cand_id[(int64_t)t * p.cap + pos] = b;
+            } else {  // cannot happen: each visible block is admitted once per query
+              set_error(p.err, QSA_DEVERR_SELECTION);
+            }
+            bin = pf_bin(s, scale);
+            if (bin < Dq) bin = -1;  // admitted on an older threshold: not counted
           }
-          p.cand_key[(int64_t)t * p.cap + pos] = score_key(s);
-          p.cand_id[(int64_t)t * p.cap + pos] = b;
-          const PfQuery& qi = S.q[jq];
-          const int bin = pf_bin(s, qi.scale);
-          if (bin >= qi.D) {
-            atomicAdd(&S.hist[jq][bin], 1);
-            atomicAdd(&S.new_ge[jq], 1);
+          const uint32_t counted = __ballot_sync(0xffffffffu, bin >= 0);
+          if (counted) {
+            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+            if (bin >= 0 && (peers & lt) == 0) atomicAdd(&S.hist[jq][bin], __popc(peers));
+            if (lane == 0) atomicAdd(&S.new_ge[jq], __popc(counted));
           }
         }
         asm volatile("bar.sync %0, 128;" ::"r"(bar_half) : "memory");
         if (leader) {  // lane i: query 32*half + i
-          const int jq = half * 32 + lane;
+          const int jq = jq_l;
           S.count[cur ^ 1][jq] = S.count[cur][jq] + (int)total_l;
           int a = S.acnt[jq] + S.new_ge[jq];
           S.new_ge[jq] = 0;
-          int Dq = S.q[jq].D;
+          int Dq = D_l;
           while (Dq < PF_BINS - 1 && a - S.hist[jq][Dq] >= TOPK) {
             a -= S.hist[jq][Dq];
             ++Dq;
           }
           S.acnt[jq] = a;
-          if (Dq != S.q[jq].D) {
+          if (Dq != D_l) {
             S.q[jq].D = Dq;
-            S.q[jq].theta = pf_theta(Dq, S.q[jq].scale);
+            S.q[jq].theta = pf_theta(Dq, scale_l);
           }
         }
       }
@@ -498,6 +532,10 @@ __global__ void __launch_bounds__(256) k_prefill_overflow(PrefillParams p) {
   for (int o = blockIdx.x; o < nov; o += gridDim.x) {
     const int t = p.ovf_list[o];
     const int n = min(p.cand_n[t], p.cap);
+    if (n <= 0) {
+      if (threadIdx.x == 0) p.sel_n[t] = 0;
+      continue;
+    }
     const uint32_t* keys = p.cand_key + (int64_t)t * p.cap;
     const int32_t* ids = p.cand_id + (int64_t)t * p.cap;
     int32_t* sel = p.sel + (int64_t)t * TOPK;
@@ -581,7 +619,10 @@ static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,
-                           cudaStream_t st) {
+                           cudaStream_t st, const cudaEvent_t* ev, int n_ev) {
+  auto mark = [&](int i) {
+    if (ev && i < 2 * n_ev) cudaEventRecord(ev[i], st);
+  };
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -594,16 +635,22 @@ cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, c
   CUtensorMap kmap, qmap;
   if (!make_map(&kmap, p.c.cidx, (uint64_t)p.c.num_pages * PAGE_BLOCKS, PAGE_BLOCKS)) return cudaErrorInvalidValue;
   if (!make_map(&qmap, p.qrot, (uint64_t)p.T * HI, PF_N)) return cudaErrorInvalidValue;
+  mark(0);
   k_prefill_rotate<<<p.T, 128, 0, st>>>(p, idx_q, fr);
+  mark(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(p.T, PF_QT);
+  mark(2);
   k_prefill_score<<<std::min(num_sms, tiles), PF_THREADS, smem, st>>>(p, kmap, qmap);
+  mark(3);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.ovf_n, 0, sizeof(int), st)) != cudaSuccess) return e;
+  mark(4);
   k_prefill_finalize<<<ceil_div(p.T, PF_FIN_WARPS), PF_FIN_WARPS * 32, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   k_prefill_overflow<<<std::min(p.T, 4 * num_sms), 256, 0, st>>>(p);
+  mark(5);
   return cudaGetLastError();
 }
 

@@ -295,7 +295,8 @@ int32_t qsa_device_error(void* ws, int32_t clear, void* stream);
 /*
  * Measurement hook: when `events` is non-NULL, qsa_decode records
  * events[2*i] before and events[2*i+1] after its i-th kernel (i < n_pairs)
- * on its stream.  Each entry is a cudaEvent_t.  Pass NULL to switch it off.
+ * on its stream; qsa_prefill_score_topk does the same around its rotation
+ * (i = 0), scoring (i = 1) and finalize (i = 2) kernels.  Each entry is a cudaEvent_t.  Pass NULL to switch it off.
  * Not thread-safe with concurrent qsa_decode calls from several host threads.
  */
 void qsa_set_profile_events(void* const* events, int32_t n_pairs);
