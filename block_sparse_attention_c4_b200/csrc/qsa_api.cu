@@ -24,7 +24,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct WsLayout {
   size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, seg_cnt = 0, cand_cnt = 0,
          pages_done = 0, seg_tab = 0, cand_key = 0, cand_id = 0, part_o = 0, part_ml = 0, total = 0;
-  size_t pf_scale = 0, pf_cand_n = 0, pf_thr = 0, pf_ovf_n = 0, pf_ovf_list = 0;
+  size_t pf_keys = 0, pf_ovf_n = 0, pf_ovf_list = 0;
   int ppc_min = 0;
   int seg_cap = 0;
   int splits_bound = 0;
@@ -65,15 +65,11 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     return at;
   };
   if (prefill) {
-    w.cap = std::max(1, max_len / QSA_BLOCK);
+    w.cap = (std::max(1, max_len / QSA_BLOCK) + 127) / 128 * 128;
     w.qrot = take((size_t)rows * HI * D * 2);
-    w.pf_scale = take((size_t)rows * 4);
-    w.pf_cand_n = take((size_t)rows * 4);
-    w.pf_thr = take((size_t)rows * 4);
+    w.pf_keys = take((size_t)ceil_div(rows, 64) * 64 * w.cap * 4);
     w.pf_ovf_n = take(4);
     w.pf_ovf_list = take((size_t)rows * 4);
-    w.cand_key = take((size_t)rows * w.cap * 4);
-    w.cand_id = take((size_t)rows * w.cap * 4);
     w.total = off;
     return true;
   }
@@ -333,16 +329,12 @@ qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, con
   p.T = T;
   p.w = w;
   p.qrot = at<__nv_bfloat16>(ws, L.qrot);
-  p.scale = at<float>(ws, L.pf_scale);
-  p.cand_key = at<uint32_t>(ws, L.cand_key);
-  p.cand_id = at<int32_t>(ws, L.cand_id);
-  p.cap = L.cap;
-  p.cand_n = at<int32_t>(ws, L.pf_cand_n);
-  p.thr_bin = at<int32_t>(ws, L.pf_thr);
-  p.sel = blocks;
-  p.sel_n = nblocks;
+  p.keys = at<uint32_t>(ws, L.pf_keys);
   p.ovf_n = at<int>(ws, L.pf_ovf_n);
   p.ovf_list = at<int32_t>(ws, L.pf_ovf_list);
+  p.cap = L.cap;
+  p.sel = blocks;
+  p.sel_n = nblocks;
   p.err = at<int>(ws, WS_ERR);
   std::lock_guard<std::mutex> lk(g_prof_mu);
   return cuda_status(launch_prefill(p, static_cast<const __nv_bfloat16*>(idx_q), make_freqs(cache->rope_theta),

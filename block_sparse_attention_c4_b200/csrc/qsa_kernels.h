@@ -94,15 +94,11 @@ struct PrefillParams {
   int T;                   // queries (positions pos0 .. pos0+T-1)
   const float* w;          // [T][4] head weights (16-byte aligned)
   __nv_bfloat16* qrot;     // [T*4][128] rotated index queries (written by the rotation kernel)
-  float* scale;            // [T] histogram scale per query
-  uint32_t* cand_key;      // [T][cap]
-  int32_t* cand_id;        // [T][cap]
-  int cap;                 // candidates per query (>= visible blocks of the last query)
-  int32_t* cand_n;         // [T]
-  int32_t* thr_bin;        // [T]
+  uint32_t* keys;          // [ceil(T/64)][cap/128][64][128] order-preserving score keys of the work tiles
+  int cap;                 // score slots per query: >= visible blocks of the last query, a multiple of 128
   int32_t* sel;            // [T][512] out
   int32_t* sel_n;          // [T] out
-  int* ovf_n;              // overflow list length
+  int* ovf_n;              // rows handed to the overflow selection (zeroed per call)
   int32_t* ovf_list;       // [T]
   int* err;
 };

@@ -51,7 +51,8 @@ def _run(Q, W, wl, pos0, T, rows=None):
     return bl, nbl
 
 
-@pytest.mark.parametrize("pos0,T", [(0, 3000), (0, 64), (0, 2100), (5000, 2000), (4097, 777), (9000, 33)])
+@pytest.mark.parametrize("pos0,T", [(0, 3000), (0, 64), (0, 2100), (5000, 2000), (4097, 777), (9000, 33),
+                                    (40000, 300)])
 def test_prefill_scorer_matches_oracle_every_row(Q, W, pos0, T):
     wl = G.custom_decode(41 + T, [pos0 + T])
     _run(Q, W, wl, pos0, T)
@@ -97,3 +98,42 @@ def test_prefill_scorer_32k(Q, W):
         b = bl[i, :nbl[i]]
         assert nbl[i] == min(nb, 512)
         assert np.all(np.diff(b) > 0) and (nbl[i] == 0 or b[-1] < nb)
+
+
+def test_prefill_heavy_ties(Q, W):
+    """Thousands of bit-identical compressed keys: every query keeps the tied blocks with the lowest
+    indices, for rows held in shared memory (3000 blocks) and rows read through L2 (20000 blocks)."""
+    for nb in (3000, 20000):
+        L = 4 * nb
+        T = 40
+        wl = G.custom_decode(31, [L])
+        cache = W.build_cache(wl, prefix_tokens=[0])
+        rng = np.random.default_rng(nb + 1)
+        a = rng.standard_normal(128)
+        b = 0.3 * a + rng.standard_normal(128)
+
+        def bits(v):  # unit vector -> bf16 bits
+            t = torch.from_numpy((v / np.linalg.norm(v)).astype(np.float32)).to(torch.bfloat16)
+            return t.view(torch.int16).numpy().view(np.uint16)
+
+        keys = np.empty((nb, 128), dtype=np.uint16)
+        keys[:] = bits(b)
+        keys[::50] = bits(a)
+        pt = wl.page_table()[0]
+        blk = np.arange(nb)
+        entries = (pt[(4 * blk) // 64].astype(np.int64) * 64 + (4 * blk) % 64) // 4
+        cache.cidx[torch.from_numpy(entries).cuda()] = W.bits_to_bf16(keys, "cuda")
+        idx_q = np.repeat(np.repeat(bits(a)[None, :], 4, axis=0)[None], T, axis=0)
+        w = np.tile(np.array([[0.5, 0.25, 0.125, 1.0]], dtype=np.float32), (T, 1))
+        pos0 = L - T
+        ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, L))
+        blocks, nblocks = Q.prefill_score_topk(cache, W.bits_to_bf16(idx_q, "cuda"), torch.from_numpy(w).cuda(), 0,
+                                               pos0, ws)
+        torch.cuda.synchronize()
+        assert ws.device_error() == 0
+        bl, nbl = blocks.cpu().numpy(), nblocks.cpu().numpy()
+        for i in range(0, T, 3):
+            t = pos0 + i
+            ob, _, s = O.select_query(idx_q[i], w[i], keys[:(t + 1) // 4], t + 1)
+            assert len(np.unique(s)) <= 2 and nbl[i] == 512
+            np.testing.assert_array_equal(bl[i], ob)
