@@ -220,7 +220,7 @@ qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_b
   p.sel_n = sel_n;
   p.err = err;
   ProfScope ps(st, 1);
-  return cuda_status(launch_score_topk(p, score_grid(num_sms()), st));
+  return cuda_status(launch_score_topk(p, num_sms(), st));
 }
 
 }  // namespace

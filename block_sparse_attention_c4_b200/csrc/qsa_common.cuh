@@ -101,6 +101,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first A-aligned byte of the dynamic shared memory `raw`, derived by pointer arithmetic so
+// that the compiler still knows every access through it to be a shared-memory access (rounding
+// the address as an integer would turn them all into slower generic loads, stores and atomics).
+template <int A>
+__device__ __forceinline__ uint8_t* smem_aligned(uint8_t* raw) {
+  return raw + ((A - (smem_u32(raw) & (A - 1))) & (A - 1));
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -562,6 +570,192 @@ __device__ void fast_topk(KeyAt key_at, int n, int k, Emit emit, FastTopScratch*
     const unsigned m = __ballot_sync(0xffffffffu, kp);
     if (kp) emit(i, out + __popc(m & ((1u << lane) - 1u)));
     out += __popc(m);
+  }
+  G::sync();
+}
+
+// ---------------------------------------------------------------------------
+// Exact top-k of n <= HT_MAX_N keys in shared memory whose histogram was
+// built while the keys were produced (ht_count, by the producing warps):
+// bins are the top HT_BITS bits of the order-preserving key, i.e. a
+// log-scale histogram of the scores (1/16 octave).  The selection then takes
+// four light steps and a single pass over the keys:
+//   (1) a scan of the histogram finds the bin D holding the k-th key;
+//   (2) one pass writes, per 32 consecutive keys, the ballot of the keys in
+//       bins above D as one word of a keep bitmap, and puts the keys of bin D
+//       into the warp's own tie list (no atomics);
+//   (3) the ties are ranked by (key desc, index asc); the first `need` set
+//       their bits;
+//   (4) a popcount prefix over the bitmap words emits the kept indices in
+//       ascending order.
+// Every loop loads several independent values before using any of them:
+// with a few warps per SM the selection is bound by latency, not work.
+// Bins hold 16-bit counts, two per word (n <= 8192 never overflows one).
+// If one warp finds more ties than its list holds, the ties are gathered
+// again with a shared counter; more than HT_TIE_CAP ties in all (heavily
+// tied keys) fall back to radix_select / select_compact, which borrow the
+// histogram's storage.  Emit(i, o): kept index i, output slot o in [0, k),
+// called after the last read of `keys`; requires k <= n.
+// ---------------------------------------------------------------------------
+constexpr int HT_BITS = 13;
+constexpr int HT_BINS = 1 << HT_BITS;  // 8192 bins
+constexpr int HT_WORDS = HT_BINS / 2;  // 4096 words of two 16-bit counts
+constexpr int HT_MAX_N = 8192;
+constexpr int HT_TIE_CAP = 256;
+
+struct HistTopScratch {
+  int warp_tot[33];
+  int D, above, tie_n;
+  int tie_cnt[32];  // ties found by each warp
+  uint32_t bits[HT_MAX_N / 32];
+  // ties of the cut bin as one comparable word: key in the high half, bitwise-inverted index in the
+  // low half, so a larger value ranks first under (key desc, index asc).  The warps' lists fill
+  // the first half; the second half holds them packed for ranking.
+  unsigned long long tie[2 * HT_TIE_CAP];
+};
+
+__device__ __forceinline__ int ht_bin(uint32_t key) { return (int)(key >> (32 - HT_BITS)); }
+
+// Counts one key (any thread, any order).
+__device__ __forceinline__ void ht_count(uint32_t* hist, uint32_t key) {
+  const int b = ht_bin(key);
+  atomicAdd(hist + (b >> 1), 1u << ((b & 1) * 16));
+}
+
+template <class G>
+__device__ __forceinline__ void ht_zero(uint32_t* hist) {
+  for (int i = threadIdx.x; i < HT_WORDS / 4; i += G::N) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+}
+
+__device__ __forceinline__ unsigned long long ht_tie_word(uint32_t key, int i) {
+  return ((unsigned long long)key << 32) | (uint32_t)~i;
+}
+
+template <class G, typename Emit>
+__device__ void hist_topk(const uint32_t* keys, uint32_t* hist, int n, int k, Emit emit, HistTopScratch* sc) {
+  constexpr int NT = G::N, NW = NT / 32;
+  constexpr int PER = HT_BINS / NT;  // bins per thread
+  constexpr int WCAP = HT_TIE_CAP / NW;
+  static_assert(PER % 8 == 0 && HT_MAX_N / 32 <= NT, "layout");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // (1) thread t owns bins top-PER*t-PER+1 .. top-PER*t (descending order of ownership)
+  const int lo_bin = HT_BINS - PER * (tid + 1);
+  uint32_t cw[PER / 2];
+#pragma unroll
+  for (int q = 0; q < PER / 8; ++q) {
+    const uint4 v = reinterpret_cast<const uint4*>(hist + lo_bin / 2)[q];
+    cw[4 * q] = v.x;
+    cw[4 * q + 1] = v.y;
+    cw[4 * q + 2] = v.z;
+    cw[4 * q + 3] = v.w;
+  }
+  int local = 0;
+#pragma unroll
+  for (int q = 0; q < PER / 2; ++q) local += (int)(cw[q] & 0xFFFFu) + (int)(cw[q] >> 16);
+  if (tid == 0) {
+    sc->D = -1;
+    sc->above = 0;
+    sc->tie_n = 0;
+  }
+  if (tid < HT_MAX_N / 32) sc->bits[tid] = 0u;
+  int tot;
+  const int ex = group_exclusive_scan<G>(local, sc->warp_tot, &tot);  // keys in bins above this thread's
+  if (ex < k && ex + local >= k) {
+    int c = ex;
+#pragma unroll
+    for (int q = PER - 1; q >= 0; --q) {
+      const int h = (int)((cw[q >> 1] >> ((q & 1) * 16)) & 0xFFFFu);
+      if (c + h >= k) {
+        sc->D = lo_bin + q;
+        sc->above = c;
+        break;
+      }
+      c += h;
+    }
+  }
+  G::sync();
+  const int D = sc->D;
+  const int need = k - sc->above;
+  // (2) one pass: keep-bitmap words for bins above D, ties of bin D into the warp's own list.
+  // Warp w takes words w, w + NW, ...; four words' keys are loaded before any of them is used.
+  unsigned long long* wtie = sc->tie + warp * WCAP;
+  unsigned long long* packed = sc->tie + HT_TIE_CAP;
+  int nt = 0;  // warp-uniform
+  const int nwords = (n + 31) >> 5;
+  for (int wd0 = warp; wd0 < nwords; wd0 += 4 * NW) {
+    uint32_t key[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = (wd0 + u * NW) * 32 + lane;
+      key[u] = i < n ? keys[i] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int wd = wd0 + u * NW;
+      const int i = wd * 32 + lane;
+      const int b = ht_bin(key[u]);
+      const unsigned def = __ballot_sync(0xffffffffu, i < n && b > D);
+      const unsigned tie = __ballot_sync(0xffffffffu, i < n && b == D);
+      if (lane == 0 && wd < nwords) sc->bits[wd] = def;
+      if (tie & (1u << lane)) {
+        const int pos = nt + __popc(tie & ((1u << lane) - 1u));
+        if (pos < WCAP) wtie[pos] = ht_tie_word(key[u], i);
+      }
+      nt += __popc(tie);
+    }
+  }
+  if (lane == 0) sc->tie_cnt[warp] = nt;
+  G::sync();
+  int m = 0, over = 0, before = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int c = sc->tie_cnt[w];
+    before += w < warp ? c : 0;
+    m += c;
+    over |= c > WCAP;
+  }
+  if (m > HT_TIE_CAP) {  // heavily tied keys: exact radix refinement (the histogram is free now)
+    SelectScratch* ss = reinterpret_cast<SelectScratch*>(hist);
+    auto key_at = [&](int i) { return keys[i]; };
+    const SelectResult r = radix_select<G>(key_at, n, k, ss);
+    select_compact<G>(key_at, n, r, emit, ss);
+    return;
+  }
+  if (over) {  // one warp's list overflowed: gather the ties again with a shared counter
+    for (int i = tid; i < n; i += NT) {
+      const uint32_t key = keys[i];
+      if (ht_bin(key) == D) packed[atomicAdd(&sc->tie_n, 1)] = ht_tie_word(key, i);
+    }
+  } else {
+    for (int c = lane; c < nt; c += 32) packed[before + c] = wtie[c];
+  }
+  G::sync();
+  // (3) exact order inside bin D: a tie is kept when fewer than `need` ties rank above it
+  for (int a = tid; a < m; a += NT) {
+    const unsigned long long va = packed[a];
+    int rank = 0;
+    int c = 0;
+    for (; c + 8 <= m; c += 8) {
+      unsigned long long vc[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) vc[u] = packed[c + u];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) rank += vc[u] > va;
+    }
+    for (; c < m; ++c) rank += packed[c] > va;
+    if (rank < need) {
+      const int ia = (int)~(uint32_t)va;
+      atomicOr(&sc->bits[ia >> 5], 1u << (ia & 31));
+    }
+  }
+  G::sync();
+  // (4) ordered emission
+  uint32_t wbits = tid < nwords ? sc->bits[tid] : 0u;
+  int o = group_exclusive_scan<G>(__popc(wbits), sc->warp_tot, &tot);
+  while (wbits) {
+    const int bit = __ffs(wbits) - 1;
+    emit(tid * 32 + bit, o++);
+    wbits &= wbits - 1u;
   }
   G::sync();
 }

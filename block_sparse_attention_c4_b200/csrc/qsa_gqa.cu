@@ -46,7 +46,7 @@ template <int MT>
 __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   constexpr int THREADS = MT * 128;
   extern __shared__ uint8_t smem_raw[];
-  GqaSmem<MT>& S = *reinterpret_cast<GqaSmem<MT>*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  GqaSmem<MT>& S = *reinterpret_cast<GqaSmem<MT>*>(smem_aligned<128>(smem_raw));
   const int row = blockIdx.y, split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nq = p.nq_row;

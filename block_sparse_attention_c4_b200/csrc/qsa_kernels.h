@@ -48,8 +48,8 @@ struct ScoreParams {
   int* err;
 };
 
-int score_grid(int num_sms);
-cudaError_t launch_score_topk(const ScoreParams& p, int grid, cudaStream_t st);
+// Launches the persistent scorer on every SM (as many CTAs per SM as are resident).
+cudaError_t launch_score_topk(const ScoreParams& p, int num_sms, cudaStream_t st);
 
 // ---- sparse GQA (qsa_gqa.cu) ----
 constexpr int GQ_MAX_SPLITS = 16;

@@ -142,7 +142,7 @@ struct PfSched {
 __global__ void __launch_bounds__(PF_THREADS, 1)
     k_prefill_score(PrefillParams p, const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap) {
   extern __shared__ uint8_t smem_raw[];
-  PfSmem& S = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  PfSmem& S = *reinterpret_cast<PfSmem*>(smem_aligned<1024>(smem_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   PfSched sch{ceil_div(p.T, PF_QT), (int)gridDim.x, p.pos0, p.T};
 

@@ -55,15 +55,24 @@ constexpr int SC_ROWS_SMEM = 512;  // rows whose page offsets are staged in shar
 
 using Cta = Group<SC_THREADS, 0>;
 
+constexpr int SC_MERGE_CAP = SC_SEG_KEYS / 2;  // merge candidates held at once
+
+// Kept small on purpose: the L1 cache shares the SM's memory with this, and the page loads in
+// flight need L1 room (a larger footprint measurably slows the streaming).
 struct ScoreSmem {
-  uint32_t keys[SC_SEG_KEYS];     // a segment's score keys; a merge's candidates
-  int32_t pid[SC_MAX_SEG_PAGES];  // physical pages of the current segment (-1: invalid)
-  int32_t off[SC_ROWS_SMEM + 1];  // exclusive prefix of pages per row
-  int4 segs[SC_MAX_SEGS];         // merge: the row's segments (start block, cand offset, count, -)
-  int vstart[SC_MAX_SEGS + 1];    // merge: prefix of the ordered segments' counts
-  FastTopScratch ft;
+  uint32_t keys[SC_SEG_KEYS];           // a segment's score keys; a merge's candidate keys
+                                        // [0, SC_MERGE_CAP) and block ids [SC_MERGE_CAP, 2 SC_MERGE_CAP)
+  alignas(16) uint32_t hist[HT_WORDS];  // histogram of `keys` (built as they are written)
+  HistTopScratch ht;
+  int32_t pid[SC_MAX_SEG_PAGES];    // physical pages of the current segment (-1: invalid)
+  int32_t off[SC_ROWS_SMEM + 1];    // exclusive prefix of pages per row
+  int4 segs[SC_MAX_SEGS];           // merge: the row's segments (start block, cand offset, count, -)
+  int vstart[SC_MAX_SEGS + 1];      // merge: prefix of the ordered segments' counts
   int bcast[4];
 };
+static_assert(SC_SEG_KEYS <= HT_MAX_N, "a segment's keys fit one selection");
+static_assert(2 * HT_TIE_CAP >= TOPK && SC_MERGE_CAP > TOPK, "merge survivors fit the tie storage");
+static_assert(sizeof(SelectScratch) <= HT_WORDS * 4, "the radix fallback borrows the histogram");
 
 struct Segment {
   int row, p0, np;  // row, first page within the row, pages
@@ -132,7 +141,7 @@ __device__ __forceinline__ void score_page(const PageRegs& r, const uint32_t (&b
 
 __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(ScoreParams p) {
   extern __shared__ uint8_t smem_raw[];
-  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(smem_aligned<128>(smem_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rows = p.rows;
 
@@ -170,7 +179,6 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
   int cur_row = -1;
   uint32_t bq[8][2];
   float wa = 0.f, wb = 0.f;
-  auto skey = [&](int i) { return S.keys[i]; };
   while (true) {
     // ---- next segment: ranges blockIdx.x, +gridDim.x, ..., cut at row boundaries and every 512 pages ----
     if (g >= gend) {
@@ -218,6 +226,17 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     const int nb = L >> 2;
     const int b0 = sg.p0 * PAGE_BLOCKS;
     const int nvalid = min(sg.np * PAGE_BLOCKS, nb - b0);
+    const int np_row = off_at(r + 1) - off_at(r);
+    // A segment that is not the whole row reserves its candidate slots now; the results are first
+    // used after the streaming, so the atomics' round trip hides behind it.
+    const bool partial = sg.np != np_row;
+    const int ncand = min(nvalid, TOPK);
+    int slot = 0, coff = 0;
+    if (tid == 0 && partial) {
+      slot = atomicAdd(p.seg_cnt + r, 1);
+      coff = atomicAdd(p.cand_cnt + r, ncand);
+    }
+    ht_zero<Cta>(S.hist);
     Cta::sync();
 
     // ---- stream: warp w scores pages w, w+8, ... (SC_U at a time) ----
@@ -238,35 +257,35 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
         if (S.pid[k] < 0) lo = hi = 0.f;  // unreadable page (flagged above)
         if (cq < 2) {
           const int local = k * PAGE_BLOCKS + g8 + 8 * cq;
-          if (local < nvalid) S.keys[local] = score_key(cq ? hi : lo);
+          if (local < nvalid) {
+            const uint32_t key = score_key(cq ? hi : lo);
+            S.keys[local] = key;
+            ht_count(S.hist, key);
+          }
         }
       }
     }
     Cta::sync();
 
     // ---- the segment's best 512 ----
-    const int np_row = off_at(r + 1) - off_at(r);
     int32_t* sel = p.sel + (int64_t)r * TOPK;
     if (sg.np == np_row) {  // the whole row (nb > 512 here): this is the answer
-      fast_topk<Cta>(skey, nvalid, TOPK, [&](int i, int o) { sel[o] = b0 + i; }, &S.ft);
+      hist_topk<Cta>(S.keys, S.hist, nvalid, TOPK, [&](int i, int o) { sel[o] = b0 + i; }, &S.ht);
       if (tid == 0) p.sel_n[r] = TOPK;
-      Cta::sync();
       continue;
     }
-    const int ncand = min(nvalid, TOPK);
     if (tid == 0) {
-      const int slot = atomicAdd(p.seg_cnt + r, 1);
-      int coff = atomicAdd(p.cand_cnt + r, ncand);
       const bool fits = slot < p.seg_cap && coff + ncand <= p.seg_cap * TOPK;
       if (!fits) {  // more segments than the workspace was sized for: drop this one, flag it
         set_error(p.err, QSA_DEVERR_SELECTION);
         coff = -1;
       }
-      if (slot < p.seg_cap) p.seg_tab[(int64_t)r * p.seg_cap + slot] = make_int4(b0, fits ? coff : 0, fits ? ncand : 0, 0);
+      if (slot < p.seg_cap)
+        p.seg_tab[(int64_t)r * p.seg_cap + slot] = make_int4(b0, fits ? coff : 0, fits ? ncand : 0, 0);
       S.bcast[0] = coff;
     }
     Cta::sync();
-    const int coff = S.bcast[0];
+    coff = S.bcast[0];
     if (coff >= 0) {
       uint32_t* ck = p.cand_key + (int64_t)r * p.seg_cap * TOPK + coff;
       int32_t* ci = p.cand_id + (int64_t)r * p.seg_cap * TOPK + coff;
@@ -275,7 +294,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
         ci[o] = b0 + i;
       };
       if (nvalid > TOPK) {
-        fast_topk<Cta>(skey, nvalid, TOPK, put, &S.ft);
+        hist_topk<Cta>(S.keys, S.hist, nvalid, TOPK, put, &S.ht);
       } else {
         for (int i = tid; i < nvalid; i += SC_THREADS) put(i, i);
       }
@@ -323,18 +342,62 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       return S.segs[lo].y + (v - S.vstart[lo]);
     };
     const int nv = S.vstart[ns];
-    auto put = [&](int v, int o) { sel[o] = __ldcg(ri + gidx(v)); };
-    if (nv <= SC_SEG_KEYS) {
-      for (int v = tid; v < nv; v += SC_THREADS) S.keys[v] = __ldcg(rk + gidx(v));
+    const int kk_sel = min(TOPK, nv);  // < 512 only when segments were dropped (flagged above)
+    // Candidates are taken in block order, SC_MERGE_CAP at a time: each chunk is selected together
+    // with the best 512 of the chunks before it (kept at the front of the buffer, still in block
+    // order), so index order stays block order and ties keep the lower block.
+    int32_t* mids = reinterpret_cast<int32_t*>(S.keys + SC_MERGE_CAP);
+    unsigned long long* surv = S.ht.tie;  // survivors (key, id) of a non-final chunk
+    for (int done = 0, held = 0;;) {
+      const int take = min(nv - done, SC_MERGE_CAP - held);
+      ht_zero<Cta>(S.hist);
       Cta::sync();
-      fast_topk<Cta>(skey, nv, TOPK, put, &S.ft);
-    } else {  // long rows: read the candidates from L2 in place
-      auto gkey = [&](int v) { return __ldcg(rk + gidx(v)); };
-      const SelectResult m = radix_select<Cta>(gkey, nv, TOPK, &S.ft.sel);
-      select_compact<Cta>(gkey, nv, m, put, &S.ft.sel);
+      for (int i = tid; i < held; i += SC_THREADS) ht_count(S.hist, S.keys[i]);
+      // stage keys and ids, SU independent loads per thread in flight, counting keys as they arrive
+      constexpr int SU = 8;
+      for (int j0 = 0; j0 < take; j0 += SU * SC_THREADS) {
+        uint32_t kk[SU];
+        int32_t ii[SU];
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int j = j0 + u * SC_THREADS + tid;
+          if (j < take) {
+            const int gi = gidx(done + j);
+            kk[u] = __ldcg(rk + gi);
+            ii[u] = __ldcg(ri + gi);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int j = j0 + u * SC_THREADS + tid;
+          if (j < take) {
+            S.keys[held + j] = kk[u];
+            mids[held + j] = ii[u];
+            ht_count(S.hist, kk[u]);
+          }
+        }
+      }
+      Cta::sync();
+      const int n = held + take;
+      done += take;
+      if (done >= nv) {
+        hist_topk<Cta>(S.keys, S.hist, n, kk_sel, [&](int v, int o) { sel[o] = mids[v]; }, &S.ht);
+        break;
+      }
+      hist_topk<Cta>(S.keys, S.hist, n, kk_sel,
+                     [&](int v, int o) { surv[o] = ((unsigned long long)S.keys[v] << 32) | (uint32_t)mids[v]; },
+                     &S.ht);
+      for (int o = tid; o < kk_sel; o += SC_THREADS) {
+        const unsigned long long e = surv[o];
+        S.keys[o] = (uint32_t)(e >> 32);
+        mids[o] = (int32_t)(uint32_t)e;
+      }
+      held = kk_sel;
+      Cta::sync();
     }
     if (tid == 0) {
-      p.sel_n[r] = TOPK;
+      if (kk_sel < TOPK) set_error(p.err, QSA_DEVERR_SELECTION);
+      p.sel_n[r] = kk_sel;
       p.seg_cnt[r] = 0;  // ready for the next call
       p.cand_cnt[r] = 0;
       p.pages_done[r] = 0;
@@ -343,19 +406,26 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
   }
 }
 
-int score_grid(int num_sms) { return QSA_SC_CTAS_PER_SM * num_sms; }
-
-cudaError_t launch_score_topk(const ScoreParams& p, int grid, cudaStream_t st) {
-  static bool attr_set[64] = {false};
+// Persistent grid: as many CTAs as are resident at once (QSA_SC_CTAS_PER_SM per SM when the
+// shared memory allows it), so that no CTA waits for a second wave.
+cudaError_t launch_score_topk(const ScoreParams& p, int num_sms, cudaStream_t st) {
+  static int resident[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   const size_t smem = sizeof(ScoreSmem) + 128;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_score_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+  int per_sm = QSA_SC_CTAS_PER_SM;
+  if (dev >= 0 && dev < 64) {
+    if (resident[dev] == 0) {
+      cudaError_t e = cudaFuncSetAttribute(k_score_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      int n = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_score_topk, SC_THREADS, smem);
+      if (e != cudaSuccess) return e;
+      resident[dev] = max(1, min(n, QSA_SC_CTAS_PER_SM));
+    }
+    per_sm = resident[dev];
   }
-  k_score_topk<<<grid, SC_THREADS, smem, st>>>(p);
+  k_score_topk<<<per_sm * num_sms, SC_THREADS, smem, st>>>(p);
   return cudaGetLastError();
 }
 
