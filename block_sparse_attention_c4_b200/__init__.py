@@ -81,6 +81,7 @@ def lib():
     L.qsa_device_error.restype = i32
     L.qsa_set_profile_events.argtypes = [ctypes.POINTER(vp), i32]
     L.qsa_set_profile_events.restype = None
+    L.qsa_decode_kernel_count.argtypes = [i32]
     L.qsa_decode_kernel_count.restype = i32
     L.qsa_status_string.argtypes = [ctypes.c_int]
     L.qsa_status_string.restype = ctypes.c_char_p
@@ -330,8 +331,9 @@ def set_profile_events(events):
     lib().qsa_set_profile_events(arr, len(events) // 2)
 
 
-def decode_kernel_count() -> int:
-    return int(lib().qsa_decode_kernel_count())
+def decode_kernel_count(batch: int) -> int:
+    """Kernels one qsa_decode call launches for `batch` requests."""
+    return int(lib().qsa_decode_kernel_count(int(batch)))
 
 
 class DecodeSession:

@@ -25,6 +25,7 @@ struct WsLayout {
   size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, seg_cnt = 0, cand_cnt = 0,
          pages_done = 0, seg_tab = 0, cand_key = 0, cand_id = 0, part_o = 0, part_ml = 0, total = 0;
   size_t pf_keys = 0, pf_ovf_n = 0, pf_ovf_list = 0;
+  size_t ready = 0;  // decode: per-row flag, selection final (scorer -> sparse GQA)
   int ppc_min = 0;
   int seg_cap = 0;
   int splits_bound = 0;
@@ -35,15 +36,15 @@ constexpr size_t WS_ERR = 0;     // int: device error word
 constexpr size_t WS_TICKET = 64;  // int: prologue arrival ticket
 
 // Scorer range sizing from the longest context: ranges of at least ppc_min
-// pages keep the segments of one row at or below seg_cap (16 up to ~1.8M
-// tokens, so a row's candidates fit the merge buffer in shared memory).
-// A row of np pages meets at most ceil(np / ppc) + 1 ranges, and each range
-// piece is cut every SC_MAX_SEG_PAGES pages.
+// pages keep the segments of one row at or below seg_cap.  A row of np pages
+// meets at most ceil(np / ppc) + 1 ranges, and each range piece is cut every
+// SC_MAX_SEG_PAGES pages.
 void scorer_sizing(int max_len, int& ppc_min, int& seg_cap) {
   const int np_max = std::max(1, ceil_div(max_len / QSA_BLOCK, PAGE_BLOCKS));
   ppc_min = std::max(SC_MIN_PPC, ceil_div(np_max, 14));
   seg_cap = ceil_div(np_max, ppc_min) + ceil_div(np_max, SC_MAX_SEG_PAGES) + 2;
 }
+
 
 int positions_bound(int op, int max_len) {
   if (op == QSA_OP_SPARSE_GQA) return max_len;
@@ -74,6 +75,7 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     return true;
   }
   w.cnt_gqa = take(sizeof(int) * (size_t)rows);
+  if (op == QSA_OP_DECODE) w.ready = take(sizeof(int) * READY_STRIDE * (size_t)rows);
   if (scorer) {
     scorer_sizing(max_len, w.ppc_min, w.seg_cap);
     if (w.seg_cap > SC_MAX_SEGS) return false;
@@ -187,12 +189,16 @@ qsa_status cuda_status(cudaError_t e) {
 qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_bfloat16* knew,
                        const __nv_bfloat16* idx_q, const int32_t* row_req, const int32_t* row_len, int len_offset,
                        int rows, int max_len, const float* w, int32_t* sel, int32_t* sel_n, void* ws,
-                       const WsLayout& L, cudaStream_t st) {
+                       const WsLayout& L, cudaStream_t st, int* row_ready = nullptr) {
   const RopeFreqs fr = make_freqs(cache->rope_theta);
   int* err = at<int>(ws, WS_ERR);
   __nv_bfloat16* qrot = at<__nv_bfloat16>(ws, L.qrot);
-  {
-    ProfScope ps(st, 0);
+  // Up to SC_ROWS_SMEM rows the scorer runs the front end itself (append, rotation, page prefix);
+  // above that a separate prologue kernel does it first.
+  const bool fused = rows <= SC_ROWS_SMEM;
+  int ev = 0;
+  if (!fused) {
+    ProfScope ps(st, ev++);
     cudaError_t e = launch_index_prologue(cv, knew, idx_q, row_req, row_len, len_offset, rows, max_len, fr, qrot,
                                           at<int32_t>(ws, L.row_pages), at<int32_t>(ws, L.page_off),
                                           at<int>(ws, WS_TICKET), err, st);
@@ -219,7 +225,11 @@ qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_b
   p.sel = sel;
   p.sel_n = sel_n;
   p.err = err;
-  ProfScope ps(st, 1);
+  p.idx_q = fused ? idx_q : nullptr;
+  p.knew = fused ? knew : nullptr;
+  p.fr = fr;
+  p.row_ready = row_ready;
+  ProfScope ps(st, ev);
   return cuda_status(launch_score_topk(p, num_sms(), st));
 }
 
@@ -275,7 +285,7 @@ void qsa_set_profile_events(void* const* events, int32_t n_pairs) {
   g_prof_pairs = n_pairs;
 }
 
-int32_t qsa_decode_kernel_count(void) { return 3; }
+int32_t qsa_decode_kernel_count(int32_t batch) { return batch <= SC_ROWS_SMEM ? 2 : 3; }
 
 qsa_status qsa_compress_append(const qsa_cache* cache, const void* idx_k_new, const int32_t* cu_new,
                                const int32_t* len_before, int32_t total_new, int32_t max_new, void* stream) {
@@ -406,8 +416,11 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   int32_t* sel = blocks_out ? blocks_out : at<int32_t>(ws, L.sel);
   int32_t* sel_n = nblocks_out ? nblocks_out : at<int32_t>(ws, L.sel_n);
   std::lock_guard<std::mutex> lk(g_prof_mu);
+  // The sparse GQA is launched as a programmatic dependent of the scorer: it starts on the SMs the
+  // scorer frees and waits per row for the row's ready flag, overlapping the scorer's last merges.
+  int* ready = at<int>(ws, L.ready);
   s = run_indexer(cache, cv, static_cast<const __nv_bfloat16*>(idx_k_new), static_cast<const __nv_bfloat16*>(idx_q),
-                  nullptr, seq_len, 0, B, max_len, w, sel, sel_n, ws, L, st);
+                  nullptr, seq_len, 0, B, max_len, w, sel, sel_n, ws, L, st, ready);
   if (s != QSA_OK) return s;
   GqaParams p{};
   p.c = cv;
@@ -426,7 +439,8 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   p.part_ml = at<float>(ws, L.part_ml);
   p.counters = at<int>(ws, L.cnt_gqa);
   p.err = err;
-  ProfScope ps(st, 2);
+  p.row_ready = ready;
+  ProfScope ps(st, qsa_decode_kernel_count(B) - 1);
   return cuda_status(launch_gqa(p, B, positions_bound(QSA_OP_DECODE, max_len), num_sms(), L.splits_bound, st));
 }
 

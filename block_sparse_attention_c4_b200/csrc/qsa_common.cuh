@@ -95,6 +95,77 @@ __device__ __forceinline__ float key_score(uint32_t k) {
 }
 
 // ---------------------------------------------------------------------------
+// Block compression (blog section "Qwen Sparse Attention: Retrieve Coarsely,
+// Attend Precisely"): the mean of 4 raw index keys as an FP32 sum in token
+// order times 1/4, divided by its L2 norm and rotated at the block's first
+// position in FP64 (host-computed inverse frequencies), rounded once to bf16.
+// ---------------------------------------------------------------------------
+// One warp compresses one block.  Lane l owns dims l, l+32, l+64, l+96, i.e.
+// the rotation pairs (l, l+64) and (l+32, l+96), so the rotation needs no
+// exchange.  `keys4[j]` points at the raw key of token 4b+j.
+__device__ __forceinline__ void warp_compress_block(const __nv_bfloat16* const keys4[4], int64_t b,
+                                                    const RopeFreqs& fr, __nv_bfloat16* out) {
+  const int lane = threadIdx.x & 31;
+  float m[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = lane + 32 * e;
+    float s = __bfloat162float(keys4[0][d]);
+    s = s + __bfloat162float(keys4[1][d]);
+    s = s + __bfloat162float(keys4[2][d]);
+    s = s + __bfloat162float(keys4[3][d]);
+    m[e] = s * 0.25f;
+  }
+  double n2 = 0.0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) n2 += (double)m[e] * (double)m[e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+  const double nrm = sqrt(n2);
+  double kh[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) kh[e] = nrm > 0.0 ? (double)m[e] / nrm : 0.0;
+  const double p = (double)(CBLK * b);
+  uint16_t res[4];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int i = lane + 32 * e;  // pair (i, i + 64): kh[e] and kh[e + 2]
+    double sn, cs;
+    sincos(p * fr.f[i], &sn, &cs);
+    const double x0 = kh[e], x1 = kh[e + 2];
+    res[e] = f64_to_bf16_bits(x0 * cs - x1 * sn);
+    res[e + 2] = f64_to_bf16_bits(x0 * sn + x1 * cs);
+  }
+  uint16_t* o = reinterpret_cast<uint16_t*>(out);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) o[lane + 32 * e] = res[e];
+}
+
+__device__ __forceinline__ int64_t cidx_entry(const CacheView& c, int req, int64_t b, int* err) {
+  const int64_t s = slot_of(c, req, (int)(CBLK * b), err);
+  return s < 0 ? -1 : s / CBLK;
+}
+
+// Decode append of one row (one warp): the new index key of position L-1 goes to ring slot
+// (L-1) mod 4, and when it completes block b = L/4 - 1 that block is compressed from ring slots
+// 0..2 and the new key.
+__device__ __forceinline__ void warp_decode_append(const CacheView& c, int req, int L, const __nv_bfloat16* key,
+                                                   const RopeFreqs& fr, int* err) {
+  const int pos = L - 1;
+  __nv_bfloat16* ring = c.ring + (int64_t)req * CBLK * D;
+  if ((pos & 3) == 3) {
+    const __nv_bfloat16* k4[4] = {ring, ring + D, ring + 2 * D, key};
+    const int64_t b = pos >> 2;
+    const int64_t e = cidx_entry(c, req, b, err);
+    if (e >= 0) warp_compress_block(k4, b, fr, c.cidx + e * D);
+    __syncwarp();
+  }
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(key);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(ring + (pos & 3) * D);
+  for (int i = threadIdx.x & 31; i < D / 2; i += 32) dst[i] = src[i];
+}
+
+// ---------------------------------------------------------------------------
 // Shared-memory / async-copy PTX wrappers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -145,6 +216,35 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Cross-kernel readiness of one row (programmatic dependent launch): the producer publishes
+// after its block barrier (release, GPU scope); a consumer thread waits for it (acquire), giving up
+// after ~2 s of wall time with QSA_DEVERR_TIMEOUT.  Returns whether the row became ready.
+__device__ __forceinline__ void publish_ready(int* flag) {
+  asm volatile("fence.acq_rel.gpu;\n\tst.release.gpu.global.b32 [%0], 1;" ::"l"(flag) : "memory");
+}
+
+__device__ __forceinline__ bool wait_ready(const int* flag, int* err) {
+  uint64_t t0 = 0;
+  for (int spin = 0;; ++spin) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0) return true;
+    if (spin == 0) {
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    } else if ((spin & 63) == 0) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > 2000000000ull) break;
+    }
+    __nanosleep(256);  // few polls: many CTAs may wait at once
+  }
+  set_error(err, QSA_DEVERR_TIMEOUT);
+  return false;
+}
+
+// Row flags sit one per 128-byte line, so that waiting CTAs do not all poll the same L2 lines.
+constexpr int READY_STRIDE = 32;
+
 // Bounded wait: gives up after ~2 s of wall time, records QSA_DEVERR_TIMEOUT
 // and returns false (the caller then proceeds without the data).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
@@ -194,9 +294,22 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint
 }
 
 // 16-byte cp.async global -> shared; src_bytes = 0 writes zeros.
+#ifndef QSA_CP_L2_PROMOTE
+#define QSA_CP_L2_PROMOTE 0
+#endif
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src, int src_bytes) {
+#if QSA_CP_L2_PROMOTE == 256
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+#elif QSA_CP_L2_PROMOTE == 128
+  asm volatile("cp.async.cg.shared.global.L2::128B [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+#else
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
+#endif
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
@@ -605,7 +718,7 @@ constexpr int HT_TIE_CAP = 256;
 
 struct HistTopScratch {
   int warp_tot[33];
-  int D, above, tie_n;
+  int D, above, tie_n;  // tie_n: shared tie counter of the regather path and of row selections
   int tie_cnt[32];  // ties found by each warp
   uint32_t bits[HT_MAX_N / 32];
   // ties of the cut bin as one comparable word: key in the high half, bitwise-inverted index in the

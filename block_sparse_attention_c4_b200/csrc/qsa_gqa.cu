@@ -24,20 +24,31 @@
 
 namespace qsa {
 
+#ifndef QSA_GQ_STAGES
+#define QSA_GQ_STAGES 4
+#endif
 constexpr int GQ_TILE = 16;
-constexpr int GQ_STAGES = 4;
+constexpr int GQ_STAGES = QSA_GQ_STAGES;
 constexpr int GQ_ROW_BYTES = D * 2;                             // 256 B: one head of one position
 constexpr int GQ_KV_BYTES = GQ_TILE * HKV * GQ_ROW_BYTES;       // 8 KiB: K (or V) of a tile
 constexpr int GQ_STAGE_BYTES = 2 * GQ_KV_BYTES;                 // 16 KiB
 
 constexpr int GQ_MAX_TILES = (QSA_MAX_SEL + QSA_MAX_DRAFT + GQ_TILE - 1) / GQ_TILE;  // per row
 
+// The queries (both KV groups, MT*16 rows each) are staged in shared memory only until they are
+// in registers; when they fit one ring stage they pass through the last stage, which the pipeline
+// first fills after every warp has read them.  Less shared memory leaves more L1 for the loads.
 template <int MT>
 struct GqaSmem {
-  alignas(128) uint8_t q[HKV][MT * 16][GQ_ROW_BYTES];
+  static constexpr int QBYTES = HKV * MT * 16 * GQ_ROW_BYTES;
+  static constexpr bool Q_IN_RING = QBYTES <= GQ_STAGE_BYTES;
   alignas(128) uint8_t kv[GQ_STAGES][GQ_STAGE_BYTES];  // [K|V][group][pos][256 B], swizzled
+  alignas(128) uint8_t qsep[Q_IN_RING ? 16 : QBYTES];
   int is_last;
   int32_t slot[1];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
+  __device__ __forceinline__ uint8_t* qrow(int g, int rho) {
+    return (Q_IN_RING ? kv[GQ_STAGES - 1] : qsep) + (g * MT * 16 + rho) * GQ_ROW_BYTES;
+  }
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return (uint32_t)(((chunk ^ (row & 7)) << 4)); }
@@ -54,14 +65,38 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   bool bad = req < 0 || req >= p.c.batch;
   if (bad && split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_REQUEST);
 
-  // ---- the row's position list ----
+  // ---- load the queries of both KV groups: row rho = query*8 + head-in-group ----
+  {
+    const __nv_bfloat16* qrow = p.q + (int64_t)row * nq * HQ * D;
+    constexpr int CHUNKS = HKV * MT * 16 * (GQ_ROW_BYTES / 16);
+    for (int c = tid; c < CHUNKS; c += THREADS) {
+      const int g = c / (MT * 16 * 16);
+      const int rho = (c / 16) % (MT * 16);
+      const int ch = c % 16;
+      const int qi = rho >> 3, h = g * GROUP + (rho & 7);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (qi < nq) v = __ldg(reinterpret_cast<const uint4*>(qrow + ((int64_t)qi * HQ + h) * D) + ch);
+      *reinterpret_cast<uint4*>(S.qrow(g, rho) + swz(rho, ch)) = v;
+    }
+  }
+
+  // ---- launched early (programmatic dependent of the scorer): wait until this row's selection
+  // is final; the queries above were loaded meanwhile ----
+  if (p.row_ready) {
+    if (tid == 0 && !wait_ready(p.row_ready + row * READY_STRIDE, p.err)) S.is_last = -1;
+    else if (tid == 0) S.is_last = 0;
+    __syncthreads();
+    if (S.is_last < 0) bad = true;
+  }
+
+  // ---- the row's position list (coherent loads: the scorer may have written it just now) ----
   int nbase = 0, nsel4 = 0, tail0 = 0;
   const int32_t* sel = nullptr;
   const int32_t* list = nullptr;
   if (!bad) {
     if (p.mode == 0) {
       const int L = __ldg(p.row_len + row) + p.len_offset;
-      const int nsel = __ldg(p.sel_n + row);
+      const int nsel = __ldcg(p.sel_n + row);
       if (L < 1 || L > p.max_len || nsel < 0 || nsel > TOPK || nsel > (L >> 2)) {
         if (split == 0 && tid == 0) set_error(p.err, QSA_DEVERR_SELECTION);
         bad = true;
@@ -96,25 +131,10 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   auto position = [&](int j) -> int {
     if (j < nbase) {
       if (list) return __ldg(list + j);
-      return j < nsel4 ? __ldg(sel + (j >> 2)) * CBLK + (j & 3) : tail0 + (j - nsel4);
+      return j < nsel4 ? __ldcg(sel + (j >> 2)) * CBLK + (j & 3) : tail0 + (j - nsel4);
     }
     return ext0 + (j - nbase);
   };
-
-  // ---- load the queries of both KV groups: row rho = query*8 + head-in-group ----
-  {
-    const __nv_bfloat16* qrow = p.q + (int64_t)row * nq * HQ * D;
-    constexpr int CHUNKS = HKV * MT * 16 * (GQ_ROW_BYTES / 16);
-    for (int c = tid; c < CHUNKS; c += THREADS) {
-      const int g = c / (MT * 16 * 16);
-      const int rho = (c / 16) % (MT * 16);
-      const int ch = c % 16;
-      const int qi = rho >> 3, h = g * GROUP + (rho & 7);
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (qi < nq) v = __ldg(reinterpret_cast<const uint4*>(qrow + ((int64_t)qi * HQ + h) * D) + ch);
-      *reinterpret_cast<uint4*>(&S.q[g][rho][swz(rho, ch)]) = v;
-    }
-  }
 
   // ---- physical slots of this CTA's positions, resolved once up front ----
   for (int j = tid; j < ntl * GQ_TILE; j += THREADS) {
@@ -158,7 +178,7 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
     const int rho = mt * 16 + (lane & 7) + ((mtx & 1) << 3);
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      ldmatrix_x4(qa[j][0], qa[j][1], qa[j][2], qa[j][3], smem_u32(&S.q[g][rho][swz(rho, 2 * j + (mtx >> 1))]));
+      ldmatrix_x4(qa[j][0], qa[j][1], qa[j][2], qa[j][3], smem_u32(S.qrow(g, rho) + swz(rho, 2 * j + (mtx >> 1))));
   }
   const int qi0 = (mt * 16 + gq) >> 3, qi1 = (mt * 16 + gq + 8) >> 3;  // query of rows gq, gq+8
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -261,6 +281,7 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   const int h0 = g * GROUP + (rho0 & 7), h1 = g * GROUP + (rho1 & 7);
   const int nh = nq * HQ;
   if (p.splits == 1) {
+    if (p.row_ready && tid == 0) p.row_ready[row * READY_STRIDE] = 0;  // ready for the next call
     const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
     __nv_bfloat16* out = p.out + (int64_t)row * nh * D;
 #pragma unroll
@@ -296,37 +317,89 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   __syncthreads();
   if (!S.is_last) return;
   __threadfence();
-  // merge: thread handles (head, 4-dim group)
+  // merge.  Every load of a step is issued before any is used: (a) per head, the (m, l) of all
+  // splits give normalized split weights (kept in the now idle ring); (b) per (head, 4 dims), the
+  // weighted sum over splits, four splits x four items of loads in flight per thread.
   const float* pob = p.part_o + (int64_t)row * p.splits * nh * D;
   const float* pmb = p.part_ml + (int64_t)row * p.splits * nh * 2;
   __nv_bfloat16* out = p.out + (int64_t)row * nh * D;
-  for (int idx = tid; idx < nh * (D / 4); idx += THREADS) {
-    const int hh = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
+  float* wsm = reinterpret_cast<float*>(S.kv[0]);  // [nh][GQ_MAX_SPLITS]
+  const int splits = p.splits;
+  for (int hh = tid; hh < nh; hh += THREADS) {
+    float mv[GQ_MAX_SPLITS], lv[GQ_MAX_SPLITS];
+#pragma unroll
+    for (int s2 = 0; s2 < GQ_MAX_SPLITS; ++s2) {
+      float2 ml = make_float2(-INFINITY, 0.f);
+      if (s2 < splits) ml = __ldcg(reinterpret_cast<const float2*>(pmb + ((int64_t)s2 * nh + hh) * 2));
+      mv[s2] = ml.x;
+      lv[s2] = ml.y;
+    }
     float M = -INFINITY;
-    for (int s2 = 0; s2 < p.splits; ++s2) M = fmaxf(M, __ldcg(pmb + ((int64_t)s2 * nh + hh) * 2));
+#pragma unroll
+    for (int s2 = 0; s2 < GQ_MAX_SPLITS; ++s2) M = fmaxf(M, mv[s2]);
     const float base = M == -INFINITY ? 0.f : M;
-    float den = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (int s2 = 0; s2 < p.splits; ++s2) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(pmb + ((int64_t)s2 * nh + hh) * 2));
-      const float f = exp2f(ml.x - base);
-      den += f * ml.y;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(pob + ((int64_t)s2 * nh + hh) * D + d4));
-      a0 += f * v.x;
-      a1 += f * v.y;
-      a2 += f * v.z;
-      a3 += f * v.w;
+    float den = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < GQ_MAX_SPLITS; ++s2) {
+      mv[s2] = exp2f(mv[s2] - base);  // 0 for unused splits
+      den += mv[s2] * lv[s2];
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
-    uint2 pk;
-    pk.x = pack_bf16x2(a0 * inv, a1 * inv);
-    pk.y = pack_bf16x2(a2 * inv, a3 * inv);
-    *reinterpret_cast<uint2*>(out + (int64_t)hh * D + d4) = pk;
-    if (p.lse && d4 == 0) {
+#pragma unroll
+    for (int s2 = 0; s2 < GQ_MAX_SPLITS; ++s2) wsm[hh * GQ_MAX_SPLITS + s2] = mv[s2] * inv;
+    if (p.lse) {
       constexpr float LN2 = 0.69314718055994530942f;
       p.lse[(int64_t)row * nh + hh] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
     }
   }
-  if (tid == 0) p.counters[row] = 0;
+  __syncthreads();
+  constexpr int IT = 4;  // items per thread in flight
+  const int nitems = nh * (D / 4);
+  for (int idx0 = 0; idx0 < nitems; idx0 += IT * THREADS) {
+    float4 acc[IT];
+#pragma unroll
+    for (int i = 0; i < IT; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < splits; s0 += 4) {
+      float4 v[IT][4];
+#pragma unroll
+      for (int i = 0; i < IT; ++i)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = idx0 + i * THREADS + tid, s2 = s0 + u;
+          v[i][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (idx < nitems && s2 < splits)
+            v[i][u] = __ldcg(reinterpret_cast<const float4*>(pob + ((int64_t)s2 * nh + idx / (D / 4)) * D +
+                                                              (idx % (D / 4)) * 4));
+        }
+#pragma unroll
+      for (int i = 0; i < IT; ++i)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = idx0 + i * THREADS + tid, s2 = s0 + u;
+          if (idx < nitems && s2 < splits) {
+            const float wgt = wsm[(idx / (D / 4)) * GQ_MAX_SPLITS + s2];
+            acc[i].x += wgt * v[i][u].x;
+            acc[i].y += wgt * v[i][u].y;
+            acc[i].z += wgt * v[i][u].z;
+            acc[i].w += wgt * v[i][u].w;
+          }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      const int idx = idx0 + i * THREADS + tid;
+      if (idx < nitems) {
+        uint2 pk;
+        pk.x = pack_bf16x2(acc[i].x, acc[i].y);
+        pk.y = pack_bf16x2(acc[i].z, acc[i].w);
+        *reinterpret_cast<uint2*>(out + (int64_t)(idx / (D / 4)) * D + (idx % (D / 4)) * 4) = pk;
+      }
+    }
+  }
+  if (tid == 0) {
+    p.counters[row] = 0;  // ready for the next call
+    if (p.row_ready) p.row_ready[row * READY_STRIDE] = 0;
+  }
 }
 
 // Workspace bound on the split count (no device needed): at most 8 resident
@@ -379,19 +452,36 @@ static void choose_splits(int rows, int max_pos, int num_sms, int bound, int& sp
 template <int MT>
 static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, int bound, cudaStream_t st) {
   static bool attr_set[64] = {false};
+  static const int carveout = [] {  // tuning override: QSA_GQA_CARVEOUT=0..100 (percent of shared memory)
+    const char* e = getenv("QSA_GQA_CARVEOUT");
+    const int v = e ? atoi(e) : -1;
+    return (v >= 0 && v <= 100) ? v : -1;
+  }();
   int dev = 0;
   cudaGetDevice(&dev);
   const size_t smem_max = gqa_smem_bytes<MT>(GQ_MAX_TILES);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e =
         cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+    if (e == cudaSuccess && carveout >= 0)
+      e = cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   choose_splits<MT>(rows, max_pos, num_sms, bound, p.splits, p.tiles_per_split);
-  dim3 grid(p.splits, rows);
-  k_sparse_gqa<MT><<<grid, MT * 128, gqa_smem_bytes<MT>(p.tiles_per_split), st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, rows);
+  cfg.blockDim = dim3(MT * 128);
+  cfg.dynamicSmemBytes = gqa_smem_bytes<MT>(p.tiles_per_split);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (p.row_ready) {  // may start before the scorer ends; each CTA waits for its row's flag
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, k_sparse_gqa<MT>, p);
 }
 
 cudaError_t launch_gqa(const GqaParams& p, int rows, int max_pos, int num_sms, int split_bound, cudaStream_t st) {

@@ -17,52 +17,6 @@
 
 namespace qsa {
 
-// One warp compresses one block.  Lane l owns dims l, l+32, l+64, l+96, i.e.
-// the rotation pairs (l, l+64) and (l+32, l+96), so the rotation needs no
-// exchange.  `keys4[j]` points at the raw key of token 4b+j.
-__device__ __forceinline__ void warp_compress_block(const __nv_bfloat16* const keys4[4], int64_t b,
-                                                    const RopeFreqs& fr, __nv_bfloat16* out) {
-  const int lane = threadIdx.x & 31;
-  float m[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int d = lane + 32 * e;
-    float s = __bfloat162float(keys4[0][d]);
-    s = s + __bfloat162float(keys4[1][d]);
-    s = s + __bfloat162float(keys4[2][d]);
-    s = s + __bfloat162float(keys4[3][d]);
-    m[e] = s * 0.25f;
-  }
-  double n2 = 0.0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) n2 += (double)m[e] * (double)m[e];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
-  const double nrm = sqrt(n2);
-  double kh[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) kh[e] = nrm > 0.0 ? (double)m[e] / nrm : 0.0;
-  const double p = (double)(CBLK * b);
-  uint16_t res[4];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int i = lane + 32 * e;  // pair (i, i + 64): kh[e] and kh[e + 2]
-    double sn, cs;
-    sincos(p * fr.f[i], &sn, &cs);
-    const double x0 = kh[e], x1 = kh[e + 2];
-    res[e] = f64_to_bf16_bits(x0 * cs - x1 * sn);
-    res[e + 2] = f64_to_bf16_bits(x0 * sn + x1 * cs);
-  }
-  uint16_t* o = reinterpret_cast<uint16_t*>(out);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) o[lane + 32 * e] = res[e];
-}
-
-__device__ __forceinline__ int64_t cidx_entry(const CacheView& c, int req, int64_t b, int* err) {
-  const int64_t s = slot_of(c, req, (int)(CBLK * b), err);
-  return s < 0 ? -1 : s / CBLK;
-}
-
 // --------------------------------------------------------------------------
 // Bulk append.  grid = (ceil(max_tasks / 4), batch), 128 threads = 4 warps,
 // one block task per warp.  Task t of request r compresses block

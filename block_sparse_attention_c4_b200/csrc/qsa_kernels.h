@@ -46,7 +46,15 @@ struct ScoreParams {
   int32_t* sel;               // [rows][512] out
   int32_t* sel_n;             // [rows] out
   int* err;
+  // Fused front end (rows <= SC_ROWS_SMEM): with idx_q set, every CTA computes the page prefix
+  // itself (page_off unused), the CTA starting a row rotates that row's index query (qrot unused),
+  // and with knew set the CTA owning a row's last page first appends the row's new index key.
+  const __nv_bfloat16* idx_q;  // nullable: [rows][4][128] unrotated index queries
+  const __nv_bfloat16* knew;   // nullable: [rows][128] decode index keys
+  RopeFreqs fr;
+  int* row_ready;              // nullable: [rows][READY_STRIDE] set to 1 once a row's selection is final
 };
+constexpr int SC_ROWS_SMEM = 512;  // rows whose page offsets fit shared memory (fused front end)
 
 // Launches the persistent scorer on every SM (as many CTAs per SM as are resident).
 cudaError_t launch_score_topk(const ScoreParams& p, int num_sms, cudaStream_t st);
@@ -79,6 +87,8 @@ struct GqaParams {
   int splits;                 // set by launch_gqa
   int tiles_per_split;        // set by launch_gqa
   int* err;
+  int* row_ready;             // nullable (mode 0, [rows][READY_STRIDE]): wait for the row's flag, then clear it;
+                              // the kernel is then launched as a programmatic dependent of the scorer
 };
 
 // Upper bound of the split count launch_gqa may choose (workspace sizing).

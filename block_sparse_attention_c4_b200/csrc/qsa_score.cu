@@ -26,14 +26,18 @@
 //     query's B fragments are built with the same permutation of dims that
 //     the loads produce, and no shuffle or shared-memory staging is needed.
 //     The FP32 pipes stay free; the tensor pipe is far from busy.
-//   * Scores become order-preserving 32-bit keys in shared memory.  At the
-//     end of a segment the CTA radix-selects its best 512 (the other CTAs on
-//     the SM keep streaming).  A segment that is a whole row gives the answer
-//     directly; otherwise its candidates go to the row's list in global
-//     memory, and the CTA that completes the row's last segment (atomic page
-//     count, no waiting) merges them: it orders the row's segments by block,
-//     stages their candidates in shared memory and selects the final 512,
-//     ascending.  Scores never travel to HBM.
+//   * Scores become order-preserving 32-bit keys in shared memory, counted
+//     as they are written into a log-scale histogram, so that the segment's
+//     exact top-512 (hist_topk) needs one pass over the keys.  A segment that
+//     is a whole row gives the answer directly; otherwise its candidates go
+//     to the row's list in global memory, and the CTA that completes the
+//     row's last segment (atomic page count, no waiting) merges them: it
+//     orders the row's segments by block and selects the final 512 from
+//     their candidates in block-ordered chunks, ascending.  Scores never
+//     travel to HBM.
+//   * The sparse GQA is launched as a programmatic dependent of this kernel
+//     and waits per row: each row's selection is published (release flag) as
+//     soon as it is final.
 #include <cstdlib>
 
 #include "qsa_common.cuh"
@@ -51,7 +55,6 @@ constexpr int SC_WARPS = 8;
 constexpr int SC_THREADS = SC_WARPS * 32;
 constexpr int SC_U = QSA_SC_PAGES_PER_LOAD;  // pages a warp loads before computing
 constexpr int SC_SEG_KEYS = SC_MAX_SEG_PAGES * PAGE_BLOCKS;  // 8192
-constexpr int SC_ROWS_SMEM = 512;  // rows whose page offsets are staged in shared memory
 
 using Cta = Group<SC_THREADS, 0>;
 
@@ -68,6 +71,9 @@ struct ScoreSmem {
   int32_t off[SC_ROWS_SMEM + 1];    // exclusive prefix of pages per row
   int4 segs[SC_MAX_SEGS];           // merge: the row's segments (start block, cand offset, count, -)
   int vstart[SC_MAX_SEGS + 1];      // merge: prefix of the ordered segments' counts
+  double cs[D / 2], sn[D / 2];      // fused front end: RoPE angles of the current row's query
+  uint32_t qraw[HI * D / 2];        // fused front end: unrotated query, then rotated (bf16 pairs)
+  int warp_tot[33];
   int bcast[4];
 };
 static_assert(SC_SEG_KEYS <= HT_MAX_N, "a segment's keys fit one selection");
@@ -91,11 +97,24 @@ __device__ __forceinline__ int row_of_page(const int32_t* off_s, const int32_t* 
   return lo;
 }
 
+#ifndef QSA_SC_L2_PROMOTE
+#define QSA_SC_L2_PROMOTE 0
+#endif
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
   uint4 v;
+#if QSA_SC_L2_PROMOTE == 256
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+#elif QSA_SC_L2_PROMOTE == 128
+  asm volatile("ld.global.nc.L1::no_allocate.L2::128B.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+#else
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
+#endif
   return v;
 }
 
@@ -112,6 +131,15 @@ __device__ __forceinline__ void load_page(PageRegs& r, const uint4* page, int g,
   for (int u = 0; u < 4; ++u) {
     r.lo[u] = ldg_stream(page + g * 16 + c + 4 * u);
     r.hi[u] = ldg_stream(page + (g + 8) * 16 + c + 4 * u);
+  }
+}
+
+// The same with coherent loads, for the one page this kernel has just written a compressed key to.
+__device__ __forceinline__ void load_page_fresh(PageRegs& r, const uint4* page, int g, int c) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    r.lo[u] = __ldcg(page + g * 16 + c + 4 * u);
+    r.hi[u] = __ldcg(page + (g + 8) * 16 + c + 4 * u);
   }
 }
 
@@ -144,26 +172,56 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
   ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(smem_aligned<128>(smem_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rows = p.rows;
+  const bool fused = p.idx_q != nullptr;  // the host sets it only when rows <= SC_ROWS_SMEM
+  // Every CTA of this grid is resident (the grid is sized to residency); the sparse GQA launched
+  // after it may start now on SMs this grid frees, and waits per row for the row's flag.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  auto row_of = [&](int r, int& req, int& L) {
+    req = p.row_req ? __ldg(p.row_req + r) : r;
+    L = __ldg(p.row_len + r) + p.len_offset;
+    return req >= 0 && req < p.c.batch && L >= 1 && L <= p.max_len;
+  };
 
-  // ---- rows with at most 512 complete blocks keep them all; bad rows keep none ----
+  // ---- rows with at most 512 complete blocks keep them all (and append here); bad rows keep none ----
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-    const int req = p.row_req ? __ldg(p.row_req + r) : r;
-    const int L = __ldg(p.row_len + r) + p.len_offset;
-    const bool bad = req < 0 || req >= p.c.batch || L < 1 || L > p.max_len;
-    const int nb = bad ? 0 : (L >> 2);
+    int req, L;
+    const bool ok = row_of(r, req, L);
+    const int nb = ok ? (L >> 2) : 0;
     if (nb > TOPK) continue;
     int32_t* sel = p.sel + (int64_t)r * TOPK;
     for (int i = tid; i < nb; i += SC_THREADS) sel[i] = i;
     if (tid == 0) {
       p.sel_n[r] = nb;
-      if (bad) set_error(p.err, (req < 0 || req >= p.c.batch) ? QSA_DEVERR_REQUEST : QSA_DEVERR_LENGTH);
+      if (!ok) set_error(p.err, (req < 0 || req >= p.c.batch) ? QSA_DEVERR_REQUEST : QSA_DEVERR_LENGTH);
+    }
+    if (fused && p.knew && ok && warp == 0) warp_decode_append(p.c, req, L, p.knew + (int64_t)r * D, p.fr, p.err);
+    if (p.row_ready) {
+      __syncthreads();
+      if (tid == 0) publish_ready(p.row_ready + r * READY_STRIDE);
     }
   }
 
   // ---- the page list ----
   const bool off_in_smem = rows <= SC_ROWS_SMEM;
-  if (off_in_smem)
+  if (fused) {  // exclusive prefix of the pages each row streams
+    int running = 0;
+    for (int base = 0; base < rows; base += SC_THREADS) {
+      const int r = base + tid;
+      int pages = 0;
+      if (r < rows) {
+        int req, L;
+        const int nb = row_of(r, req, L) ? (L >> 2) : 0;
+        pages = nb > TOPK ? ceil_div(nb, PAGE_BLOCKS) : 0;
+      }
+      int tot;
+      const int ex = group_exclusive_scan<Cta>(pages, S.warp_tot, &tot);
+      if (r < rows) S.off[r] = running + ex;
+      running += tot;
+    }
+    if (tid == 0) S.off[rows] = running;
+  } else if (off_in_smem) {
     for (int i = tid; i <= rows; i += SC_THREADS) S.off[i] = __ldg(p.page_off + i);
+  }
   __syncthreads();
   const int32_t* off_s = off_in_smem ? S.off : nullptr;
   auto off_at = [&](int r) { return off_in_smem ? S.off[r] : __ldg(p.page_off + r); };
@@ -196,6 +254,13 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     if (sg.np <= 0) continue;
     const int r = sg.row;
     const int req = p.row_req ? __ldg(p.row_req + r) : r;
+    const int L = __ldg(p.row_len + r) + p.len_offset;
+    const bool new_row = r != cur_row;
+    uint32_t qv = 0;
+    if (fused && new_row) {  // the row's index query and its RoPE angles at position L - 1
+      qv = __ldg(reinterpret_cast<const uint32_t*>(p.idx_q + (int64_t)r * HI * D) + tid);
+      if (tid < D / 2) sincos((double)(L - 1) * p.fr.f[tid], &S.sn[tid], &S.cs[tid]);
+    }
     {  // the segment's physical pages
       const int32_t* pt = p.c.page_table + (int64_t)req * p.c.max_pages;
       for (int k = tid; k < sg.np; k += SC_THREADS) {
@@ -208,25 +273,47 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
         S.pid[k] = phys;
       }
     }
-    if (r != cur_row) {
+    if (new_row) {
       // B operand, permuted like the loads: column n = index head n (zero for n >= 4); for k-step
       // j = 2u + h, lane (n, c) holds dims 8(c+4u) + 4h + {0,1} (b0) and + {2,3} (b1).
       cur_row = r;
       const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.qrot + (int64_t)r * HI * D);
+      if (fused) {  // rotate here: pairs (i, i + 64) of head h, FP64 angles, one bf16 rounding
+        S.qraw[tid] = qv;
+        __syncthreads();
+        const int h = tid >> 6, i = tid & 63;
+        const uint16_t* q16 = reinterpret_cast<const uint16_t*>(S.qraw) + h * D;
+        const double x0 = (double)bf16_bits_to_f32(q16[i]);
+        const double x1 = (double)bf16_bits_to_f32(q16[i + D / 2]);
+        const uint16_t y0 = f64_to_bf16_bits(x0 * S.cs[i] - x1 * S.sn[i]);
+        const uint16_t y1 = f64_to_bf16_bits(x0 * S.sn[i] + x1 * S.cs[i]);
+        __syncthreads();
+        uint16_t* o16 = reinterpret_cast<uint16_t*>(S.qraw) + h * D;
+        o16[i] = y0;
+        o16[i + D / 2] = y1;
+        __syncthreads();
+        q32 = S.qraw;
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int d0 = 8 * (cq + 4 * (j >> 1)) + 4 * (j & 1);
-        bq[j][0] = g8 < HI ? __ldg(q32 + ((g8 * D + d0) >> 1)) : 0u;
-        bq[j][1] = g8 < HI ? __ldg(q32 + ((g8 * D + d0 + 2) >> 1)) : 0u;
+        bq[j][0] = g8 < HI ? q32[(g8 * D + d0) >> 1] : 0u;  // shared (fused) or global memory
+        bq[j][1] = g8 < HI ? q32[(g8 * D + d0 + 2) >> 1] : 0u;
       }
       wa = cq < 2 ? __ldg(p.w + (int64_t)r * HI + 2 * cq) : 0.f;
       wb = cq < 2 ? __ldg(p.w + (int64_t)r * HI + 2 * cq + 1) : 0.f;
     }
-    const int L = __ldg(p.row_len + r) + p.len_offset;
     const int nb = L >> 2;
     const int b0 = sg.p0 * PAGE_BLOCKS;
     const int nvalid = min(sg.np * PAGE_BLOCKS, nb - b0);
     const int np_row = off_at(r + 1) - off_at(r);
+    // The row's decode append is made by the CTA owning its last page, before that page is read;
+    // when it completes block nb - 1 (in the last page), that page is read with coherent loads.
+    int fresh_k = -1;
+    if (fused && p.knew && sg.p0 + sg.np == np_row) {
+      if (warp == 0) warp_decode_append(p.c, req, L, p.knew + (int64_t)r * D, p.fr, p.err);
+      if ((L & 3) == 0) fresh_k = sg.np - 1;
+    }
     // A segment that is not the whole row reserves its candidate slots now; the results are first
     // used after the streaming, so the atomics' round trip hides behind it.
     const bool partial = sg.np != np_row;
@@ -246,7 +333,10 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       for (int u = 0; u < SC_U; ++u) {
         const int k = k0 + u;
         const int phys = k < sg.np ? S.pid[k] : -1;
-        if (phys >= 0) load_page(pr[u], cidx + (int64_t)phys * (PAGE_BLOCKS * D / 8), g8, cq);
+        if (phys >= 0) {
+          if (k == fresh_k) load_page_fresh(pr[u], cidx + (int64_t)phys * (PAGE_BLOCKS * D / 8), g8, cq);
+          else load_page(pr[u], cidx + (int64_t)phys * (PAGE_BLOCKS * D / 8), g8, cq);
+        }
       }
 #pragma unroll
       for (int u = 0; u < SC_U; ++u) {
@@ -271,7 +361,10 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     int32_t* sel = p.sel + (int64_t)r * TOPK;
     if (sg.np == np_row) {  // the whole row (nb > 512 here): this is the answer
       hist_topk<Cta>(S.keys, S.hist, nvalid, TOPK, [&](int i, int o) { sel[o] = b0 + i; }, &S.ht);
-      if (tid == 0) p.sel_n[r] = TOPK;
+      if (tid == 0) {
+        p.sel_n[r] = TOPK;
+        if (p.row_ready) publish_ready(p.row_ready + r * READY_STRIDE);
+      }
       continue;
     }
     if (tid == 0) {
@@ -401,6 +494,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       p.seg_cnt[r] = 0;  // ready for the next call
       p.cand_cnt[r] = 0;
       p.pages_done[r] = 0;
+      if (p.row_ready) publish_ready(p.row_ready + r * READY_STRIDE);
     }
     Cta::sync();
   }

@@ -116,8 +116,9 @@ typedef enum {
  * positions per query; for QSA_OP_DECODE_INDEXSHARE pass the capture length
  * L0).  Returns 0 for invalid arguments.  The workspace must be 256-byte
  * aligned and must be zeroed once with qsa_workspace_init before its first
- * use; the kernels leave it ready for the next call.  Calls that share one
- * workspace must be ordered on the GPU (same stream or synchronised).
+ * use; the kernels leave it ready for the next call (after a call that
+ * returned QSA_ERR_CUDA, zero it again).  Calls that share one workspace must
+ * be ordered on the GPU (same stream or synchronised).
  */
 size_t qsa_workspace_bytes(int32_t op, int32_t rows, int32_t max_len);
 
@@ -227,7 +228,9 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
  *              (out, may both be NULL; IndexShare captures them from here)
  *   ws         workspace of qsa_workspace_bytes(QSA_OP_DECODE, batch, max_len)
  * Calling it twice with the same inputs gives the same result (the append is
- * idempotent).
+ * idempotent).  The attention kernel is launched as a programmatic dependent
+ * of the scoring kernel: it may start while the scorer finishes and waits, per
+ * request, for that request's selection (bounded wait; QSA_DEVERR_TIMEOUT).
  */
 qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
                       const void* q, const int32_t* seq_len, int32_t max_len, float scale, void* out, float* lse,
@@ -301,8 +304,10 @@ int32_t qsa_device_error(void* ws, int32_t clear, void* stream);
  */
 void qsa_set_profile_events(void* const* events, int32_t n_pairs);
 
-/* Number of kernels qsa_decode launches per call. */
-int32_t qsa_decode_kernel_count(void);
+/* Number of kernels qsa_decode launches per call for `batch` requests: 2 up to
+ * 512 requests (the scorer runs the indexer front end itself, then the sparse
+ * GQA), 3 above (a separate front-end kernel first). */
+int32_t qsa_decode_kernel_count(int32_t batch);
 
 const char* qsa_status_string(qsa_status s);
 /* Text of the CUDA error behind the calling thread's last QSA_ERR_CUDA. */

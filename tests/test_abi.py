@@ -39,7 +39,8 @@ def test_version_and_status_strings(qsa):
     assert "sm_100a" in qsa.version()
     for s in range(5):
         assert qsa.lib().qsa_status_string(s)
-    assert qsa.decode_kernel_count() == 3
+    assert qsa.decode_kernel_count(64) == 2 and qsa.decode_kernel_count(512) == 2
+    assert qsa.decode_kernel_count(513) == 3
 
 
 def test_workspace_bytes(qsa):
