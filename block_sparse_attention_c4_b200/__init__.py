@@ -40,7 +40,7 @@ class CacheStruct(ctypes.Structure):
     _fields_ = [
         ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("cidx", ctypes.c_void_p), ("ring", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p), ("num_slots", ctypes.c_int64), ("page_size", ctypes.c_int32),
-        ("max_pages", ctypes.c_int32), ("batch", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32), ("batch", ctypes.c_int32), ("kv_stride", ctypes.c_int32),
         ("rope_theta", ctypes.c_double),
     ]
 
@@ -153,17 +153,29 @@ class Workspace:
 class LayerCache:
     """The layer's paged cache: raw K/V pool, compressed index keys, ring and page table.
 
-    k, v: bf16 [num_slots, 2, 128]; cidx: bf16 [num_slots/4, 128]; ring: bf16 [batch, 4, 128];
+    k, v: bf16 [num_slots, 2, 128] views; cidx: bf16 [num_slots/4, 128]; ring: bf16 [batch, 4, 128];
     page_table: int32 [batch, max_pages].
+    kv_layout "interleaved" keeps each slot's K and V rows together (kv: [num_slots, 2, 2, 128], k and
+    v its two halves), so the 4 slots of a compressed block are one 4 KiB run; "separate" allocates
+    two arrays.
     """
 
     def __init__(self, num_slots: int, batch: int, max_pages: int, rope_theta: float = 1.0e7, device="cuda",
-                 page_table: torch.Tensor | None = None):
+                 page_table: torch.Tensor | None = None, kv_layout: str = "interleaved"):
         if num_slots % PAGE_SIZE:
             raise QsaError("num_slots must be a multiple of 64")
+        if kv_layout not in ("interleaved", "separate"):
+            raise QsaError(f"kv_layout must be 'interleaved' or 'separate', got {kv_layout!r}")
         self.num_slots, self.batch, self.max_pages, self.rope_theta = num_slots, batch, max_pages, rope_theta
-        self.k = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
-        self.v = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.kv_layout = kv_layout
+        if kv_layout == "interleaved":
+            self.kv = torch.zeros(num_slots, 2, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+            self.k, self.v = self.kv[:, 0], self.kv[:, 1]
+            self.kv_stride = 2 * KV_HEADS * HEAD_DIM
+        else:
+            self.k = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+            self.v = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+            self.kv_stride = 0
         self.cidx = torch.zeros(num_slots // BLOCK, HEAD_DIM, dtype=torch.bfloat16, device=device)
         self.ring = torch.zeros(max(batch, 1), BLOCK, HEAD_DIM, dtype=torch.bfloat16, device=device)
         if page_table is None:
@@ -173,7 +185,7 @@ class LayerCache:
     def struct(self, batch: int | None = None) -> CacheStruct:
         return CacheStruct(self.k.data_ptr(), self.v.data_ptr(), self.cidx.data_ptr(), self.ring.data_ptr(),
                            self.page_table.data_ptr(), self.num_slots, PAGE_SIZE, self.max_pages,
-                           self.batch if batch is None else batch, 0, self.rope_theta)
+                           self.batch if batch is None else batch, self.kv_stride, self.rope_theta)
 
 
 def compress_append(cache: LayerCache, idx_k_new, cu_new, len_before, max_new: int, stream=None):

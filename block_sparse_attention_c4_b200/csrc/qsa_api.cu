@@ -130,6 +130,7 @@ qsa_status check_cache(const qsa_cache* c) {
   if (c->num_slots / QSA_PAGE_SIZE > (int64_t)INT32_MAX / QSA_PAGE_SIZE) return QSA_ERR_UNSUPPORTED;
   if (c->max_pages <= 0 || c->batch < 0) return QSA_ERR_INVALID_ARG;
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) return QSA_ERR_INVALID_ARG;
+  if (c->kv_stride != 0 && (c->kv_stride < HKV * D || c->kv_stride % 8 != 0)) return QSA_ERR_INVALID_ARG;
   if (!aligned(c->k, 16) || !aligned(c->v, 16) || !aligned(c->cidx, 16) || !aligned(c->ring, 16) ||
       !aligned(c->page_table, 4))
     return QSA_ERR_INVALID_ARG;
@@ -144,6 +145,7 @@ CacheView view_of(const qsa_cache* c) {
   v.ring = static_cast<__nv_bfloat16*>(c->ring);
   v.page_table = c->page_table;
   v.num_pages = c->num_slots / QSA_PAGE_SIZE;
+  v.kv_stride = c->kv_stride ? c->kv_stride : HKV * D;
   v.max_pages = c->max_pages;
   v.batch = c->batch;
   return v;

@@ -31,6 +31,7 @@ struct CacheView {
   __nv_bfloat16* ring;
   const int32_t* page_table;
   int64_t num_pages;
+  int64_t kv_stride;  // bf16 elements from one slot's K (or V) rows to the next slot's
   int32_t max_pages;
   int32_t batch;
 };

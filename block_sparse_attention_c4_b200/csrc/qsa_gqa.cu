@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
       const int kvsel = c >> 9, j = (c >> 5) & 15, g = (c >> 4) & 1, ch = c & 15;
       const int64_t sl = tslot[j];
       const __nv_bfloat16* base = kvsel ? p.c.v : p.c.k;
-      const __nv_bfloat16* src = sl >= 0 ? base + (sl * HKV + g) * D + ch * 8 : base;
+      const __nv_bfloat16* src = sl >= 0 ? base + sl * p.c.kv_stride + g * D + ch * 8 : base;
       uint8_t* dst = dst0 + kvsel * GQ_KV_BYTES + g * (GQ_TILE * GQ_ROW_BYTES) + j * GQ_ROW_BYTES + swz(j, ch);
       cp_async_16(dst, src, sl >= 0 ? 16 : 0);
     }

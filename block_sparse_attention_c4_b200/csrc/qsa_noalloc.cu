@@ -78,6 +78,7 @@ extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void*
     return QSA_ERR_INVALID_ARG;
   if (!is_aligned(cache->k, 16) || !is_aligned(cache->v, 16) || !is_aligned(cache->page_table, 4))
     return QSA_ERR_INVALID_ARG;
+  if (cache->kv_stride != 0 && (cache->kv_stride < 256 || cache->kv_stride % 8 != 0)) return QSA_ERR_INVALID_ARG;
   if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !(scale > 0.f)) return QSA_ERR_INVALID_ARG;
   if (nq > QSA_NOALLOC_MAX_QUERIES) return QSA_ERR_UNSUPPORTED;  // beyond the array's stated capacity
   if (max_pos > QSA_MAX_SEL) return QSA_ERR_UNSUPPORTED;
@@ -96,6 +97,7 @@ extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void*
   p.c.v = static_cast<const __nv_bfloat16*>(cache->v);
   p.c.page_table = cache->page_table;
   p.c.num_pages = cache->num_slots / QSA_PAGE_SIZE;
+  p.c.kv_stride = cache->kv_stride ? cache->kv_stride : 256;
   p.c.max_pages = cache->max_pages;
   p.c.batch = cache->batch;
   p.q = static_cast<const __nv_bfloat16*>(q);

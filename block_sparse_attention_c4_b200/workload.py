@@ -25,14 +25,15 @@ def slots_of(page_table_row: np.ndarray, n_tok: int, tok0: int = 0) -> np.ndarra
     return page_table_row[t // PAGE_SIZE].astype(np.int64) * PAGE_SIZE + (t % PAGE_SIZE)
 
 
-def build_cache(wl, device="cuda", prefix_tokens=None, chunk_tokens: int = 1 << 16) -> LayerCache:
+def build_cache(wl, device="cuda", prefix_tokens=None, chunk_tokens: int = 1 << 16,
+                kv_layout: str = "interleaved") -> LayerCache:
     """Allocate the cache of `wl`, fill K/V for every stored token, and append the raw index keys of
     the first `prefix_tokens[r]` tokens of each request (default: lens[r] - 1, the state before a
     decode step) through qsa_compress_append."""
     pt = wl.page_table()
     B = wl.batch
     cache = LayerCache(wl.total_pages * PAGE_SIZE, B, pt.shape[1], rope_theta=wl.rope_theta, device=device,
-                       page_table=torch.from_numpy(pt).to(device))
+                       page_table=torch.from_numpy(pt).to(device), kv_layout=kv_layout)
     if prefix_tokens is None:
         prefix_tokens = [int(wl.lens[r]) - 1 for r in range(B)]
     for r in range(B):

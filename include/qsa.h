@@ -74,14 +74,21 @@ typedef enum {
 
 /*
  * The layer's cache.  All pointers are device pointers owned by the caller.
- *   k, v        bf16 [num_slots][2][128]  raw attention keys / values (paged pool)
+ *   k, v        bf16 raw attention keys / values of the paged pool: slot s holds
+ *               its two KV heads' 128-d rows at k + s * kv_stride (and likewise v)
  *   cidx        bf16 [num_slots / 4][128] compressed index keys; block b of request r
  *               lives at entry (page_table[r][4b / 64] * 64 + 4b % 64) / 4, so one
  *               page's 16 entries are contiguous (page-aligned full_slot / 4 rule)
  *   ring        bf16 [batch][4][128]      raw index keys of each request's
  *               unfinished block, slot = position mod 4
  *   page_table  int32 [batch][max_pages]  physical page of each logical page
- *   num_slots   multiple of page_size; page_size must be 64
+  *   num_slots   multiple of page_size; page_size must be 64
+ *   kv_stride   bf16 elements from one slot to the next in k (and in v): 0 means
+ *               256, i.e. separate [num_slots][2][128] arrays; 512 with
+ *               v = k + 256 interleaves each slot's K and V rows, so that the
+ *               4 slots of a compressed block are one 4 KiB run (the sparse
+ *               GQA then reads whole 4 KiB runs instead of two 2 KiB pieces).
+ *               Otherwise a multiple of 8, at least 256.
  *   rope_theta  RoPE base of the index keys/queries (1e7 for the workloads here)
  * Alignment: k, v, cidx, ring 16-byte aligned; page_table 4-byte aligned.
  */
@@ -95,7 +102,7 @@ typedef struct {
   int32_t page_size;
   int32_t max_pages;
   int32_t batch;
-  int32_t reserved;
+  int32_t kv_stride;
   double rope_theta;
 } qsa_cache;
 

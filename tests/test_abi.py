@@ -83,6 +83,11 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
     # misaligned pool pointer
     bad = fake_cache(qsa, k=0x1002)
     assert L.qsa_decode(ctypes.byref(bad), p, p, p, p, p, 100, 0.1, p, None, None, None, ws, big, None) == INVALID
+    # slot stride below the two KV heads' rows, or not a whole number of 16-byte chunks
+    for stride in (128, 255, 260):
+        bad = fake_cache(qsa, kv_stride=stride)
+        assert L.qsa_decode(ctypes.byref(bad), p, p, p, p, p, 100, 0.1, p, None, None, None, ws, big, None) == INVALID
+        assert L.qsa_sparse_gqa_noalloc(ctypes.byref(bad), p, p, p, p, 10, 10, 1, 0.1, p, None, None) == INVALID
     # max_len beyond the page table
     assert L.qsa_decode(ctypes.byref(c), p, p, p, p, p, 641, 0.1, p, None, None, None, ws, big, None) == INVALID
     # non-positive scale

@@ -173,9 +173,10 @@ def test_expand_indices_matches_oracle(Q, W):
 # a6: sparse GQA over explicit positions
 # ---------------------------------------------------------------------------------------------
 
-def test_sparse_gqa_matches_oracle(Q, W):
+@pytest.mark.parametrize("kv_layout", ["interleaved", "separate"])
+def test_sparse_gqa_matches_oracle(Q, W, kv_layout):
     wl = G.custom_decode(25, [5000, 3000], extra=0)
-    cache = W.build_cache(wl, prefix_tokens=[0, 0])
+    cache = W.build_cache(wl, prefix_tokens=[0, 0], kv_layout=kv_layout)
     rng = np.random.default_rng(3)
     cases = [(0, 0), (0, 1), (1, 17), (0, 2051), (1, 1000), (0, 33), (1, 2051), (0, 2048)]
     nq = len(cases)
@@ -209,8 +210,8 @@ def test_sparse_gqa_matches_oracle(Q, W):
 # the fused decode step
 # ---------------------------------------------------------------------------------------------
 
-def _run_decode(Q, W, wl, keep_cache=False):
-    cache = W.build_cache(wl)
+def _run_decode(Q, W, wl, keep_cache=False, kv_layout="interleaved"):
+    cache = W.build_cache(wl, kv_layout=kv_layout)
     inp = W.decode_inputs(wl)
     B = wl.batch
     max_len = int(max(wl.lens))
@@ -247,9 +248,10 @@ def _check_decode_request(wl, r, res, cache=None):
     return o
 
 
-def test_decode_small_batch_matches_oracle(Q, W):
+@pytest.mark.parametrize("kv_layout", ["interleaved", "separate"])
+def test_decode_small_batch_matches_oracle(Q, W, kv_layout):
     wl = G.decode_small()
-    res = _run_decode(Q, W, wl, keep_cache=True)
+    res = _run_decode(Q, W, wl, keep_cache=True, kv_layout=kv_layout)
     for r in range(wl.batch):
         _check_decode_request(wl, r, res, cache=res["cache"])
 
