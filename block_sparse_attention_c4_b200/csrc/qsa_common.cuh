@@ -714,8 +714,8 @@ __device__ void fast_topk(KeyAt key_at, int n, int k, Emit emit, FastTopScratch*
 constexpr int HT_BITS = 13;
 constexpr int HT_BINS = 1 << HT_BITS;  // 8192 bins
 constexpr int HT_WORDS = HT_BINS / 2;  // 4096 words of two 16-bit counts
-constexpr int HT_MAX_N = 8192;
-constexpr int HT_TIE_CAP = 256;
+constexpr int HT_MAX_N = 16384;
+constexpr int HT_TIE_CAP = 512;
 
 struct HistTopScratch {
   int warp_tot[33];
@@ -750,7 +750,7 @@ __device__ void hist_topk(const uint32_t* keys, uint32_t* hist, int n, int k, Em
   constexpr int NT = G::N, NW = NT / 32;
   constexpr int PER = HT_BINS / NT;  // bins per thread
   constexpr int WCAP = HT_TIE_CAP / NW;
-  static_assert(PER % 8 == 0 && HT_MAX_N / 32 <= NT, "layout");
+  static_assert(PER % 8 == 0, "layout");  // callers keep n <= 32 * NT (one bitmap word per thread)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // (1) thread t owns bins top-PER*t-PER+1 .. top-PER*t (descending order of ownership)
   const int lo_bin = HT_BINS - PER * (tid + 1);
@@ -771,7 +771,7 @@ __device__ void hist_topk(const uint32_t* keys, uint32_t* hist, int n, int k, Em
     sc->above = 0;
     sc->tie_n = 0;
   }
-  if (tid < HT_MAX_N / 32) sc->bits[tid] = 0u;
+  for (int i = tid; i < HT_MAX_N / 32; i += NT) sc->bits[i] = 0u;
   int tot;
   const int ex = group_exclusive_scan<G>(local, sc->warp_tot, &tot);  // keys in bins above this thread's
   if (ex < k && ex + local >= k) {

@@ -21,7 +21,11 @@ cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblocks, const i
                           int32_t* npos, int* err, cudaStream_t st);
 
 // ---- streaming scorer + top-512 (qsa_score.cu) ----
-constexpr int SC_MAX_SEG_PAGES = 512;  // pages of one segment (8192 blocks of score keys in shared memory)
+#ifndef QSA_SC_WARPS
+#define QSA_SC_WARPS 16
+#endif
+// pages of one segment (16 blocks of score keys each, all in shared memory)
+constexpr int SC_MAX_SEG_PAGES = QSA_SC_WARPS >= 16 ? 1024 : 512;
 constexpr int SC_MAX_SEGS = 64;        // segments per row a merge can order
 constexpr int SC_MIN_PPC = 32;         // pages per CTA range, lower bound
 

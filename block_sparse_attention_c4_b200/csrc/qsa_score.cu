@@ -48,10 +48,12 @@ namespace qsa {
 #ifndef QSA_SC_PAGES_PER_LOAD
 #define QSA_SC_PAGES_PER_LOAD 1
 #endif
+// One CTA of 16 warps per SM: the streaming keeps 16 warps' pages in flight per SM, and the
+// selection phases, which are bound by latency, run on all 16 warps instead of half of them.
 #ifndef QSA_SC_CTAS_PER_SM
-#define QSA_SC_CTAS_PER_SM 2
+#define QSA_SC_CTAS_PER_SM (16 / QSA_SC_WARPS)
 #endif
-constexpr int SC_WARPS = 8;
+constexpr int SC_WARPS = QSA_SC_WARPS;
 constexpr int SC_THREADS = SC_WARPS * 32;
 constexpr int SC_U = QSA_SC_PAGES_PER_LOAD;  // pages a warp loads before computing
 constexpr int SC_SEG_KEYS = SC_MAX_SEG_PAGES * PAGE_BLOCKS;  // 8192
@@ -76,7 +78,7 @@ struct ScoreSmem {
   int warp_tot[33];
   int bcast[4];
 };
-static_assert(SC_SEG_KEYS <= HT_MAX_N, "a segment's keys fit one selection");
+static_assert(SC_SEG_KEYS <= HT_MAX_N && SC_SEG_KEYS <= 32 * SC_THREADS, "a segment's keys fit one selection");
 static_assert(2 * HT_TIE_CAP >= TOPK && SC_MERGE_CAP > TOPK, "merge survivors fit the tie storage");
 static_assert(sizeof(SelectScratch) <= HT_WORDS * 4, "the radix fallback borrows the histogram");
 
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     const bool new_row = r != cur_row;
     uint32_t qv = 0;
     if (fused && new_row) {  // the row's index query and its RoPE angles at position L - 1
-      qv = __ldg(reinterpret_cast<const uint32_t*>(p.idx_q + (int64_t)r * HI * D) + tid);
+      if (tid < HI * D / 2) qv = __ldg(reinterpret_cast<const uint32_t*>(p.idx_q + (int64_t)r * HI * D) + tid);
       if (tid < D / 2) sincos((double)(L - 1) * p.fr.f[tid], &S.sn[tid], &S.cs[tid]);
     }
     {  // the segment's physical pages
@@ -279,18 +281,24 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       cur_row = r;
       const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.qrot + (int64_t)r * HI * D);
       if (fused) {  // rotate here: pairs (i, i + 64) of head h, FP64 angles, one bf16 rounding
-        S.qraw[tid] = qv;
+        constexpr int NR = HI * D / 2;  // threads of the rotation: one pair (i, i + 64) of one head each
+        if (tid < NR) S.qraw[tid] = qv;
         __syncthreads();
         const int h = tid >> 6, i = tid & 63;
-        const uint16_t* q16 = reinterpret_cast<const uint16_t*>(S.qraw) + h * D;
-        const double x0 = (double)bf16_bits_to_f32(q16[i]);
-        const double x1 = (double)bf16_bits_to_f32(q16[i + D / 2]);
-        const uint16_t y0 = f64_to_bf16_bits(x0 * S.cs[i] - x1 * S.sn[i]);
-        const uint16_t y1 = f64_to_bf16_bits(x0 * S.sn[i] + x1 * S.cs[i]);
+        uint16_t y0 = 0, y1 = 0;
+        if (tid < NR) {
+          const uint16_t* q16 = reinterpret_cast<const uint16_t*>(S.qraw) + h * D;
+          const double x0 = (double)bf16_bits_to_f32(q16[i]);
+          const double x1 = (double)bf16_bits_to_f32(q16[i + D / 2]);
+          y0 = f64_to_bf16_bits(x0 * S.cs[i] - x1 * S.sn[i]);
+          y1 = f64_to_bf16_bits(x0 * S.sn[i] + x1 * S.cs[i]);
+        }
         __syncthreads();
-        uint16_t* o16 = reinterpret_cast<uint16_t*>(S.qraw) + h * D;
-        o16[i] = y0;
-        o16[i + D / 2] = y1;
+        if (tid < NR) {
+          uint16_t* o16 = reinterpret_cast<uint16_t*>(S.qraw) + h * D;
+          o16[i] = y0;
+          o16[i + D / 2] = y1;
+        }
         __syncthreads();
         q32 = S.qraw;
       }
