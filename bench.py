@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-scorer measurement")
+    ap.add_argument("--only-prefill", action="store_true",
+                    help="run only the prefill-scorer measurement and print its JSON (for profiling it alone)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     return ap.parse_args()
 
@@ -484,6 +486,16 @@ def main():
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+    if args.only_prefill:
+        import torch
+
+        from block_sparse_attention_c4_b200 import build
+
+        build.build()
+        torch.cuda.set_device(local_rank)
+        if rank == 0:
+            print(json.dumps({"prefill_scorer": run_prefill_scorer(torch.device("cuda", local_rank))}), flush=True)
         return
     res, wl = run_ours(args, rank, world, local_rank)
     if rank == 0:
