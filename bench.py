@@ -100,6 +100,13 @@ class ClockSampler:
         self.gpu, self.proc, self.lines = gpu_index, None, []
 
     def start(self):
+        # NVML in a thread (10 ms period; read-only queries), else an nvidia-smi subprocess
+        self.stop_flag = threading.Event()
+        self.nv = self._nvml_handle()
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.t.start()
+            return
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "50"],
@@ -109,19 +116,57 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def _nvml_handle(self):
+        try:
+            import pynvml as nv
+            import torch
+
+            nv.nvmlInit()
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+                h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.h = h
+            return nv
+        except Exception:
+            return None
+
+    def _poll_nvml(self):
+        nv, h = self.nv, self.h
+        bits = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                r = int(get_reasons(h))
+                act = ["Active" if r & b else "Not Active" for b in bits.values()]
+                self.lines.append(", ".join([str(self.gpu), str(sm), str(mx), "0", hex(r)] + act))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self):
-        if self.proc is None:
+        if self.nv is not None:
+            self.stop_flag.set()
+            self.t.join(timeout=2)
+            src = "nvml, 10 ms"
+        elif self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.t.join(timeout=2)
+        else:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+            src = "nvidia-smi, 50 ms"
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
@@ -137,7 +182,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "sampler": src}
 
 
 def algorithmic_bytes(lens):

@@ -377,6 +377,7 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
   if (!layout(QSA_OP_SPARSE_GQA, nq, max_pos, L)) return QSA_ERR_INVALID_ARG;
   if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
   GqaParams p{};
+  p.cluster_merge = 1;
   p.c = view_of(cache);
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.nq_row = 1;
@@ -425,6 +426,7 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
                   nullptr, seq_len, 0, B, max_len, w, sel, sel_n, ws, L, st, ready);
   if (s != QSA_OK) return s;
   GqaParams p{};
+  p.cluster_merge = 1;
   p.c = cv;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.nq_row = 1;
@@ -462,6 +464,7 @@ qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_p
   if (!layout(QSA_OP_DECODE_INDEXSHARE, B, 1, L)) return QSA_ERR_INVALID_ARG;
   if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
   GqaParams p{};
+  p.cluster_merge = 1;
   p.c = view_of(cache);
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.nq_row = n_plus_1;

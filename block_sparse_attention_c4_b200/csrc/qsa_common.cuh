@@ -370,6 +370,31 @@ __device__ __forceinline__ int group_exclusive_scan(int v, int* warp_tot, int* t
   return res;
 }
 
+// The same with a single barrier: every thread adds up the warp totals before its own warp.  The
+// caller must pass another barrier before `warp_tot` is written again.
+template <class G>
+__device__ __forceinline__ int group_exclusive_scan_1b(int v, int* warp_tot, int* total) {
+  constexpr int NW = G::N / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  G::sync();
+  int before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int t = warp_tot[w];
+    before += w < warp ? t : 0;
+    tot += t;
+  }
+  *total = tot;
+  return before + x - v;
+}
+
 // ---------------------------------------------------------------------------
 // Exact top-k selection on 32-bit keys over a group (larger key first, then
 // lower index first).
@@ -773,7 +798,7 @@ __device__ void hist_topk(const uint32_t* keys, uint32_t* hist, int n, int k, Em
   }
   for (int i = tid; i < HT_MAX_N / 32; i += NT) sc->bits[i] = 0u;
   int tot;
-  const int ex = group_exclusive_scan<G>(local, sc->warp_tot, &tot);  // keys in bins above this thread's
+  const int ex = group_exclusive_scan_1b<G>(local, sc->warp_tot, &tot);  // keys in bins above this thread's
   if (ex < k && ex + local >= k) {
     int c = ex;
 #pragma unroll
@@ -865,7 +890,7 @@ __device__ void hist_topk(const uint32_t* keys, uint32_t* hist, int n, int k, Em
   G::sync();
   // (4) ordered emission
   uint32_t wbits = tid < nwords ? sc->bits[tid] : 0u;
-  int o = group_exclusive_scan<G>(__popc(wbits), sc->warp_tot, &tot);
+  int o = group_exclusive_scan_1b<G>(__popc(wbits), sc->warp_tot, &tot);
   while (wbits) {
     const int bit = __ffs(wbits) - 1;
     emit(tid * 32 + bit, o++);

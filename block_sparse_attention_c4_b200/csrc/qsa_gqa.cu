@@ -15,8 +15,13 @@
 // into a 4-deep, XOR-swizzled shared-memory ring.  Warp (g, d-half, m-tile):
 // S = Q_g K_g^T with m16n8k16 bf16 MMAs (rows = query heads of KV group g),
 // an online softmax in the log2 domain, and O += P V_g for its 64 output
-// dims.  Splits write (O, m, l) partials; the last CTA of the row (atomic
-// ticket, no waiting) merges them.
+// dims.  The splits of a row form one thread-block cluster: each leaves its
+// (O, m, l) partial in its own shared memory and, after a cluster barrier,
+// merges one slice of the row's outputs from all of them through distributed
+// shared memory.  (Without clusters -- the allocation-free entry point, or
+// more splits than a cluster holds -- partials go through global memory and
+// the last CTA of the row, by atomic ticket, merges them.)
+#include <cooperative_groups.h>
 #include <cstdlib>
 
 #include "qsa_common.cuh"
@@ -83,6 +88,12 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   // ---- launched early (programmatic dependent of the scorer): wait until this row's selection
   // is final; the queries above were loaded meanwhile ----
   if (p.row_ready) {
+    if (!bad) {  // the row's page-table lines into L2 meanwhile: the slots are looked up right after
+      const int L = __ldg(p.row_len + row) + p.len_offset;
+      const int npg = L >= 1 && L <= p.max_len ? min(ceil_div(L, PAGE), p.c.max_pages) : 0;
+      const int32_t* pt = p.c.page_table + (int64_t)req * p.c.max_pages;
+      for (int i = tid * 32; i < npg; i += THREADS * 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(pt + i));
+    }
     if (tid == 0 && !wait_ready(p.row_ready + row * READY_STRIDE, p.err)) S.is_last = -1;
     else if (tid == 0) S.is_last = 0;
     __syncthreads();
@@ -299,6 +310,76 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
     }
     return;
   }
+  if (p.cluster_merge) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    // own partial into the (now idle) ring: O [heads][128] fp32, then (m, l) per head
+    static_assert(32 * MT * D * 4 <= sizeof(S.kv), "O partial fits the ring");
+    constexpr bool ML_IN_RING = (32 * MT * D + 32 * MT * 2) * 4 <= sizeof(S.kv);
+    static_assert(ML_IN_RING || sizeof(S.qsep) >= 32 * MT * 2 * 4, "(m, l) partial fits");
+    __syncthreads();  // every warp is done with the ring
+    float* po_s = reinterpret_cast<float*>(S.kv[0]);
+    float* pml_s = ML_IN_RING ? po_s + 32 * MT * D : reinterpret_cast<float*>(S.qsep);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int d = dh * 64 + 8 * n + 2 * cq;
+      if (qi0 < nq) *reinterpret_cast<float2*>(po_s + (qi0 * HQ + h0) * D + d) = make_float2(o[n][0], o[n][1]);
+      if (qi1 < nq) *reinterpret_cast<float2*>(po_s + (qi1 * HQ + h1) * D + d) = make_float2(o[n][2], o[n][3]);
+    }
+    if (dh == 0 && cq == 0) {
+      if (qi0 < nq) *reinterpret_cast<float2*>(pml_s + (qi0 * HQ + h0) * 2) = make_float2(m0, l0);
+      if (qi1 < nq) *reinterpret_cast<float2*>(pml_s + (qi1 * HQ + h1) * 2) = make_float2(m1, l1);
+    }
+    cl.sync();
+    // this CTA's slice of (head, 4 dims) items, merged from every split's shared memory
+    const int ns = p.splits;  // the cluster size
+    const int rank = (int)cl.block_rank();
+    const int nitems = nh * (D / 4);
+    const int per = ceil_div(nitems, ns);
+    const int i_end = min(nitems, (rank + 1) * per);
+    __nv_bfloat16* out = p.out + (int64_t)row * nh * D;
+    for (int idx = rank * per + tid; idx < i_end; idx += THREADS) {
+      const int hh = idx / (D / 4), c4 = idx % (D / 4);
+      float2 ml[GQ_CLUSTER_MAX];
+      float4 ov[GQ_CLUSTER_MAX];
+#pragma unroll
+      for (int s2 = 0; s2 < GQ_CLUSTER_MAX; ++s2) {
+        ml[s2] = make_float2(-INFINITY, 0.f);
+        ov[s2] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s2 < ns) {
+          ml[s2] = *reinterpret_cast<const float2*>(cl.map_shared_rank(pml_s, s2) + hh * 2);
+          ov[s2] = *reinterpret_cast<const float4*>(cl.map_shared_rank(po_s, s2) + hh * D + c4 * 4);
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < GQ_CLUSTER_MAX; ++s2) M = fmaxf(M, ml[s2].x);
+      const float base = M == -INFINITY ? 0.f : M;
+      float den = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s2 = 0; s2 < GQ_CLUSTER_MAX; ++s2) {
+        const float wgt = exp2f(ml[s2].x - base);  // 0 for splits without positions
+        den += wgt * ml[s2].y;
+        acc.x += wgt * ov[s2].x;
+        acc.y += wgt * ov[s2].y;
+        acc.z += wgt * ov[s2].z;
+        acc.w += wgt * ov[s2].w;
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      uint2 pk;
+      pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+      pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(out + (int64_t)hh * D + c4 * 4) = pk;
+      if (p.lse && c4 == 0) {
+        constexpr float LN2 = 0.69314718055994530942f;
+        p.lse[(int64_t)row * nh + hh] = den > 0.f ? (M + log2f(den)) * LN2 : -INFINITY;
+      }
+    }
+    cl.sync();  // no CTA leaves while another still reads its shared memory
+    if (rank == 0 && tid == 0 && p.row_ready) p.row_ready[row * READY_STRIDE] = 0;  // ready for the next call
+    return;
+  }
   float* po = p.part_o + ((int64_t)row * p.splits + split) * nh * D;
   float* pml = p.part_ml + ((int64_t)row * p.splits + split) * nh * 2;
 #pragma unroll
@@ -468,19 +549,30 @@ static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, in
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  choose_splits<MT>(rows, max_pos, num_sms, bound, p.splits, p.tiles_per_split);
+  choose_splits<MT>(rows, max_pos, num_sms, p.cluster_merge ? min(bound, GQ_CLUSTER_MAX) : bound, p.splits,
+                    p.tiles_per_split);
+  if (p.splits < 2 || p.splits > GQ_CLUSTER_MAX) p.cluster_merge = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.splits, rows);
   cfg.blockDim = dim3(MT * 128);
   cfg.dynamicSmemBytes = gqa_smem_bytes<MT>(p.tiles_per_split);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  int na = 0;
   if (p.row_ready) {  // may start before the scorer ends; each CTA waits for its row's flag
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
   }
+  if (p.cluster_merge) {  // one cluster per row: its splits
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)p.splits;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = na ? attr : nullptr;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, k_sparse_gqa<MT>, p);
 }
 

@@ -93,7 +93,11 @@ struct GqaParams {
   int* err;
   int* row_ready;             // nullable (mode 0, [rows][READY_STRIDE]): wait for the row's flag, then clear it;
                               // the kernel is then launched as a programmatic dependent of the scorer
+  int cluster_merge;          // 1: a row's splits may form one thread-block cluster and merge their partials
+                              // through distributed shared memory (part_o, part_ml, counters unused);
+                              // 0: partials go through global memory, the last split merges them
 };
+constexpr int GQ_CLUSTER_MAX = 8;  // splits of one row in a cluster (portable cluster size)
 
 // Upper bound of the split count launch_gqa may choose (workspace sizing).
 int gqa_split_bound(int rows, int max_pos);

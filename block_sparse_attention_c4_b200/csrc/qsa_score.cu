@@ -77,6 +77,7 @@ struct ScoreSmem {
   uint32_t qraw[HI * D / 2];        // fused front end: unrotated query, then rotated (bf16 pairs)
   int warp_tot[33];
   int bcast[4];
+  int next_page;  // streaming: the next unclaimed page group of the segment
 };
 static_assert(SC_SEG_KEYS <= HT_MAX_N && SC_SEG_KEYS <= 32 * SC_THREADS, "a segment's keys fit one selection");
 static_assert(2 * HT_TIE_CAP >= TOPK && SC_MERGE_CAP > TOPK, "merge survivors fit the tie storage");
@@ -332,10 +333,14 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       coff = atomicAdd(p.cand_cnt + r, ncand);
     }
     ht_zero<Cta>(S.hist);
+    if (tid == 0) S.next_page = SC_WARPS * SC_U;
     Cta::sync();
 
-    // ---- stream: warp w scores pages w, w+8, ... (SC_U at a time) ----
-    for (int k0 = warp * SC_U; k0 < sg.np; k0 += SC_WARPS * SC_U) {
+    // ---- stream: warp w starts with pages w*U .. w*U+U-1, then claims the next U pages from a
+    // shared counter (claimed while its current pages load), so the warps end together ----
+    for (int k0 = warp * SC_U; k0 < sg.np;) {
+      int k_next = 0;
+      if (lane == 0) k_next = atomicAdd(&S.next_page, SC_U);
       PageRegs pr[SC_U];
 #pragma unroll
       for (int u = 0; u < SC_U; ++u) {
@@ -362,6 +367,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
           }
         }
       }
+      k0 = __shfl_sync(0xffffffffu, k_next, 0);
     }
     Cta::sync();
 
