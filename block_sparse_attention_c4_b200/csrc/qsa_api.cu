@@ -80,7 +80,7 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     scorer_sizing(max_len, w.ppc_min, w.seg_cap);
     if (w.seg_cap > SC_MAX_SEGS) return false;
     const int np_max = ceil_div(max_len / QSA_BLOCK, PAGE_BLOCKS);
-    if ((int64_t)rows * np_max >= (int64_t)INT32_MAX) return false;
+    if ((int64_t)rows * (np_max + SC_ROW_COST) >= (int64_t)INT32_MAX) return false;
     w.qrot = take((size_t)rows * HI * D * 2);
     w.sel = take((size_t)rows * TOPK * 4);
     w.sel_n = take((size_t)rows * 4);

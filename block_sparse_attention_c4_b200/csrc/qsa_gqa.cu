@@ -51,6 +51,11 @@ struct GqaSmem {
   alignas(128) uint8_t qsep[Q_IN_RING ? 16 : QBYTES];
   int is_last;
   int32_t slot[1];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
+  // cluster merge: the O partial (up to 32*MT heads x 128 fp32) in the ring, (m, l) after it or in qsep
+  static constexpr int PO_BYTES = 32 * MT * D * 4, PML_BYTES = 32 * MT * 2 * 4;
+  static constexpr bool ML_IN_RING = PO_BYTES + PML_BYTES <= GQ_STAGES * GQ_STAGE_BYTES;
+  static constexpr bool CLUSTER_FITS =
+      PO_BYTES <= GQ_STAGES * GQ_STAGE_BYTES && (ML_IN_RING || (Q_IN_RING ? 16 : QBYTES) >= PML_BYTES);
   __device__ __forceinline__ uint8_t* qrow(int g, int rho) {
     return (Q_IN_RING ? kv[GQ_STAGES - 1] : qsep) + (g * MT * 16 + rho) * GQ_ROW_BYTES;
   }
@@ -310,16 +315,13 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
     }
     return;
   }
-  if (p.cluster_merge) {
+  if (GqaSmem<MT>::CLUSTER_FITS && p.cluster_merge) {
     namespace cg = cooperative_groups;
     cg::cluster_group cl = cg::this_cluster();
     // own partial into the (now idle) ring: O [heads][128] fp32, then (m, l) per head
-    static_assert(32 * MT * D * 4 <= sizeof(S.kv), "O partial fits the ring");
-    constexpr bool ML_IN_RING = (32 * MT * D + 32 * MT * 2) * 4 <= sizeof(S.kv);
-    static_assert(ML_IN_RING || sizeof(S.qsep) >= 32 * MT * 2 * 4, "(m, l) partial fits");
     __syncthreads();  // every warp is done with the ring
     float* po_s = reinterpret_cast<float*>(S.kv[0]);
-    float* pml_s = ML_IN_RING ? po_s + 32 * MT * D : reinterpret_cast<float*>(S.qsep);
+    float* pml_s = GqaSmem<MT>::ML_IN_RING ? po_s + 32 * MT * D : reinterpret_cast<float*>(S.qsep);
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const int d = dh * 64 + 8 * n + 2 * cq;
@@ -530,6 +532,39 @@ static void choose_splits(int rows, int max_pos, int num_sms, int bound, int& sp
   tps = tiles;
 }
 
+// Clusters of `splits` CTAs that can be resident at once (device query, cached per device and
+// cluster size; the shared memory of the longest split, so an upper bound on what a launch uses).
+#ifndef QSA_GQA_CLUSTER_SLACK
+#define QSA_GQA_CLUSTER_SLACK 0  // percent of the cluster slots left free
+#endif
+template <int MT>
+static int active_clusters(int splits) {
+  static int cache[64][GQ_CLUSTER_MAX + 1] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || splits < 1 || splits > GQ_CLUSTER_MAX) return 0;
+  if (cache[dev][splits] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, 1);
+    cfg.blockDim = dim3(MT * 128);
+    cfg.dynamicSmemBytes = gqa_smem_bytes<MT>(GQ_MAX_TILES);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_sparse_gqa<MT>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cache[dev][splits] = n > 0 ? n : -1;
+  }
+  return max(cache[dev][splits], 0);
+}
+
 template <int MT>
 static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, int bound, cudaStream_t st) {
   static bool attr_set[64] = {false};
@@ -551,6 +586,17 @@ static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, in
   }
   choose_splits<MT>(rows, max_pos, num_sms, p.cluster_merge ? min(bound, GQ_CLUSTER_MAX) : bound, p.splits,
                     p.tiles_per_split);
+  if (!GqaSmem<MT>::CLUSTER_FITS) p.cluster_merge = 0;
+  if (p.cluster_merge) {
+    // every row's cluster resident at once (QSA_GQA_CLUSTER_SLACK percent of the slots spare): a
+    // cluster that finds no GPC with room for all its CTAs waits a whole CTA lifetime for one
+    const int tiles = ceil_div(max(max_pos, 1), GQ_TILE);
+    while (p.splits >= 2 &&
+           (int64_t)rows * 100 > (int64_t)active_clusters<MT>(p.splits) * (100 - QSA_GQA_CLUSTER_SLACK)) {
+      --p.splits;
+      p.tiles_per_split = ceil_div(tiles, p.splits);
+    }
+  }
   if (p.splits < 2 || p.splits > GQ_CLUSTER_MAX) p.cluster_merge = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.splits, rows);

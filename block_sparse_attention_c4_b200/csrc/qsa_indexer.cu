@@ -77,10 +77,11 @@ __global__ void __launch_bounds__(128) k_compress_append(CacheView c, const __nv
 // ring slot (L-1) mod 4, and when it completes block b = L/4 - 1 that block is
 // compressed from the ring slots 0..2 and the new key.  Always: the 4 index
 // query heads are rotated at position L-1 (L = row_len[row] + len_offset) and
-// stored as bf16 in qrot [rows][4][128]; row_pages[row] gets the number of
-// 64-token pages the scorer streams for the row (0 when it keeps every block
-// or the row is invalid), and the last CTA to finish (atomic ticket) writes
-// their exclusive prefix to page_off[0..rows].
+// stored as bf16 in qrot [rows][4][128]; row_pages[row] gets the length of the
+// row in the scorer's page list: the 64-token pages it streams plus
+// SC_ROW_COST empty ones in front (0 when it keeps every block or the row is
+// invalid), and the last CTA to finish (atomic ticket) writes their exclusive
+// prefix to page_off[0..rows].
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) k_index_prologue(CacheView c, const __nv_bfloat16* __restrict__ knew,
                                                         const __nv_bfloat16* __restrict__ idx_q,
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(128) k_index_prologue(CacheView c, const __nv_
   }
   if (row_pages == nullptr) return;
   const int nb = valid ? (L >> 2) : 0;
-  if (tid == 0) row_pages[row] = nb > TOPK ? ceil_div(nb, PAGE_BLOCKS) : 0;
+  if (tid == 0) row_pages[row] = nb > TOPK ? SC_ROW_COST + ceil_div(nb, PAGE_BLOCKS) : 0;
   __threadfence();
   __syncthreads();
   if (tid == 0) is_last = atomicAdd(ticket, 1) == rows - 1;

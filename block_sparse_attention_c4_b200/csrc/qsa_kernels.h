@@ -28,6 +28,13 @@ cudaError_t launch_expand(const int32_t* blocks, const int32_t* nblocks, const i
 constexpr int SC_MAX_SEG_PAGES = QSA_SC_WARPS >= 16 ? 1024 : 512;
 constexpr int SC_MAX_SEGS = 64;        // segments per row a merge can order
 constexpr int SC_MIN_PPC = 32;         // pages per CTA range, lower bound
+// Work of starting a row's segment (row setup, a partial top-512, its hand-over), in pages of
+// streaming: the page list gives every row this many empty pages in front of its own, so a range
+// that crosses into a row streams that many fewer pages.
+#ifndef QSA_SC_ROW_COST
+#define QSA_SC_ROW_COST 64
+#endif
+constexpr int SC_ROW_COST = QSA_SC_ROW_COST;
 
 struct ScoreParams {
   CacheView c;

@@ -8,12 +8,13 @@
 // ties keep the lower block index.
 //
 // Design (B200).  The pass is HBM-bound: 256 bytes of compressed key per block
-// against 4 dot products of 128.  Work is balanced exactly, whatever the mix
-// of context lengths: all pages to score (64 tokens = 16 compressed keys =
-// 4 KiB, contiguous because the cache is page aligned) are laid end to end
-// over the rows, and each persistent CTA (two per SM) owns equal contiguous
-// ranges of that list.  A range crosses at most a few rows; its piece of one
-// row is a "segment".
+// against 4 dot products of 128.  Work is balanced whatever the mix of context
+// lengths: all pages to score (64 tokens = 16 compressed keys = 4 KiB,
+// contiguous because the cache is page aligned) are laid end to end over the
+// rows, each row preceded by SC_ROW_COST empty pages that stand for the fixed
+// work of starting a segment, and each persistent CTA (one of 16 warps per SM)
+// owns an equal contiguous range of that list.  A range crosses at most a few
+// rows; its piece of one row is a "segment".
 //   * Pages sit at random places in HBM, so what bounds the pass is how many
 //     independent 4 KiB reads are in flight; a measured probe of this access
 //     pattern peaks with many warps each holding whole pages, not with one
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       if (r < rows) {
         int req, L;
         const int nb = row_of(r, req, L) ? (L >> 2) : 0;
-        pages = nb > TOPK ? ceil_div(nb, PAGE_BLOCKS) : 0;
+        pages = nb > TOPK ? SC_ROW_COST + ceil_div(nb, PAGE_BLOCKS) : 0;
       }
       int tot;
       const int ex = group_exclusive_scan<Cta>(pages, S.warp_tot, &tot);
@@ -251,7 +252,12 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     Segment sg;
     sg.row = row_of_page(off_s, p.page_off, rows, g);
     const int rend = off_at(sg.row + 1);
-    sg.p0 = g - off_at(sg.row);
+    const int rstart = off_at(sg.row) + SC_ROW_COST;  // the row's first page to stream
+    if (g < rstart) {  // the row's empty pages: nothing to do
+      g = min(rstart, gend);
+      continue;
+    }
+    sg.p0 = g - rstart;
     sg.np = min(min(gend, rend), g + SC_MAX_SEG_PAGES) - g;
     g += sg.np;
     if (sg.np <= 0) continue;
@@ -315,7 +321,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     const int nb = L >> 2;
     const int b0 = sg.p0 * PAGE_BLOCKS;
     const int nvalid = min(sg.np * PAGE_BLOCKS, nb - b0);
-    const int np_row = off_at(r + 1) - off_at(r);
+    const int np_row = off_at(r + 1) - off_at(r) - SC_ROW_COST;
     // The row's decode append is made by the CTA owning its last page, before that page is read;
     // when it completes block nb - 1 (in the last page), that page is read with coherent loads.
     int fresh_k = -1;
