@@ -214,14 +214,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           if (a_it >= PF_STAGES) mbar_wait(&S.empty_a[s], ((a_it / PF_STAGES) - 1) & 1, p.err);
           mbar_arrive_expect_tx(&S.full_a[s], PF_A_BYTES);
         }
-#pragma unroll
-        for (int pg = 0; pg < PF_M / PAGE_BLOCKS; ++pg) {
-          const int row = __shfl_sync(0xffffffffu, rows_cur, r * (PF_M / PAGE_BLOCKS) + pg);
-          if (lane == 0) {
-            tma_load_2d(S.a[s][0] + pg * PAGE_BLOCKS * 128, &kmap, 0, row, &S.full_a[s]);
-            tma_load_2d(S.a[s][1] + pg * PAGE_BLOCKS * 128, &kmap, 64, row, &S.full_a[s]);
-          }
-        }
+        __syncwarp();  // the stage is free (and its bytes expected) before any lane copies into it
+        // 16 lanes issue the M-tile's 16 copies at once: lane 2*pg + half copies the 64-dim half
+        // `half` of page pg (16 keys)
+        constexpr int PAGES = PF_M / PAGE_BLOCKS;  // 8 pages per M-tile
+        const int pg = (lane >> 1) & (PAGES - 1), half = lane & 1;
+        const int row = __shfl_sync(0xffffffffu, rows_cur, r * PAGES + pg);
+        if (lane < 2 * PAGES)
+          tma_load_2d(S.a[s][half] + pg * PAGE_BLOCKS * 128, &kmap, half * 64, row, &S.full_a[s]);
         if (r == GROUP - 1) rows_cur = rows_nxt;
       }
     }
