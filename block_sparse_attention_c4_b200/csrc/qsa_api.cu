@@ -22,8 +22,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WsLayout {
-  size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, seg_cnt = 0, cand_cnt = 0,
-         pages_done = 0, seg_tab = 0, cand_key = 0, cand_id = 0, part_o = 0, part_ml = 0, total = 0;
+  size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, pages_done = 0, cand_key = 0,
+         cand_id = 0, part_o = 0, part_ml = 0, total = 0;
   size_t pf_keys = 0, pf_ovf_n = 0, pf_ovf_list = 0;
   size_t ready = 0;  // decode: per-row flag, selection final (scorer -> sparse GQA)
   int ppc_min = 0;
@@ -86,10 +86,7 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     w.sel_n = take((size_t)rows * 4);
     w.row_pages = take((size_t)rows * 4);
     w.page_off = take((size_t)(rows + 1) * 4);
-    w.seg_cnt = take((size_t)rows * 4);
-    w.cand_cnt = take((size_t)rows * 4);
     w.pages_done = take((size_t)rows * 4);
-    w.seg_tab = take((size_t)rows * w.seg_cap * 16);
     w.cand_key = take((size_t)rows * w.seg_cap * TOPK * 4);
     w.cand_id = take((size_t)rows * w.seg_cap * TOPK * 4);
   }
@@ -218,9 +215,6 @@ qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_b
   p.page_off = at<int32_t>(ws, L.page_off);
   p.ppc_min = L.ppc_min;
   p.seg_cap = L.seg_cap;
-  p.seg_tab = at<int4>(ws, L.seg_tab);
-  p.seg_cnt = at<int>(ws, L.seg_cnt);
-  p.cand_cnt = at<int>(ws, L.cand_cnt);
   p.pages_done = at<int>(ws, L.pages_done);
   p.cand_key = at<uint32_t>(ws, L.cand_key);
   p.cand_id = at<int32_t>(ws, L.cand_id);

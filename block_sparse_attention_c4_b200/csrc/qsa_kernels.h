@@ -47,10 +47,8 @@ struct ScoreParams {
   const float* w;             // [rows][4]
   const int32_t* page_off;    // [rows + 1] exclusive prefix of pages to score per row
   int ppc_min;                // pages per CTA range, lower bound
-  int seg_cap;                // segment slots per row
-  int4* seg_tab;              // [rows][seg_cap] (first block, candidate offset, count, -)
-  int* seg_cnt;               // [rows], zero between calls
-  int* cand_cnt;              // [rows], zero between calls
+  int seg_cap;                // segment slots per row (a partial segment's 512 candidates go to slot j,
+                              // its rank among the row's segments in block order)
   int* pages_done;            // [rows], zero between calls
   uint32_t* cand_key;         // [rows][seg_cap * 512]
   int32_t* cand_id;           // [rows][seg_cap * 512]

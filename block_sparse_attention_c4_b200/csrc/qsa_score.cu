@@ -101,6 +101,21 @@ __device__ __forceinline__ int row_of_page(const int32_t* off_s, const int32_t* 
   return lo;
 }
 
+// The segments of a row, in block order: its pages (page-list interval [rs, re)) cut at every range
+// boundary (multiples of ppc) and every SC_MAX_SEG_PAGES pages from a range piece's start -- the
+// same cuts the segment loop makes.  Calls f(j, first page in the list, pages) for segment j and
+// returns the number of segments.  A partial segment's candidates go to slot j of the row's list.
+template <class F>
+__device__ __forceinline__ int for_each_segment(int rs, int re, int ppc, F f) {
+  int j = 0;
+  for (int g = rs; g < re;) {
+    const int e = min(re, (g / ppc + 1) * ppc);
+    for (int a = g; a < e; a += SC_MAX_SEG_PAGES, ++j) f(j, a, min(e, a + SC_MAX_SEG_PAGES) - a);
+    g = e;
+  }
+  return j;
+}
+
 #ifndef QSA_SC_L2_PROMOTE
 #define QSA_SC_L2_PROMOTE 0
 #endif
@@ -259,6 +274,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     }
     sg.p0 = g - rstart;
     sg.np = min(min(gend, rend), g + SC_MAX_SEG_PAGES) - g;
+    const int g_seg = g;
     g += sg.np;
     if (sg.np <= 0) continue;
     const int r = sg.row;
@@ -329,15 +345,12 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       if (warp == 0) warp_decode_append(p.c, req, L, p.knew + (int64_t)r * D, p.fr, p.err);
       if ((L & 3) == 0) fresh_k = sg.np - 1;
     }
-    // A segment that is not the whole row reserves its candidate slots now; the results are first
-    // used after the streaming, so the atomics' round trip hides behind it.
+    // A segment that is not the whole row writes its candidates to slot `ord` of the row's list:
+    // its rank among the row's segments, in block order.
     const bool partial = sg.np != np_row;
     const int ncand = min(nvalid, TOPK);
-    int slot = 0, coff = 0;
-    if (tid == 0 && partial) {
-      slot = atomicAdd(p.seg_cnt + r, 1);
-      coff = atomicAdd(p.cand_cnt + r, ncand);
-    }
+    int ord = 0;
+    if (partial) for_each_segment(rstart, rend, ppc, [&](int j, int a, int) { ord = a < g_seg ? j + 1 : ord; });
     ht_zero<Cta>(S.hist);
     if (tid == 0) S.next_page = SC_WARPS * SC_U;
     Cta::sync();
@@ -387,21 +400,12 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
       }
       continue;
     }
-    if (tid == 0) {
-      const bool fits = slot < p.seg_cap && coff + ncand <= p.seg_cap * TOPK;
-      if (!fits) {  // more segments than the workspace was sized for: drop this one, flag it
-        set_error(p.err, QSA_DEVERR_SELECTION);
-        coff = -1;
-      }
-      if (slot < p.seg_cap)
-        p.seg_tab[(int64_t)r * p.seg_cap + slot] = make_int4(b0, fits ? coff : 0, fits ? ncand : 0, 0);
-      S.bcast[0] = coff;
-    }
-    Cta::sync();
-    coff = S.bcast[0];
-    if (coff >= 0) {
-      uint32_t* ck = p.cand_key + (int64_t)r * p.seg_cap * TOPK + coff;
-      int32_t* ci = p.cand_id + (int64_t)r * p.seg_cap * TOPK + coff;
+    const int seg_slots = min(p.seg_cap, SC_MAX_SEGS);
+    if (ord >= seg_slots) {  // more segments than the workspace was sized for: drop this one, flag it
+      if (tid == 0) set_error(p.err, QSA_DEVERR_SELECTION);
+    } else {
+      uint32_t* ck = p.cand_key + ((int64_t)r * p.seg_cap + ord) * TOPK;
+      int32_t* ci = p.cand_id + ((int64_t)r * p.seg_cap + ord) * TOPK;
       auto put = [&](int i, int o) {
         ck[o] = S.keys[i];
         ci[o] = b0 + i;
@@ -419,29 +423,25 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     if (!S.bcast[1]) continue;
 
     // ---- this CTA finished the row: merge its segments' candidates ----
+    // The segments, their first blocks and candidate counts follow from the page list alone.
     __threadfence();
-    const int ns = min(__ldcg(p.seg_cnt + r), min(p.seg_cap, SC_MAX_SEGS));
-    const int4* tab = p.seg_tab + (int64_t)r * p.seg_cap;
-    // order the segments by first block (rank sort in shared memory; the starts are distinct)
-    int4* raw = reinterpret_cast<int4*>(S.keys);
-    for (int j = tid; j < ns; j += SC_THREADS) raw[j] = __ldcg(tab + j);
-    Cta::sync();
-    for (int j = tid; j < ns; j += SC_THREADS) {
-      const int4 e = raw[j];
-      int rank = 0;
-      for (int m = 0; m < ns; ++m) rank += raw[m].x < e.x;
-      S.segs[rank] = e;
-    }
-    Cta::sync();
     if (tid == 0) {
-      int acc = 0;
-      for (int j = 0; j < ns; ++j) {
+      const int seg_slots = min(p.seg_cap, SC_MAX_SEGS);
+      int acc = 0, ns_ = 0;
+      for_each_segment(rstart, rend, ppc, [&](int j, int a, int npg) {
+        if (j >= seg_slots) return;  // dropped by its writer (flagged there)
+        const int sb0 = (a - rstart) * PAGE_BLOCKS;
+        const int cnt = min(min(npg * PAGE_BLOCKS, nb - sb0), TOPK);
+        S.segs[j] = make_int4(sb0, j * TOPK, cnt, 0);
         S.vstart[j] = acc;
-        acc += S.segs[j].z;
-      }
-      S.vstart[ns] = acc;
+        acc += cnt;
+        ns_ = j + 1;
+      });
+      S.vstart[ns_] = acc;
+      S.bcast[2] = ns_;
     }
     Cta::sync();
+    const int ns = S.bcast[2];
     const uint32_t* rk = p.cand_key + (int64_t)r * p.seg_cap * TOPK;
     const int32_t* ri = p.cand_id + (int64_t)r * p.seg_cap * TOPK;
     // virtual index v (ascending block order) -> index into the row's candidate list
@@ -511,9 +511,7 @@ __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(S
     if (tid == 0) {
       if (kk_sel < TOPK) set_error(p.err, QSA_DEVERR_SELECTION);
       p.sel_n[r] = kk_sel;
-      p.seg_cnt[r] = 0;  // ready for the next call
-      p.cand_cnt[r] = 0;
-      p.pages_done[r] = 0;
+      p.pages_done[r] = 0;  // ready for the next call
       if (p.row_ready) publish_ready(p.row_ready + r * READY_STRIDE);
     }
     Cta::sync();
