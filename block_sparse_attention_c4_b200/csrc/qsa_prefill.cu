@@ -375,8 +375,8 @@ constexpr int PW_BINS = 256;
 constexpr int PW_L3 = 64;
 
 struct __align__(16) PwWarp {
-  uint32_t lkey[PW_LIST * 32];  // [slot][lane]
-  uint16_t lidx[PW_LIST * 32];
+  uint32_t lkey[(PW_LIST + 1) * 32];  // [slot][lane]; slot PW_LIST is a spare for writes past a full list
+  uint16_t lidx[(PW_LIST + 1) * 32];
   uint32_t hist[PW_BINS];
   uint32_t bitmap[PW_FAST_N / 32];
   uint32_t k3[PW_L3];
@@ -528,15 +528,14 @@ __global__ void __launch_bounds__(PW_WARPS * 32) k_prefill_select(PrefillParams 
           if (c >= nch) break;
           const int b0 = c * PF_M + 4 * lane;
           const uint32_t kk[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          // branch-free: every key is written to the lane's next slot, which advances only for a
+          // key >= L; past a full list the writes go to a spare slot (the row then overflows)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            if (kk[e] >= L && (c < nfull || b0 + e < n)) {
-              if (lc < PW_LIST) {
-                W.lkey[lc * 32 + lane] = kk[e];
-                W.lidx[lc * 32 + lane] = (uint16_t)(b0 + e);
-              }
-              ++lc;
-            }
+            const int slot = min(lc, PW_LIST) * 32 + lane;
+            W.lkey[slot] = kk[e];
+            W.lidx[slot] = (uint16_t)(b0 + e);
+            lc += (kk[e] >= L && (c < nfull || b0 + e < n)) ? 1 : 0;
           }
         }
       }
