@@ -28,10 +28,12 @@
 // the MMAs.  Work tiles are ordered longest first (causal imbalance) and dealt
 // to CTAs in a snake.
 //
-// Selection (k_prefill_select): one CTA per query row, longest rows first;
-// the row's keys are staged in shared memory (or read through L2 when longer
-// than the stage) and the exact top-512 by (score desc, block asc) is taken
-// by fast_topk, which emits the kept blocks in ascending order.
+// Selection (k_prefill_select): one warp per query row, longest rows first:
+// a lower bound from a sample of the row's keys, one pass collecting the keys
+// at or above it, the exact cut among those (score desc, block asc), and the
+// kept blocks written in ascending order.  Rows that do not fit that path
+// (longer than 8192 blocks, heavy ties, a bound that keeps too few or too
+// many) go to k_prefill_select_overflow: an exact CTA-wide selection.
 #include <mutex>
 
 #include "qsa_common.cuh"
@@ -173,8 +175,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     // =============================== TMA producer ===============================
     // The whole warp walks the schedule: lane i fetches the physical page of
     // logical page 32g + i for the group g of four M-tiles (32 pages) ahead of
-    // use, and lane 0 issues the copies, so no page-table load sits on the
-    // path of a copy.
+    // use, so no page-table load sits on the path of a copy; lane 0 waits for
+    // the stage and expects its bytes, then 16 lanes issue one copy each.
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&qmap);
