@@ -348,43 +348,72 @@ def decode_kernel_count(batch: int) -> int:
     return int(lib().qsa_decode_kernel_count(int(batch)))
 
 
+class PackedInputs:
+    """A decode step's inputs as 256-byte-aligned views of one contiguous buffer, so that a step
+    moves them host -> device with a single copy.  `views` maps each input name to its tensor."""
+
+    ALIGN = 256
+
+    def __init__(self, specs, device=None, pin_memory: bool = False):
+        offs, off = {}, 0
+        for name, shape, dtype in specs:
+            nbytes = int(torch.Size(shape).numel()) * torch.empty((), dtype=dtype).element_size()
+            offs[name] = (off, shape, dtype, nbytes)
+            off += (nbytes + self.ALIGN - 1) // self.ALIGN * self.ALIGN
+        self.nbytes = off
+        self.buf = torch.empty(off, dtype=torch.uint8, device=device, pin_memory=pin_memory)
+        self.views = {name: self.buf[o:o + n].view(dt).view(sh) for name, (o, sh, dt, n) in offs.items()}
+        self.payload_bytes = sum(n for (_, _, _, n) in offs.values())
+
+    def copy_from(self, other: "PackedInputs", non_blocking: bool = True):
+        self.buf.copy_(other.buf, non_blocking=non_blocking)
+
+
 class DecodeSession:
     """Decode steps fed from host memory: the call a serving loop makes once per step.
 
-    step() copies the step's inputs from (pinned) host tensors to device staging buffers, runs
-    qsa_decode, and copies the attention output back to a pinned host tensor, all on one stream.
+    step() copies the step's inputs from a pinned host buffer to a device staging buffer (one
+    copy: both hold the inputs packed the same way), runs qsa_decode, and copies the attention
+    output back to a pinned host tensor, all on one stream.
     """
 
     INPUTS = ("idx_k_new", "idx_q", "w", "q", "seq_len")
+
+    @staticmethod
+    def input_specs(B: int):
+        bf = torch.bfloat16
+        return [("idx_k_new", (B, HEAD_DIM), bf), ("idx_q", (B, INDEX_HEADS, HEAD_DIM), bf),
+                ("w", (B, INDEX_HEADS), torch.float32), ("q", (B, Q_HEADS, HEAD_DIM), bf),
+                ("seq_len", (B,), torch.int32)]
 
     def __init__(self, cache: LayerCache, max_len: int, device="cuda"):
         B = cache.batch
         self.cache, self.max_len = cache, int(max_len)
         self.ws = Workspace(workspace_bytes(OP_DECODE, B, self.max_len), device=device)
-        bf = torch.bfloat16
-        self.dev = {
-            "idx_k_new": torch.empty(B, HEAD_DIM, dtype=bf, device=device),
-            "idx_q": torch.empty(B, INDEX_HEADS, HEAD_DIM, dtype=bf, device=device),
-            "w": torch.empty(B, INDEX_HEADS, dtype=torch.float32, device=device),
-            "q": torch.empty(B, Q_HEADS, HEAD_DIM, dtype=bf, device=device),
-            "seq_len": torch.empty(B, dtype=torch.int32, device=device),
-        }
-        self.out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=bf, device=device)
-        self.host_out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=bf, pin_memory=True)
+        self.staging = PackedInputs(self.input_specs(B), device=device)
+        self.dev = self.staging.views
+        self.out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.host_out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, pin_memory=True)
 
     @staticmethod
-    def pinned_inputs(device_inputs: dict) -> dict:
-        return {k: device_inputs[k].cpu().pin_memory() for k in DecodeSession.INPUTS}
+    def pinned_inputs(device_inputs: dict) -> PackedInputs:
+        """The step's inputs packed into one pinned host buffer (what step() takes)."""
+        B = int(device_inputs["seq_len"].shape[0])
+        host = PackedInputs(DecodeSession.input_specs(B), pin_memory=True)
+        for k in DecodeSession.INPUTS:
+            host.views[k].copy_(device_inputs[k].cpu())
+        return host
 
     def h2d_bytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in self.dev.values())
+        return self.staging.payload_bytes
 
     def d2h_bytes(self) -> int:
         return self.host_out.numel() * self.host_out.element_size()
 
-    def step(self, host_inputs: dict, stream=None) -> torch.Tensor:
-        for k, t in self.dev.items():
-            t.copy_(host_inputs[k], non_blocking=True)
+    def step(self, host_inputs: PackedInputs, stream=None) -> torch.Tensor:
+        if host_inputs.nbytes != self.staging.nbytes:
+            raise QsaError("host inputs were packed for another batch size")
+        self.staging.copy_from(host_inputs)
         decode(self.cache, self.dev["idx_k_new"], self.dev["idx_q"], self.dev["w"], self.dev["q"],
                self.dev["seq_len"], self.max_len, self.ws, out=self.out, stream=stream)
         self.host_out.copy_(self.out, non_blocking=True)

@@ -129,3 +129,31 @@ def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(Q, "_lib", None)
     with pytest.raises(Q.QsaError):
         Q.lib()
+
+
+def test_decode_inputs_pack_into_one_buffer():
+    """A decode step's host inputs are views of one contiguous buffer, so a step moves them with a
+    single copy; the views keep their dtypes, shapes and 256-byte alignment, and a buffer-to-buffer
+    copy carries every input (CPU tensors here; the session does the same host -> device)."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+
+    B = 5
+    specs = Q.DecodeSession.input_specs(B)
+    src = Q.PackedInputs(specs)
+    dst = Q.PackedInputs(specs)
+    g = torch.Generator().manual_seed(3)
+    for name, shape, dtype in specs:
+        v = src.views[name]
+        assert v.shape == torch.Size(shape) and v.dtype == dtype and v.is_contiguous()
+        assert (v.data_ptr() - src.buf.data_ptr()) % Q.PackedInputs.ALIGN == 0
+        if dtype == torch.int32:
+            v.copy_(torch.randint(0, 1 << 20, shape, generator=g, dtype=torch.int32))
+        else:
+            v.copy_(torch.randn(shape, generator=g).to(dtype))
+    dst.copy_from(src, non_blocking=False)
+    for name, _, _ in specs:
+        assert torch.equal(dst.views[name], src.views[name])
+    assert src.payload_bytes == B * (128 * 2 + 4 * 128 * 2 + 4 * 4 + 16 * 128 * 2 + 4)
+    assert set(n for n, _, _ in specs) == set(Q.DecodeSession.INPUTS)
