@@ -28,6 +28,8 @@ MAX_DRAFT = 8
 
 OP_INDEX_SCORE_TOPK, OP_SPARSE_GQA, OP_DECODE, OP_DECODE_INDEXSHARE, OP_COMPRESS_APPEND = 1, 2, 3, 4, 5
 OP_PREFILL_SCORE_TOPK = 6
+OP_DECODE_INDEXER, OP_DECODE_ATTEND = 7, 8
+PROJ_FEATURES = INDEX_HEADS * HEAD_DIM + HEAD_DIM + INDEX_HEADS  # 644
 
 DEVERR_BITS = {1: "page", 2: "length", 4: "position", 8: "request", 16: "selection", 32: "timeout"}
 
@@ -50,7 +52,8 @@ EXPORTS = [
     "qsa_workspace_bytes", "qsa_workspace_init", "qsa_compress_append", "qsa_index_score_topk",
     "qsa_expand_indices", "qsa_sparse_gqa", "qsa_decode", "qsa_decode_indexshare", "qsa_device_error",
     "qsa_set_profile_events", "qsa_decode_kernel_count", "qsa_status_string", "qsa_version",
-    "qsa_prefill_score_topk",
+    "qsa_prefill_score_topk", "qsa_sparse_gqa_noalloc", "qsa_check_bounded_wait", "qsa_last_error_string",
+    "qsa_index_project", "qsa_decode_indexer", "qsa_decode_attend",
 ]
 
 
@@ -77,6 +80,13 @@ def lib():
     L.qsa_decode_indexshare.argtypes = [cp, vp, vp, i32, vp, i32, vp, f32, vp, vp, sz, vp]
     L.qsa_sparse_gqa_noalloc.argtypes = [cp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp]
     L.qsa_sparse_gqa_noalloc.restype = ctypes.c_int
+    L.qsa_index_project.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp]
+    L.qsa_decode_indexer.argtypes = [cp, vp, vp, i32, vp, i32, vp, vp, vp, sz, vp]
+    L.qsa_decode_attend.argtypes = [cp, vp, vp, i32, vp, vp, f32, vp, vp, vp, sz, vp]
+    for f in (L.qsa_index_project, L.qsa_decode_indexer, L.qsa_decode_attend):
+        f.restype = ctypes.c_int
+    L.qsa_check_bounded_wait.argtypes = [cp, vp, vp, ctypes.c_uint64, vp, sz, vp]
+    L.qsa_check_bounded_wait.restype = ctypes.c_int
     L.qsa_device_error.argtypes = [vp, i32, vp]
     L.qsa_device_error.restype = i32
     L.qsa_set_profile_events.argtypes = [ctypes.POINTER(vp), i32]
@@ -334,6 +344,71 @@ def decode_indexshare(cache: LayerCache, frozen_pos, frozen_n, len0, q, ws: Work
     return out
 
 
+def index_project(x, w_proj, idx_q=None, idx_k=None, w=None, stream=None):
+    """Hidden states x [n, hidden] -> (idx_q [n,4,128] bf16, idx_k [n,128] bf16, w [n,4] f32)."""
+    n, hidden = int(x.shape[0]), int(x.shape[1])
+    dev = x.device
+    _dev(x, torch.bfloat16, "x", (n, hidden))
+    _dev(w_proj, torch.bfloat16, "w_proj", (PROJ_FEATURES, hidden))
+    idx_q = torch.empty(n, INDEX_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=dev) if idx_q is None else idx_q
+    idx_k = torch.empty(n, HEAD_DIM, dtype=torch.bfloat16, device=dev) if idx_k is None else idx_k
+    w = torch.empty(n, INDEX_HEADS, dtype=torch.float32, device=dev) if w is None else w
+    _dev(idx_q, torch.bfloat16, "idx_q", (n, INDEX_HEADS, HEAD_DIM))
+    _dev(idx_k, torch.bfloat16, "idx_k", (n, HEAD_DIM))
+    _dev(w, torch.float32, "w", (n, INDEX_HEADS))
+    _check(lib().qsa_index_project(_ptr(x), _ptr(w_proj), n, hidden, _ptr(idx_q), _ptr(idx_k), _ptr(w),
+                                   _stream(stream)), "qsa_index_project")
+    return idx_q, idx_k, w
+
+
+def decode_indexer(cache: LayerCache, x, w_proj, seq_len, max_len: int, ws: Workspace, blocks=None, nblocks=None,
+                   stream=None):
+    """Index phase of a decode step from the new tokens' hidden states: projection, append, scoring,
+    top-512.  Returns (blocks [B,512], nblocks [B])."""
+    B = cache.batch
+    hidden = int(x.shape[1])
+    dev = x.device
+    blocks = torch.full((B, TOPK), -1, dtype=torch.int32, device=dev) if blocks is None else blocks
+    nblocks = torch.zeros(B, dtype=torch.int32, device=dev) if nblocks is None else nblocks
+    c = cache.struct()
+    _dev(blocks, torch.int32, "blocks", (B, TOPK))
+    _dev(nblocks, torch.int32, "nblocks", (B,))
+    _check(lib().qsa_decode_indexer(ctypes.byref(c), _ptr(_dev(x, torch.bfloat16, "x", (B, hidden))),
+                                    _ptr(_dev(w_proj, torch.bfloat16, "w_proj", (PROJ_FEATURES, hidden))), hidden,
+                                    _ptr(_dev(seq_len, torch.int32, "seq_len", (B,))), int(max_len), _ptr(blocks),
+                                    _ptr(nblocks), ws.ptr, ws.nbytes, _stream(stream)), "qsa_decode_indexer")
+    return blocks, nblocks
+
+
+def decode_attend(cache: LayerCache, q, seq_len, max_len: int, blocks, nblocks, ws: Workspace,
+                  scale: float | None = None, out=None, lse=None, stream=None):
+    """Attention phase of a decode step over the indexer's kept blocks plus each request's tail."""
+    B = cache.batch
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device) if out is None else out
+    c = cache.struct()
+    _dev(out, torch.bfloat16, "out", (B, Q_HEADS, HEAD_DIM))
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (B, Q_HEADS))
+    _check(lib().qsa_decode_attend(ctypes.byref(c), _ptr(_dev(q, torch.bfloat16, "q", (B, Q_HEADS, HEAD_DIM))),
+                                   _ptr(_dev(seq_len, torch.int32, "seq_len", (B,))), int(max_len),
+                                   _ptr(_dev(blocks, torch.int32, "blocks", (B, TOPK))),
+                                   _ptr(_dev(nblocks, torch.int32, "nblocks", (B,))), float(scale), _ptr(out),
+                                   _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)), "qsa_decode_attend")
+    return out
+
+
+def check_bounded_wait(cache: LayerCache, q, out, limit_ns: int, ws: Workspace, stream=None):
+    """Launch the decode attention for request 0 with a selection nothing publishes and a wait limit of
+    `limit_ns`: the kernel gives up, records the timeout bit in ws's error word and writes zeros to `out`."""
+    c = cache.struct()
+    _dev(q, torch.bfloat16, "q", (Q_HEADS, HEAD_DIM))
+    _dev(out, torch.bfloat16, "out", (Q_HEADS, HEAD_DIM))
+    _check(lib().qsa_check_bounded_wait(ctypes.byref(c), _ptr(q), _ptr(out), int(limit_ns), ws.ptr, ws.nbytes,
+                                        _stream(stream)), "qsa_check_bounded_wait")
+    return out
+
+
 def set_profile_events(events):
     """events: list of torch.cuda.Event (2 per kernel: start, end), or None to switch off."""
     if not events:
@@ -411,10 +486,14 @@ class DecodeSession:
         return self.host_out.numel() * self.host_out.element_size()
 
     def step(self, host_inputs: PackedInputs, stream=None) -> torch.Tensor:
+        """One step on `stream` (default: the current stream): both copies and the decode are enqueued
+        on that one stream, in order.  The returned pinned tensor is valid once the stream is done."""
         if host_inputs.nbytes != self.staging.nbytes:
             raise QsaError("host inputs were packed for another batch size")
-        self.staging.copy_from(host_inputs)
-        decode(self.cache, self.dev["idx_k_new"], self.dev["idx_q"], self.dev["w"], self.dev["q"],
-               self.dev["seq_len"], self.max_len, self.ws, out=self.out, stream=stream)
-        self.host_out.copy_(self.out, non_blocking=True)
+        st = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(st):
+            self.staging.copy_from(host_inputs)
+            decode(self.cache, self.dev["idx_k_new"], self.dev["idx_q"], self.dev["w"], self.dev["q"],
+                   self.dev["seq_len"], self.max_len, self.ws, out=self.out, stream=st)
+            self.host_out.copy_(self.out, non_blocking=True)
         return self.host_out

@@ -26,6 +26,7 @@ struct WsLayout {
          cand_id = 0, part_o = 0, part_ml = 0, total = 0;
   size_t pf_keys = 0, pf_ovf_n = 0, pf_ovf_list = 0;
   size_t ready = 0;  // decode: per-row flag, selection final (scorer -> sparse GQA)
+  size_t pj_q = 0, pj_k = 0, pj_w = 0;  // decode indexer: projected index queries, keys, head weights
   int ppc_min = 0;
   int seg_cap = 0;
   int splits_bound = 0;
@@ -55,10 +56,12 @@ int positions_bound(int op, int max_len) {
 // Workspace carving.  Returns false for invalid arguments.
 bool layout(int op, int rows, int max_len, WsLayout& w) {
   if (rows < 0 || max_len < 0 || max_len > QSA_MAX_CONTEXT) return false;
-  const bool scorer = op == QSA_OP_INDEX_SCORE_TOPK || op == QSA_OP_DECODE;
-  const bool gqa = op == QSA_OP_SPARSE_GQA || op == QSA_OP_DECODE || op == QSA_OP_DECODE_INDEXSHARE;
+  const bool scorer = op == QSA_OP_INDEX_SCORE_TOPK || op == QSA_OP_DECODE || op == QSA_OP_DECODE_INDEXER;
+  const bool gqa = op == QSA_OP_SPARSE_GQA || op == QSA_OP_DECODE || op == QSA_OP_DECODE_INDEXSHARE ||
+                   op == QSA_OP_DECODE_ATTEND;
   const bool prefill = op == QSA_OP_PREFILL_SCORE_TOPK;
   if (!scorer && !gqa && !prefill && op != QSA_OP_COMPRESS_APPEND) return false;
+  if (op == QSA_OP_DECODE_ATTEND) op = QSA_OP_DECODE;  // the decode step's attention part
   size_t off = 256;  // error word, prologue ticket, spare
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -76,6 +79,11 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
   }
   w.cnt_gqa = take(sizeof(int) * (size_t)rows);
   if (op == QSA_OP_DECODE) w.ready = take(sizeof(int) * READY_STRIDE * (size_t)rows);
+  if (op == QSA_OP_DECODE_INDEXER) {
+    w.pj_q = take((size_t)rows * HI * D * 2);
+    w.pj_k = take((size_t)rows * D * 2);
+    w.pj_w = take((size_t)rows * HI * 4);
+  }
   if (scorer) {
     scorer_sizing(max_len, w.ppc_min, w.seg_cap);
     if (w.seg_cap > SC_MAX_SEGS) return false;
@@ -120,17 +128,11 @@ RopeFreqs make_freqs(double theta) {
 }
 
 qsa_status check_cache(const qsa_cache* c) {
-  if (!c) return QSA_ERR_INVALID_ARG;
-  if (!c->k || !c->v || !c->cidx || !c->ring || !c->page_table) return QSA_ERR_INVALID_ARG;
-  if (c->page_size != QSA_PAGE_SIZE) return QSA_ERR_UNSUPPORTED;
-  if (c->num_slots <= 0 || c->num_slots % QSA_PAGE_SIZE != 0) return QSA_ERR_INVALID_ARG;
-  if (c->num_slots / QSA_PAGE_SIZE > (int64_t)INT32_MAX / QSA_PAGE_SIZE) return QSA_ERR_UNSUPPORTED;
-  if (c->max_pages <= 0 || c->batch < 0) return QSA_ERR_INVALID_ARG;
+  const qsa_status s = check_kv_cache(c);
+  if (s != QSA_OK) return s;
+  if (!c->cidx || !c->ring) return QSA_ERR_INVALID_ARG;
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) return QSA_ERR_INVALID_ARG;
-  if (c->kv_stride != 0 && (c->kv_stride < HKV * D || c->kv_stride % 8 != 0)) return QSA_ERR_INVALID_ARG;
-  if (!aligned(c->k, 16) || !aligned(c->v, 16) || !aligned(c->cidx, 16) || !aligned(c->ring, 16) ||
-      !aligned(c->page_table, 4))
-    return QSA_ERR_INVALID_ARG;
+  if (!aligned(c->cidx, 16) || !aligned(c->ring, 16)) return QSA_ERR_INVALID_ARG;
   return QSA_OK;
 }
 
@@ -188,14 +190,14 @@ qsa_status cuda_status(cudaError_t e) {
 qsa_status run_indexer(const qsa_cache* cache, const CacheView& cv, const __nv_bfloat16* knew,
                        const __nv_bfloat16* idx_q, const int32_t* row_req, const int32_t* row_len, int len_offset,
                        int rows, int max_len, const float* w, int32_t* sel, int32_t* sel_n, void* ws,
-                       const WsLayout& L, cudaStream_t st, int* row_ready = nullptr) {
+                       const WsLayout& L, cudaStream_t st, int* row_ready = nullptr, int ev0 = 0) {
   const RopeFreqs fr = make_freqs(cache->rope_theta);
   int* err = at<int>(ws, WS_ERR);
   __nv_bfloat16* qrot = at<__nv_bfloat16>(ws, L.qrot);
   // Up to SC_ROWS_SMEM rows the scorer runs the front end itself (append, rotation, page prefix);
   // above that a separate prologue kernel does it first.
   const bool fused = rows <= SC_ROWS_SMEM;
-  int ev = 0;
+  int ev = ev0;
   if (!fused) {
     ProfScope ps(st, ev++);
     cudaError_t e = launch_index_prologue(cv, knew, idx_q, row_req, row_len, len_offset, rows, max_len, fr, qrot,
@@ -361,7 +363,7 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
                           void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
   qsa_status s = check_cache(cache);
   if (s != QSA_OK) return s;
-  if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !(scale > 0.f) || !std::isfinite(scale))
+  if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !valid_scale(scale))
     return QSA_ERR_INVALID_ARG;
   if (max_pos > QSA_MAX_SEL) return QSA_ERR_UNSUPPORTED;
   if (nq == 0) return QSA_OK;
@@ -395,7 +397,7 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
                       int32_t* blocks_out, int32_t* nblocks_out, void* ws, size_t ws_bytes, void* stream) {
   qsa_status s = check_cache(cache);
   if (s != QSA_OK) return s;
-  if (max_len < 1 || max_len > QSA_MAX_CONTEXT || !(scale > 0.f) || !std::isfinite(scale))
+  if (max_len < 1 || max_len > QSA_MAX_CONTEXT || !valid_scale(scale))
     return QSA_ERR_INVALID_ARG;
   if ((int64_t)max_len > (int64_t)cache->max_pages * QSA_PAGE_SIZE) return QSA_ERR_INVALID_ARG;
   if ((blocks_out == nullptr) != (nblocks_out == nullptr)) return QSA_ERR_INVALID_ARG;
@@ -442,13 +444,138 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   return cuda_status(launch_gqa(p, B, positions_bound(QSA_OP_DECODE, max_len), num_sms(), L.splits_bound, st));
 }
 
+qsa_status qsa_index_project(const void* x, const void* w_proj, int32_t n, int32_t hidden, void* idx_q, void* idx_k,
+                             float* w, void* stream) {
+  if (n < 0 || hidden < QSA_HEAD_DIM || hidden > QSA_MAX_HIDDEN || hidden % QSA_HEAD_DIM != 0)
+    return QSA_ERR_INVALID_ARG;
+  if (n == 0) return QSA_OK;
+  if (!x || !w_proj || !idx_q || !idx_k || !w) return QSA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_proj, 16) || !aligned(idx_q, 2) || !aligned(idx_k, 2) || !aligned(w, 4))
+    return QSA_ERR_INVALID_ARG;
+  ProjParams p;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.w = static_cast<const __nv_bfloat16*>(w_proj);
+  p.n = n;
+  p.hidden = hidden;
+  p.idx_q = static_cast<__nv_bfloat16*>(idx_q);
+  p.idx_k = static_cast<__nv_bfloat16*>(idx_k);
+  p.wout = w;
+  return cuda_status(launch_index_proj(p, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_decode_indexer(const qsa_cache* cache, const void* x, const void* w_proj, int32_t hidden,
+                              const int32_t* seq_len, int32_t max_len, int32_t* blocks, int32_t* nblocks, void* ws,
+                              size_t ws_bytes, void* stream) {
+  qsa_status s = check_cache(cache);
+  if (s != QSA_OK) return s;
+  if (max_len < 1 || max_len > QSA_MAX_CONTEXT) return QSA_ERR_INVALID_ARG;
+  if ((int64_t)max_len > (int64_t)cache->max_pages * QSA_PAGE_SIZE) return QSA_ERR_INVALID_ARG;
+  if (hidden < QSA_HEAD_DIM || hidden > QSA_MAX_HIDDEN || hidden % QSA_HEAD_DIM != 0) return QSA_ERR_INVALID_ARG;
+  const int B = cache->batch;
+  if (B == 0) return QSA_OK;
+  if (!x || !w_proj || !seq_len || !blocks || !nblocks) return QSA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_proj, 16)) return QSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!layout(QSA_OP_DECODE_INDEXER, B, max_len, L)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProjParams pj;
+  pj.x = static_cast<const __nv_bfloat16*>(x);
+  pj.w = static_cast<const __nv_bfloat16*>(w_proj);
+  pj.n = B;
+  pj.hidden = hidden;
+  pj.idx_q = at<__nv_bfloat16>(ws, L.pj_q);
+  pj.idx_k = at<__nv_bfloat16>(ws, L.pj_k);
+  pj.wout = at<float>(ws, L.pj_w);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  {
+    ProfScope ps(st, 0);
+    cudaError_t e = launch_index_proj(pj, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  // the projected key, queries and weights feed the same front end and scorer as qsa_decode
+  return run_indexer(cache, view_of(cache), pj.idx_k, pj.idx_q, nullptr, seq_len, 0, B, max_len, pj.wout, blocks,
+                     nblocks, ws, L, st, nullptr, 1);
+}
+
+qsa_status qsa_decode_attend(const qsa_cache* cache, const void* q, const int32_t* seq_len, int32_t max_len,
+                             const int32_t* blocks, const int32_t* nblocks, float scale, void* out, float* lse,
+                             void* ws, size_t ws_bytes, void* stream) {
+  qsa_status s = check_kv_cache(cache);
+  if (s != QSA_OK) return s;
+  if (max_len < 1 || max_len > QSA_MAX_CONTEXT || !valid_scale(scale)) return QSA_ERR_INVALID_ARG;
+  if ((int64_t)max_len > (int64_t)cache->max_pages * QSA_PAGE_SIZE) return QSA_ERR_INVALID_ARG;
+  const int B = cache->batch;
+  if (B == 0) return QSA_OK;
+  if (!q || !seq_len || !blocks || !nblocks || !out) return QSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || (lse && !aligned(lse, 4))) return QSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!layout(QSA_OP_DECODE_ATTEND, B, max_len, L)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
+  GqaParams p{};
+  p.cluster_merge = 1;
+  p.c = view_of(cache);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.nq_row = 1;
+  p.mode = 0;
+  p.sel = blocks;
+  p.sel_n = nblocks;
+  p.row_len = seq_len;
+  p.len_offset = 0;
+  p.max_len = max_len;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.part_o = at<float>(ws, L.part_o);
+  p.part_ml = at<float>(ws, L.part_ml);
+  p.counters = at<int>(ws, L.cnt_gqa);
+  p.err = at<int>(ws, WS_ERR);
+  return cuda_status(launch_gqa(p, B, positions_bound(QSA_OP_DECODE, max_len), num_sms(), L.splits_bound,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_check_bounded_wait(const qsa_cache* cache, const void* q, void* out, uint64_t limit_ns, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  qsa_status s = check_cache(cache);
+  if (s != QSA_OK) return s;
+  if (cache->batch < 1 || !q || !out || limit_ns < 1 || limit_ns > WAIT_LIMIT_NS) return QSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return QSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!layout(QSA_OP_DECODE, 1, 8, L)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
+  // The decode attention of one row, launched exactly as qsa_decode launches it, but with no scorer
+  // before it: the row's ready flag (zeroed workspace) is never set.  Its length and selection are
+  // read from the zeroed workspace too, and only after the wait, which gives up first.
+  GqaParams p{};
+  p.cluster_merge = 1;
+  p.c = view_of(cache);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.nq_row = 1;
+  p.mode = 0;
+  p.sel = at<int32_t>(ws, L.sel);
+  p.sel_n = at<int32_t>(ws, L.sel_n);
+  p.row_len = at<int32_t>(ws, L.sel_n);
+  p.len_offset = 0;
+  p.max_len = 8;
+  p.scale_log2 = 1.f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.part_o = at<float>(ws, L.part_o);
+  p.part_ml = at<float>(ws, L.part_ml);
+  p.counters = at<int>(ws, L.cnt_gqa);
+  p.err = at<int>(ws, WS_ERR);
+  p.row_ready = at<int>(ws, L.ready);
+  p.wait_ns = limit_ns;
+  return cuda_status(launch_gqa(p, 1, positions_bound(QSA_OP_DECODE, 8), num_sms(), L.splits_bound,
+                                static_cast<cudaStream_t>(stream)));
+}
+
 qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_pos, const int32_t* frozen_n,
                                  int32_t frozen_stride, const int32_t* len0, int32_t n_plus_1, const void* q,
                                  float scale, void* out, void* ws, size_t ws_bytes, void* stream) {
   qsa_status s = check_cache(cache);
   if (s != QSA_OK) return s;
   if (n_plus_1 < 1 || n_plus_1 > QSA_MAX_DRAFT) return QSA_ERR_UNSUPPORTED;
-  if (frozen_stride < 0 || frozen_stride > QSA_MAX_SEL || !(scale > 0.f) || !std::isfinite(scale))
+  if (frozen_stride < 0 || frozen_stride > QSA_MAX_SEL || !valid_scale(scale))
     return QSA_ERR_INVALID_ARG;
   const int B = cache->batch;
   if (B == 0) return QSA_OK;

@@ -217,14 +217,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Every wait inside a kernel is bounded: it gives up after `limit_ns` of wall time (the host passes
+// WAIT_LIMIT_NS unless a diagnostic asks for a shorter limit), records QSA_DEVERR_TIMEOUT and returns
+// false; the caller then proceeds without the data and the kernel ends.
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
 // Cross-kernel readiness of one row (programmatic dependent launch): the producer publishes
-// after its block barrier (release, GPU scope); a consumer thread waits for it (acquire), giving up
-// after ~2 s of wall time with QSA_DEVERR_TIMEOUT.  Returns whether the row became ready.
+// after its block barrier (release, GPU scope); a consumer thread waits for it (acquire).
+// Returns whether the row became ready.
 __device__ __forceinline__ void publish_ready(int* flag) {
   asm volatile("fence.acq_rel.gpu;\n\tst.release.gpu.global.b32 [%0], 1;" ::"l"(flag) : "memory");
 }
 
-__device__ __forceinline__ bool wait_ready(const int* flag, int* err) {
+__device__ __forceinline__ bool wait_ready(const int* flag, int* err, uint64_t limit_ns) {
   uint64_t t0 = 0;
   for (int spin = 0;; ++spin) {
     int v;
@@ -232,10 +237,10 @@ __device__ __forceinline__ bool wait_ready(const int* flag, int* err) {
     if (v != 0) return true;
     if (spin == 0) {
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-    } else if ((spin & 63) == 0) {
+    } else if ((spin & 15) == 0) {
       uint64_t t;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      if (t - t0 > 2000000000ull) break;
+      if (t - t0 > limit_ns) break;
     }
     __nanosleep(256);  // few polls: many CTAs may wait at once
   }
@@ -246,14 +251,14 @@ __device__ __forceinline__ bool wait_ready(const int* flag, int* err) {
 // Row flags sit one per 128-byte line, so that waiting CTAs do not all poll the same L2 lines.
 constexpr int READY_STRIDE = 32;
 
-// Bounded wait: gives up after ~2 s of wall time, records QSA_DEVERR_TIMEOUT
-// and returns false (the caller then proceeds without the data).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// Bounded mbarrier wait (see WAIT_LIMIT_NS).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          uint64_t limit_ns = WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > 2000000000ull) break;
+    if (global_timer_ns() - t0 > limit_ns) break;
   }
   set_error(err, QSA_DEVERR_TIMEOUT);
   return false;

@@ -22,7 +22,6 @@
 // more splits than a cluster holds -- partials go through global memory and
 // the last CTA of the row, by atomic ticket, merges them.)
 #include <cooperative_groups.h>
-#include <cstdlib>
 
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
@@ -99,7 +98,8 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
       const int32_t* pt = p.c.page_table + (int64_t)req * p.c.max_pages;
       for (int i = tid * 32; i < npg; i += THREADS * 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(pt + i));
     }
-    if (tid == 0 && !wait_ready(p.row_ready + row * READY_STRIDE, p.err)) S.is_last = -1;
+    if (tid == 0 && !wait_ready(p.row_ready + row * READY_STRIDE, p.err, p.wait_ns ? p.wait_ns : WAIT_LIMIT_NS))
+      S.is_last = -1;
     else if (tid == 0) S.is_last = 0;
     __syncthreads();
     if (S.is_last < 0) bad = true;
@@ -510,19 +510,13 @@ static int occupancy(size_t smem) {
 // resident CTAs per SM x SMs), each split at least two tiles.
 template <int MT>
 static void choose_splits(int rows, int max_pos, int num_sms, int bound, int& splits, int& tps) {
-  static const int forced = [] {  // tuning override: QSA_GQA_CTAS_PER_SM=1..8 (resident CTAs to plan for)
-    const char* e = getenv("QSA_GQA_CTAS_PER_SM");
-    const int v = e ? atoi(e) : 0;
-    return (v >= 1 && v <= 8) ? v : 0;
-  }();
   const int tiles = ceil_div(max(max_pos, 1), GQ_TILE);
   rows = max(rows, 1);
   for (int occ_try = 8; occ_try >= 1; --occ_try) {
-    if (forced && occ_try != forced) continue;
     int s = (occ_try * num_sms) / rows;
     s = max(1, min(s, min(max(1, tiles / 2), min(bound, GQ_MAX_SPLITS))));
     const int t = ceil_div(tiles, s);
-    if (forced || occupancy<MT>(gqa_smem_bytes<MT>(t)) >= occ_try || occ_try == 1) {
+    if (occupancy<MT>(gqa_smem_bytes<MT>(t)) >= occ_try || occ_try == 1) {
       splits = s;
       tps = t;
       return;
@@ -568,19 +562,12 @@ static int active_clusters(int splits) {
 template <int MT>
 static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, int bound, cudaStream_t st) {
   static bool attr_set[64] = {false};
-  static const int carveout = [] {  // tuning override: QSA_GQA_CARVEOUT=0..100 (percent of shared memory)
-    const char* e = getenv("QSA_GQA_CARVEOUT");
-    const int v = e ? atoi(e) : -1;
-    return (v >= 0 && v <= 100) ? v : -1;
-  }();
   int dev = 0;
   cudaGetDevice(&dev);
   const size_t smem_max = gqa_smem_bytes<MT>(GQ_MAX_TILES);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e =
+    const cudaError_t e =
         cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
-    if (e == cudaSuccess && carveout >= 0)
-      e = cudaFuncSetAttribute(k_sparse_gqa<MT>, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }

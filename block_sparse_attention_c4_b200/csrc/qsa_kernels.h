@@ -6,6 +6,26 @@
 
 namespace qsa {
 
+// Host checks of the paged K/V part of a cache (what the sparse GQA reads), shared by every entry
+// point that attends: pointers, page size, pool size, strides and alignment.
+inline bool host_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline qsa_status check_kv_cache(const qsa_cache* c) {
+  if (!c) return QSA_ERR_INVALID_ARG;
+  if (!c->k || !c->v || !c->page_table) return QSA_ERR_INVALID_ARG;
+  if (c->page_size != QSA_PAGE_SIZE) return QSA_ERR_UNSUPPORTED;
+  if (c->num_slots <= 0 || c->num_slots % QSA_PAGE_SIZE != 0) return QSA_ERR_INVALID_ARG;
+  if (c->num_slots / QSA_PAGE_SIZE > (int64_t)INT32_MAX / QSA_PAGE_SIZE) return QSA_ERR_UNSUPPORTED;
+  if (c->max_pages <= 0 || c->batch < 0) return QSA_ERR_INVALID_ARG;
+  if (c->kv_stride != 0 && (c->kv_stride < HKV * D || c->kv_stride % 8 != 0)) return QSA_ERR_INVALID_ARG;
+  if (!host_aligned(c->k, 16) || !host_aligned(c->v, 16) || !host_aligned(c->page_table, 4))
+    return QSA_ERR_INVALID_ARG;
+  return QSA_OK;
+}
+
+// A softmax scale the kernels accept: positive and finite.
+inline bool valid_scale(float scale) { return scale > 0.f && scale <= 3.4e38f; }
+
 // ---- indexer front end (qsa_indexer.cu) ----
 cudaError_t launch_compress_append(const CacheView& c, const __nv_bfloat16* knew, const int32_t* cu_new,
                                    const int32_t* len_before, int total_new, int max_new, const RopeFreqs& fr,
@@ -101,6 +121,7 @@ struct GqaParams {
   int cluster_merge;          // 1: a row's splits may form one thread-block cluster and merge their partials
                               // through distributed shared memory (part_o, part_ml, counters unused);
                               // 0: partials go through global memory, the last split merges them
+  uint64_t wait_ns;           // limit of the row-flag wait (0: WAIT_LIMIT_NS)
 };
 constexpr int GQ_CLUSTER_MAX = 8;  // splits of one row in a cluster (portable cluster size)
 
@@ -124,7 +145,19 @@ struct PrefillParams {
   int* ovf_n;              // rows handed to the overflow selection (zeroed per call)
   int32_t* ovf_list;       // [T]
   int* err;
+  uint64_t wait_ns;        // limit of each mbarrier wait (0: WAIT_LIMIT_NS)
 };
+
+// ---- index projection (qsa_proj.cu) ----
+struct ProjParams {
+  const __nv_bfloat16* x;  // [n][hidden] hidden states
+  const __nv_bfloat16* w;  // [QSA_PROJ_FEATURES][hidden] projection weights
+  int n, hidden;           // hidden: a multiple of 128
+  __nv_bfloat16* idx_q;    // [n][4][128] out
+  __nv_bfloat16* idx_k;    // [n][128] out
+  float* wout;             // [n][4] out
+};
+cudaError_t launch_index_proj(const ProjParams& p, cudaStream_t st);
 
 // ev (nullable): n_ev event pairs recorded around the rotation, scoring and finalize kernels.
 cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,

@@ -64,27 +64,21 @@ int sm_count() {
   return n;
 }
 
-bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
 }  // namespace
 
 extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void* q, const int32_t* q_req,
                                              const int32_t* pos, const int32_t* npos, int32_t pos_stride,
                                              int32_t max_pos, int32_t nq, float scale, void* out, float* lse,
                                              void* stream) {
-  if (!cache || !cache->k || !cache->v || !cache->page_table) return QSA_ERR_INVALID_ARG;
-  if (cache->page_size != QSA_PAGE_SIZE) return QSA_ERR_UNSUPPORTED;
-  if (cache->num_slots <= 0 || cache->num_slots % QSA_PAGE_SIZE != 0 || cache->max_pages <= 0 || cache->batch < 0)
-    return QSA_ERR_INVALID_ARG;
-  if (!is_aligned(cache->k, 16) || !is_aligned(cache->v, 16) || !is_aligned(cache->page_table, 4))
-    return QSA_ERR_INVALID_ARG;
-  if (cache->kv_stride != 0 && (cache->kv_stride < 256 || cache->kv_stride % 8 != 0)) return QSA_ERR_INVALID_ARG;
-  if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !(scale > 0.f)) return QSA_ERR_INVALID_ARG;
+  // the same checks as qsa_sparse_gqa (the compressed index cache and ring are not read here)
+  const qsa_status cs = check_kv_cache(cache);
+  if (cs != QSA_OK) return cs;
+  if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !valid_scale(scale)) return QSA_ERR_INVALID_ARG;
   if (nq > QSA_NOALLOC_MAX_QUERIES) return QSA_ERR_UNSUPPORTED;  // beyond the array's stated capacity
   if (max_pos > QSA_MAX_SEL) return QSA_ERR_UNSUPPORTED;
   if (nq == 0) return QSA_OK;
   if (!q || !q_req || !pos || !npos || !out) return QSA_ERR_INVALID_ARG;
-  if (!is_aligned(q, 16) || !is_aligned(out, 16) || (lse && !is_aligned(lse, 4))) return QSA_ERR_INVALID_ARG;
+  if (!host_aligned(q, 16) || !host_aligned(out, 16) || (lse && !host_aligned(lse, 4))) return QSA_ERR_INVALID_ARG;
 
   uint8_t* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) return QSA_ERR_CUDA;
@@ -97,7 +91,7 @@ extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void*
   p.c.v = static_cast<const __nv_bfloat16*>(cache->v);
   p.c.page_table = cache->page_table;
   p.c.num_pages = cache->num_slots / QSA_PAGE_SIZE;
-  p.c.kv_stride = cache->kv_stride ? cache->kv_stride : 256;
+  p.c.kv_stride = cache->kv_stride ? cache->kv_stride : HKV * D;
   p.c.max_pages = cache->max_pages;
   p.c.batch = cache->batch;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -114,6 +108,7 @@ extern "C" qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void*
   p.part_ml = reinterpret_cast<float*>(base + OFF_ML);
   p.counters = reinterpret_cast<int*>(base + OFF_COUNTERS);
   const int cap = ROW_SPLITS / nq > 0 ? ROW_SPLITS / nq : 1;  // partials that fit the array
-  p.err = nullptr;  // no error word: positions outside their request are skipped silently
+  p.err = nullptr;  // no error word: positions outside the request's page-table row or the page pool are
+                    // skipped silently
   return launch_gqa(p, nq, max_pos, sm_count(), cap, st) == cudaSuccess ? QSA_OK : QSA_ERR_CUDA;
 }

@@ -65,7 +65,28 @@ struct __align__(1024) PfSmem {
   float4 w[2][PF_QT];                        // halved head weights of the work tile's queries (by tile parity)
   uint64_t full_a[PF_STAGES], empty_a[PF_STAGES], full_b, empty_b, tfull[2], tempty[2];
   uint32_t tmem_base;
+  int abort;  // set by the first role whose wait gives up: every role then stops issuing work
 };
+
+// Wait of one role: bounded, and it stops as soon as any role of the CTA has given up, so that one
+// barrier that never completes ends the whole CTA instead of costing a full limit per later wait.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* err, uint64_t limit_ns,
+                                        volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!*abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_timer_ns() - t0 > limit_ns) {
+      set_error(err, QSA_DEVERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+  return false;
+}
+
+// Phases armed (or committed) on stage s of a ring after `n` uses in round-robin order.
+__device__ __forceinline__ int ring_uses(int n, int s, int stages) { return n / stages + (s < n % stages ? 1 : 0); }
 
 // ---- tcgen05 / TMEM wrappers ----
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -147,8 +168,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   PfSmem& S = *reinterpret_cast<PfSmem*>(smem_aligned<1024>(smem_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   PfSched sch{ceil_div(p.T, PF_QT), (int)gridDim.x, p.pos0, p.T};
+  const uint64_t lim = p.wait_ns ? p.wait_ns : WAIT_LIMIT_NS;
+  volatile int* abort = &S.abort;
 
   if (tid == 0) {
+    S.abort = 0;
     for (int s = 0; s < PF_STAGES; ++s) {
       mbar_init(&S.full_a[s], 1);
       mbar_init(&S.empty_a[s], 1);
@@ -194,18 +218,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       return row;
     };
     int a_it = 0, wt = 0;
-    for (int j = 0;; ++j) {
+    bool ok = true;
+    for (int j = 0; ok; ++j) {
       const int qt = sch.nth(blockIdx.x, j);
       if (qt < 0) break;
       const int nm = sch.mtiles(qt);
       if (nm == 0) continue;
       const int nbv_hi = sch.nbv_of(min(p.T, (qt + 1) * PF_QT) - 1);
+      int go = 1;
       if (lane == 0) {
-        if (wt > 0) mbar_wait(&S.empty_b, (wt - 1) & 1, p.err);
-        mbar_arrive_expect_tx(&S.full_b, PF_B_BYTES);
-        tma_load_2d(S.b[0], &qmap, 0, qt * PF_N, &S.full_b);
-        tma_load_2d(S.b[1], &qmap, 64, qt * PF_N, &S.full_b);
+        go = wt == 0 || pf_wait(&S.empty_b, (wt - 1) & 1, p.err, lim, abort);
+        if (go) {
+          mbar_arrive_expect_tx(&S.full_b, PF_B_BYTES);
+          tma_load_2d(S.b[0], &qmap, 0, qt * PF_N, &S.full_b);
+          tma_load_2d(S.b[1], &qmap, 64, qt * PF_N, &S.full_b);
+        }
       }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
       ++wt;
       int rows_cur = page_row(lane, nbv_hi), rows_nxt = oob_row;
       for (int mt = 0; mt < nm; ++mt, ++a_it) {
@@ -213,10 +242,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         if (r == 0 && (g + 1) * GROUP < nm) rows_nxt = page_row((g + 1) * 32 + lane, nbv_hi);
         const int s = a_it % PF_STAGES;
         if (lane == 0) {
-          if (a_it >= PF_STAGES) mbar_wait(&S.empty_a[s], ((a_it / PF_STAGES) - 1) & 1, p.err);
-          mbar_arrive_expect_tx(&S.full_a[s], PF_A_BYTES);
+          go = a_it < PF_STAGES || pf_wait(&S.empty_a[s], ((a_it / PF_STAGES) - 1) & 1, p.err, lim, abort);
+          if (go) mbar_arrive_expect_tx(&S.full_a[s], PF_A_BYTES);
         }
-        __syncwarp();  // the stage is free (and its bytes expected) before any lane copies into it
+        // the stage is free (and its bytes expected) before any lane copies into it
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
         // 16 lanes issue the M-tile's 16 copies at once: lane 2*pg + half copies the 64-dim half
         // `half` of page pg (16 keys)
         constexpr int PAGES = PF_M / PAGE_BLOCKS;  // 8 pages per M-tile
@@ -227,23 +260,36 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         if (r == GROUP - 1) rows_cur = rows_nxt;
       }
     }
+    // drain: every copy issued above has landed before the CTA may exit (in the normal case these
+    // phases completed long ago and the waits return at once)
+    if (lane == 0) {
+      if (wt > 0) mbar_wait(&S.full_b, (wt - 1) & 1, p.err, lim);
+      for (int s = 0; s < PF_STAGES; ++s) {
+        const int uses = ring_uses(a_it, s, PF_STAGES);
+        if (uses > 0) mbar_wait(&S.full_a[s], (uses - 1) & 1, p.err, lim);
+      }
+    }
   } else if (warp == 1) {
     // =============================== MMA issuer ===============================
     if (lane == 0) {
       const uint32_t idesc = pf_idesc();
-      int a_it = 0, m_it = 0, wt = 0;
-      for (int j = 0;; ++j) {
+      int a_it = 0, m_it = 0, wt = 0, b_commits = 0;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
         const int qt = sch.nth(blockIdx.x, j);
         if (qt < 0) break;
         const int nm = sch.mtiles(qt);
         if (nm == 0) continue;
-        mbar_wait(&S.full_b, wt & 1, p.err);
+        if (!pf_wait(&S.full_b, wt & 1, p.err, lim, abort)) break;
         ++wt;
         for (int mt = 0; mt < nm; ++mt, ++a_it, ++m_it) {
           const int s = a_it % PF_STAGES;
           const int buf = m_it & 1;
-          mbar_wait(&S.full_a[s], (a_it / PF_STAGES) & 1, p.err);
-          if (m_it >= 2) mbar_wait(&S.tempty[buf], ((m_it >> 1) - 1) & 1, p.err);
+          if (!pf_wait(&S.full_a[s], (a_it / PF_STAGES) & 1, p.err, lim, abort) ||
+              (m_it >= 2 && !pf_wait(&S.tempty[buf], ((m_it >> 1) - 1) & 1, p.err, lim, abort))) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(buf * PF_N);
 #pragma unroll
@@ -257,12 +303,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           tc_commit(&S.tfull[buf]);
         }
         tc_commit(&S.empty_b);
+        ++b_commits;
       }
-      // tail: every commit issued above must have arrived before the CTA may exit
-      if (wt > 0) mbar_wait(&S.empty_b, (wt - 1) & 1, p.err);
+      // tail: every commit issued above has arrived (its MMAs are done) before the CTA may exit
+      if (b_commits > 0) mbar_wait(&S.empty_b, (b_commits - 1) & 1, p.err, lim);
       for (int s = 0; s < PF_STAGES; ++s) {
-        const int uses = a_it / PF_STAGES + (s < a_it % PF_STAGES ? 1 : 0);
-        if (uses > 0) mbar_wait(&S.empty_a[s], (uses - 1) & 1, p.err);
+        const int uses = ring_uses(a_it, s, PF_STAGES);
+        if (uses > 0) mbar_wait(&S.empty_a[s], (uses - 1) & 1, p.err, lim);
       }
     }
   } else {
@@ -296,7 +343,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
       for (int mt = 0; mt < nm; ++mt, ++m_it) {
         const int buf = m_it & 1;
-        mbar_wait(&S.tfull[buf], (m_it >> 1) & 1, p.err);
+        // after a timeout anywhere in the CTA the loops still run to their end (no work, no waits), so
+        // that every epilogue warp meets the same named barriers
+        if (!pf_wait(&S.tfull[buf], (m_it >> 1) & 1, p.err, lim, abort)) continue;
         tc_fence_after();
         uint32_t r[PF_QPW / 8][32];
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * PF_N + qg * PF_QPW * 4);

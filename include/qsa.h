@@ -55,6 +55,9 @@ extern "C" {
 #define QSA_PAGE_SIZE 64    /* tokens per K/V page (16 compressed entries)        */
 #define QSA_MAX_DRAFT 8     /* largest n_plus_1 of qsa_decode_indexshare          */
 #define QSA_MAX_CONTEXT (1 << 20) /* largest context length accepted (1,048,576)    */
+/* Outputs of the index projection per token: 4 x 128 query dims, 128 key dims, 4 head weights. */
+#define QSA_PROJ_FEATURES (QSA_INDEX_HEADS * QSA_HEAD_DIM + QSA_HEAD_DIM + QSA_INDEX_HEADS) /* 644 */
+#define QSA_MAX_HIDDEN 32768 /* largest hidden size of the index projection (a multiple of 128) */
 
 typedef enum {
   QSA_OK = 0,
@@ -82,7 +85,7 @@ typedef enum {
  *   ring        bf16 [batch][4][128]      raw index keys of each request's
  *               unfinished block, slot = position mod 4
  *   page_table  int32 [batch][max_pages]  physical page of each logical page
-  *   num_slots   multiple of page_size; page_size must be 64
+ *   num_slots   multiple of page_size; page_size must be 64
  *   kv_stride   bf16 elements from one slot to the next in k (and in v): 0 means
  *               256, i.e. separate [num_slots][2][128] arrays; 512 with
  *               v = k + 256 interleaves each slot's K and V rows, so that the
@@ -113,7 +116,9 @@ typedef enum {
   QSA_OP_DECODE = 3,
   QSA_OP_DECODE_INDEXSHARE = 4,
   QSA_OP_COMPRESS_APPEND = 5,
-  QSA_OP_PREFILL_SCORE_TOPK = 6
+  QSA_OP_PREFILL_SCORE_TOPK = 6,
+  QSA_OP_DECODE_INDEXER = 7, /* qsa_decode_indexer: rows = batch, max_len = longest context */
+  QSA_OP_DECODE_ATTEND = 8   /* qsa_decode_attend:  rows = batch, max_len = longest context */
 } qsa_op;
 
 /*
@@ -263,6 +268,55 @@ qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_p
                                  float scale, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Index projection: hidden states -> index queries, index keys, head weights.
+ * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely":
+ * the indexer has 4 query heads of 128 dims and one shared 128-dim key per
+ * token.  The pages give no hidden size and do not say how the head weights
+ * are formed; this library reads them as one bias-free linear map:
+ *   [idx_q (4 x 128) | idx_k (128) | w (4)] = W_proj x
+ * accumulated in FP32; idx_q and idx_k rounded once to bf16, w kept FP32.
+ *   x       bf16 [n][hidden]                       hidden states (16-byte aligned rows)
+ *   w_proj  bf16 [QSA_PROJ_FEATURES][hidden]       rows 0..511: query head h dim d at 128h + d;
+ *                                                   rows 512..639: key dims; rows 640..643: head weights
+ *   hidden  multiple of 128, at most QSA_MAX_HIDDEN
+ *   idx_q   bf16 [n][4][128] out; idx_k bf16 [n][128] out; w f32 [n][4] out
+ */
+qsa_status qsa_index_project(const void* x, const void* w_proj, int32_t n, int32_t hidden, void* idx_q, void* idx_k,
+                             float* w, void* stream);
+
+/*
+ * The decode step in two phases, so that the indexer can run on a second CUDA
+ * stream while the caller computes the layer's main Q/K/V projection (blog
+ * section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely": the
+ * indexer can overlap the main Q/K/V projection on a second stream).
+ *
+ * qsa_decode_indexer needs only the new tokens' hidden states: it projects
+ * them (qsa_index_project), appends each request's new index key (ring, and
+ * the compressed key when it completes a block), rotates the index queries,
+ * scores the complete blocks and keeps the top 512.
+ *   x        bf16 [batch][hidden] hidden state of each request's new token
+ *   w_proj   bf16 [QSA_PROJ_FEATURES][hidden] (see qsa_index_project)
+ *   seq_len  int32 [batch] context length including the new token (device)
+ *   max_len  host bound of seq_len
+ *   blocks   int32 [batch][512] out, ascending; nblocks int32 [batch] out
+ *   ws       workspace of qsa_workspace_bytes(QSA_OP_DECODE_INDEXER, batch, max_len)
+ * qsa_decode_attend then runs the sparse GQA over the kept blocks plus each
+ * request's tail; it needs the attention queries and the new token's K/V in
+ * the pool (the caller's main projection), and the indexer's blocks/nblocks
+ * (order the streams with an event).
+ *   q        bf16 [batch][16][128]; out bf16 [batch][16][128]; lse f32 [batch][16] or NULL
+ *   ws       workspace of qsa_workspace_bytes(QSA_OP_DECODE_ATTEND, batch, max_len)
+ *            (its own: the two phases of consecutive steps may run at once)
+ * Together they compute what qsa_decode computes from the projected inputs.
+ */
+qsa_status qsa_decode_indexer(const qsa_cache* cache, const void* x, const void* w_proj, int32_t hidden,
+                              const int32_t* seq_len, int32_t max_len, int32_t* blocks, int32_t* nblocks, void* ws,
+                              size_t ws_bytes, void* stream);
+qsa_status qsa_decode_attend(const qsa_cache* cache, const void* q, const int32_t* seq_len, int32_t max_len,
+                             const int32_t* blocks, const int32_t* nblocks, float scale, void* out, float* lse,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Sparse GQA without a workspace: the same computation as qsa_sparse_gqa
  * (same arguments minus ws / ws_bytes), for callers that cannot allocate
  * device memory or pass the library scratch space -- e.g. a plugin whose host
@@ -284,7 +338,9 @@ qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_p
  *   All calls share the one array, which keeps the last call's contents: calls
  *   that overlap on the GPU (different streams, no ordering) race and give
  *   wrong results.  Device-side data errors are not reported (there is no
- *   error word): positions outside their request are skipped.
+ *   error word): a position whose page lies outside the request's page-table row, or whose
+ *   page id lies outside the pool, is skipped (a position past the request's length on a
+ *   page it owns is read like any other).
  */
 #define QSA_NOALLOC_MAX_QUERIES 4096
 #define QSA_NOALLOC_ROW_SPLITS 512
@@ -294,6 +350,25 @@ qsa_status qsa_decode_indexshare(const qsa_cache* cache, const int32_t* frozen_p
 qsa_status qsa_sparse_gqa_noalloc(const qsa_cache* cache, const void* q, const int32_t* q_req, const int32_t* pos,
                                   const int32_t* npos, int32_t pos_stride, int32_t max_pos, int32_t nq, float scale,
                                   void* out, float* lse, void* stream);
+
+/*
+ * Failure detection without a GPU fault: a check that the kernels' bounded
+ * waits end.  Every wait inside a kernel of this library (the decode attention
+ * waiting for its request's selection, the prefill scorer's pipeline barriers)
+ * gives up after a limit (2 s), records QSA_DEVERR_TIMEOUT and lets the kernel
+ * finish, so no wait can hang the GPU.  This call launches the decode attention
+ * kernel for request 0 of `cache` with a selection that nothing publishes and a
+ * limit of `limit_ns` nanoseconds: the kernel waits, gives up, sets
+ * QSA_DEVERR_TIMEOUT in the workspace's error word and writes zeros to `out`.
+ * The CUDA context stays usable; read the outcome with qsa_device_error.
+ * Not a step of the method (the QSA description has no counterpart).
+ *   q         bf16 [16][128] a query (device; read, its values do not matter)
+ *   out       bf16 [16][128] out (zeros)
+ *   limit_ns  1 .. 2e9
+ *   ws        workspace of qsa_workspace_bytes(QSA_OP_DECODE, 1, 8), zeroed
+ */
+qsa_status qsa_check_bounded_wait(const qsa_cache* cache, const void* q, void* out, uint64_t limit_ns, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * Read (and optionally clear) the device error word of a workspace.  This

@@ -65,9 +65,10 @@ def lib():
                                           ctypes.c_int]
         L.oracle_prefill_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, f64, f64, vp, vp, vp, vp, ctypes.c_int]
         L.oracle_indexshare.argtypes = [vp, i32, i64, i32, vp, vp, vp, f64, vp]
+        L.oracle_index_project.argtypes = [vp, vp, i64, i64, vp, vp, vp, ctypes.c_int]
         for name in ("oracle_rope_f64", "oracle_compress_block", "oracle_compress", "oracle_append",
                      "oracle_rotate_query", "oracle_block_scores", "oracle_sparse_gqa", "oracle_decode_batch",
-                     "oracle_prefill_rows", "oracle_indexshare"):
+                     "oracle_prefill_rows", "oracle_indexshare", "oracle_index_project"):
             getattr(L, name).restype = None
         _lib = L
     return _lib
@@ -233,6 +234,23 @@ def prefill_rows(rows, idx_q, w, q, comp, K, V, theta: float = 1e7, scale: float
                               _p(out) if out is not None else None, _p(blocks), _p(nblocks), _p(npos),
                               nthreads or threads())
     return (out[:n] if out is not None else None), [blocks[i, :nblocks[i]].copy() for i in range(n)]
+
+
+PROJ_FEATURES = HI * D + D + HI  # 644
+
+
+def index_project(x: np.ndarray, W: np.ndarray, nthreads: int | None = None):
+    """x [n, hidden] and W [644, hidden] bf16 bits -> (idx_q [n,4,128] bits, idx_k [n,128] bits, w [n,4] f32)."""
+    x = _u16(x)
+    W = _u16(W)
+    n, hidden = x.shape
+    assert W.shape == (PROJ_FEATURES, hidden)
+    idx_q = np.empty((n, HI, D), dtype=np.uint16)
+    idx_k = np.empty((n, D), dtype=np.uint16)
+    w = np.empty((n, HI), dtype=np.float32)
+    if n:
+        lib().oracle_index_project(_p(x), _p(W), n, hidden, _p(idx_q), _p(idx_k), _p(w), nthreads or threads())
+    return idx_q, idx_k, w
 
 
 def indexshare(frozen_pos: np.ndarray, L0: int, n_plus_1: int, q: np.ndarray, K: np.ndarray, V: np.ndarray,

@@ -300,6 +300,32 @@ void oracle_prefill_rows(const int64_t* rows, int64_t nrows, const uint16_t* idx
   });
 }
 
+// Index projection of n tokens (reading: the indexer's query heads, key and head weights are one
+// bias-free linear map of the token's hidden state; the pages give neither the map nor the hidden
+// size).  For token i and feature f: y = sum_j W[f][j] * x[i][j] in FP64.  Features 0..511 are the
+// 4 index query heads (head h, dim d at 128h + d) and 512..639 the index key, each rounded once to
+// bf16; 640..643 are the 4 head weights, rounded once to float.
+// x: [n][hidden] bf16; W: [644][hidden] bf16; idx_q: [n][4][128]; idx_k: [n][128]; w: [n][4].
+void oracle_index_project(const uint16_t* x, const uint16_t* W, int64_t n, int64_t hidden, uint16_t* idx_q,
+                          uint16_t* idx_k, float* w, int nthreads) {
+  constexpr int F = HI * D + D + HI;
+  parallel(n, nthreads, [&](int64_t i) {
+    const uint16_t* xi = x + i * hidden;
+    for (int f = 0; f < F; ++f) {
+      const uint16_t* wf = W + static_cast<int64_t>(f) * hidden;
+      double y = 0.0;
+      for (int64_t j = 0; j < hidden; ++j) y += bf16_to_f64(wf[j]) * bf16_to_f64(xi[j]);
+      if (f < HI * D) {
+        idx_q[i * HI * D + f] = f64_to_bf16(y);
+      } else if (f < HI * D + D) {
+        idx_k[i * D + (f - HI * D)] = f64_to_bf16(y);
+      } else {
+        w[i * HI + (f - HI * D - D)] = static_cast<float>(y);
+      }
+    }
+  });
+}
+
 // IndexShare draft step of one request: draft query i (i = 0..n_plus_1-1) at
 // position L0+i attends to the frozen positions (selected at position L0-1)
 // plus positions L0..L0+i.  q: [n_plus_1][16][128]; out: [n_plus_1][16][128].

@@ -32,6 +32,7 @@ PAGE = 64
 
 # stream kinds
 K_IDXQ, K_W, K_IDXK, K_BIAS, K_Q, K_K, K_V, K_PAGES, K_LENS = 1, 2, 3, 4, 5, 6, 7, 8, 9
+K_HIDDEN, K_WPROJ = 10, 11
 
 
 def _threads() -> int:
@@ -56,6 +57,8 @@ def lib():
         u64, i64, i32, f32, f64 = ctypes.c_uint64, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double
         vp = ctypes.c_void_p
         L.qsa_gen_normal_bf16.argtypes = [u64, u64, u64, i64, vp, i32]
+        L.qsa_gen_normal_scaled_bf16.argtypes = [u64, u64, u64, i64, f64, vp, i32]
+        L.qsa_gen_normal_scaled_bf16.restype = None
         L.qsa_gen_uniform_f32.argtypes = [u64, u64, u64, i64, f32, f32, vp]
         L.qsa_gen_uniform_i64.argtypes = [u64, u64, u64, i64, i64, i64, vp]
         L.qsa_gen_bernoulli_u8.argtypes = [u64, u64, u64, i64, f64, vp]
@@ -83,6 +86,13 @@ def normal_bf16(seed: int, strm: int, shape, offset: int = 0) -> np.ndarray:
     """N(0,1) values rounded once to bf16; returned as raw uint16 bits."""
     out = np.empty(shape, dtype=np.uint16)
     lib().qsa_gen_normal_bf16(seed, strm, offset, out.size, _ptr(out), _threads())
+    return out
+
+
+def normal_scaled_bf16(seed: int, strm: int, shape, std: float, offset: int = 0) -> np.ndarray:
+    """N(0, std^2) values rounded once to bf16; raw uint16 bits."""
+    out = np.empty(shape, dtype=np.uint16)
+    lib().qsa_gen_normal_scaled_bf16(seed, strm, offset, out.size, float(std), _ptr(out), _threads())
     return out
 
 
@@ -179,6 +189,12 @@ class Workload:
             n = self.n_queries(r) if self.kind != "indexshare" else self.n_draft + 1
         return normal_bf16(self.seed, stream(K_Q, r), (n, Q_HEADS, HEAD_DIM), offset=q0 * Q_HEADS * HEAD_DIM)
 
+    def hidden(self, r: int, hidden: int, q0: int = 0, n: int | None = None) -> np.ndarray:
+        """Hidden states [n, hidden] of request r's query tokens (bf16 bits, N(0,1)), the input of the
+        index projection."""
+        n = self.n_queries(r) if n is None else n
+        return normal_bf16(self.seed, stream(K_HIDDEN, r), (n, hidden), offset=q0 * hidden)
+
     def bias_direction(self, r: int) -> np.ndarray:
         nq = self.n_queries(r)
         return self.idx_q(r, q0=nq - 1, n=1)[0, 0]
@@ -220,6 +236,15 @@ class Workload:
                 off += n
             self._cache["pt"] = pt
         return self._cache["pt"]
+
+
+PROJ_FEATURES = INDEX_HEADS * HEAD_DIM + HEAD_DIM + INDEX_HEADS  # 644
+
+
+def projection_weights(seed: int, hidden: int) -> np.ndarray:
+    """Index projection weights [644, hidden] ~ N(0, 1/hidden) (bf16 bits): rows 0..511 the 4 query
+    heads, 512..639 the key, 640..643 the head weights."""
+    return normal_scaled_bf16(seed, stream(K_WPROJ), (PROJ_FEATURES, hidden), hidden ** -0.5)
 
 
 def _lens_uniform(seed: int, n: int, lo: int, hi: int) -> np.ndarray:

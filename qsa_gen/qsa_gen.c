@@ -125,17 +125,25 @@ static void parallel_for(int64_t n, int nthreads, range_fn fn, void* ctx) {
  * ------------------------------------------------------------------------- */
 typedef struct {
   uint64_t key, offset;
+  double std;
   uint16_t* out;
 } normal_ctx;
 
 static void normal_range(void* p, int64_t lo, int64_t hi) {
   normal_ctx* c = (normal_ctx*)p;
-  for (int64_t i = lo; i < hi; ++i) c->out[i] = bf16_rne(normal_at(c->key, c->offset + (uint64_t)i));
+  for (int64_t i = lo; i < hi; ++i) c->out[i] = bf16_rne(c->std * normal_at(c->key, c->offset + (uint64_t)i));
 }
 
 void qsa_gen_normal_bf16(uint64_t seed, uint64_t stream, uint64_t offset, int64_t n, uint16_t* out,
                          int nthreads) {
-  normal_ctx c = {stream_key(seed, stream), offset, out};
+  normal_ctx c = {stream_key(seed, stream), offset, 1.0, out};
+  parallel_for(n, nthreads, normal_range, &c);
+}
+
+/* N(0, std^2): the same deviates times std (in FP64), rounded once to bf16. */
+void qsa_gen_normal_scaled_bf16(uint64_t seed, uint64_t stream, uint64_t offset, int64_t n, double std,
+                                uint16_t* out, int nthreads) {
+  normal_ctx c = {stream_key(seed, stream), offset, std, out};
   parallel_for(n, nthreads, normal_range, &c);
 }
 

@@ -118,6 +118,20 @@ def test_invalid_arguments_are_rejected_before_launch(qsa):
     assert L.qsa_expand_indices(p, p, p, 0, p, p, None) == 0
     assert L.qsa_compress_append(ctypes.byref(c), p, p, p, -1, 0, None) == INVALID
     assert L.qsa_compress_append(ctypes.byref(c), p, p, p, 0, 0, None) == 0
+    # a non-finite or non-positive scale is rejected by both sparse-GQA entry points alike
+    for sc in (float("inf"), float("nan"), 0.0, -1.0):
+        assert L.qsa_sparse_gqa(ctypes.byref(c), p, p, p, p, 100, 100, 4, sc, p, None, ws, big, None) == INVALID
+        assert L.qsa_sparse_gqa_noalloc(ctypes.byref(c), p, p, p, p, 100, 100, 4, sc, p, None, None) == INVALID
+        assert L.qsa_decode(ctypes.byref(c), p, p, p, p, p, 100, sc, p, None, None, None, ws, big, None) == INVALID
+    # a pool too large for 32-bit page ids, rejected by both
+    huge = fake_cache(qsa, num_slots=64 * (1 << 31))
+    assert L.qsa_sparse_gqa(ctypes.byref(huge), p, p, p, p, 100, 100, 4, 0.1, p, None, ws, big, None) == UNSUPPORTED
+    assert L.qsa_sparse_gqa_noalloc(ctypes.byref(huge), p, p, p, p, 100, 100, 4, 0.1, p, None, None) == UNSUPPORTED
+    # bounded-wait check: limit in 1 ns .. 2 s, outputs present
+    assert L.qsa_check_bounded_wait(ctypes.byref(c), p, p, 0, ws, big, None) == INVALID
+    assert L.qsa_check_bounded_wait(ctypes.byref(c), p, p, 2_000_000_001, ws, big, None) == INVALID
+    assert L.qsa_check_bounded_wait(ctypes.byref(c), p, None, 1000, ws, big, None) == INVALID
+    assert L.qsa_check_bounded_wait(ctypes.byref(c), p, p, 1000, ws, 16, None) == WORKSPACE
     # workspace init rejects misaligned memory
     assert L.qsa_workspace_init(ctypes.c_void_p(0x100010), 1024, None) == WORKSPACE
 

@@ -167,3 +167,85 @@ def test_long_context_262k(Q, W):
     entries = (pt[(4 * b) // 64].astype(np.int64) * 64 + (4 * b) % 64) // 4
     got = cache.cidx[torch.from_numpy(entries).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
     np.testing.assert_array_equal(got, O.compress(raw))
+
+
+# ---------------------------------------------------------------------------------------------
+# The tensor-core prefill scorer at full size, chained into expansion and sparse GQA
+# ---------------------------------------------------------------------------------------------
+
+def _prefill_chain(Q, W, wl, cache, pos0, T, check_rows, L_keys, comp=None):
+    """qsa_prefill_score_topk over the causal chunk pos0 .. pos0+T-1 of request 0, then
+    qsa_expand_indices and qsa_sparse_gqa over every query of the chunk.  Every row is validated;
+    the rows in `check_rows` (positions) are checked against the oracle: kept blocks under the
+    near-tie rule, attention against the oracle run on the GPU's own selection."""
+    dev = "cuda"
+    idx_q = W.bits_to_bf16(wl.idx_q(0, q0=pos0, n=T), dev)
+    w = torch.from_numpy(wl.w(0, q0=pos0, n=T)).to(dev)
+    q = W.bits_to_bf16(wl.q(0, q0=pos0, n=T), dev)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, pos0 + T))
+    blocks, nblocks = Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws)
+    q_pos = torch.arange(pos0, pos0 + T, dtype=torch.int32, device=dev)
+    pos, npos = Q.expand_indices(blocks, nblocks, q_pos)
+    ws2 = Q.Workspace(Q.workspace_bytes(Q.OP_SPARSE_GQA, T, 2051))
+    out = Q.sparse_gqa(cache, q, torch.zeros(T, dtype=torch.int32, device=dev), pos, npos, 2051, ws2)
+    torch.cuda.synchronize()
+    assert ws.device_error() == 0 and ws2.device_error() == 0
+    del ws, ws2
+    bl, nbl = blocks.cpu().numpy(), nblocks.cpu().numpy()
+    t_all = np.arange(pos0, pos0 + T)
+    _valid_rows(bl, nbl, [(int(t) + 1) // 4 for t in t_all])
+    pp, npp = pos.cpu().numpy(), npos.cpu().numpy()
+    assert np.all(npp == 4 * nbl + (t_all + 1) % 4)
+    o = bf16_tensor_to_f32(out)
+    assert np.all(np.isfinite(o))
+    if comp is None:
+        comp = O.compress(wl.idx_keys(0, 0, L_keys))
+    K, V = wl.k(0, 0, L_keys), wl.v(0, 0, L_keys)
+    for t in sorted(check_rows):
+        i = t - pos0
+        idx_q_t, w_t = wl.idx_q(0, q0=t, n=1)[0], wl.w(0, q0=t, n=1)[0]
+        ob, opos, s = O.select_query(idx_q_t, w_t, comp, t + 1)
+        sel = check_selection(bl[i, :nbl[i]], ob, s, (t + 1) // 4, what=f"tensor-core prefill row {t}")
+        gpos = O.expand(sel.astype(np.int32), t + 1)
+        np.testing.assert_array_equal(pp[i, :npp[i]], gpos)
+        ref, _ = O.sparse_gqa(wl.q(0, q0=t, n=1)[0], K, V, gpos)
+        check_attention(o[i], ref, what=f"tensor-core prefill row {t}")
+    return bl, nbl
+
+
+def test_prefill_32k_tensor_core_chain(Q, W):
+    """Config 1 end to end on the tensor-core path: 32768 queries scored by qsa_prefill_score_topk,
+    expanded, attended; every row validated, edge and seeded rows against the oracle."""
+    wl = G.prefill_32k()
+    cache = W.build_cache(wl, prefix_tokens=[32768])
+    rng = np.random.default_rng(21)
+    rows = {0, 1, 3, 4, 2047, 2050, 2051, 2052, 4095, 8191, 16384, 32766, 32767}
+    rows |= set(rng.integers(0, 32768, 40).tolist())
+    _prefill_chain(Q, W, wl, cache, 0, 32768, rows, 32768)
+
+
+@pytest.fixture(scope="module")
+def long_cache(Q, W):
+    """The 262144-token context of config 4 with every index key appended in causal chunks of 8192."""
+    wl = G.long_262k()
+    cache = W.build_cache(wl, prefix_tokens=[0])
+    for t0 in range(0, 262144, 8192):
+        W.append_tokens(cache, wl, 0, t0, 8192)
+    torch.cuda.synchronize()
+    comp = O.compress(wl.idx_keys(0, 0, 262144))
+    return wl, cache, comp
+
+
+@pytest.mark.parametrize("pos0", [0, 131072, 253952])
+def test_long_context_prefill_chunk_tensor_core(Q, W, long_cache, pos0):
+    """Config 4's prefill: a causal chunk of 8192 queries at pos0 (up to 65,536 visible blocks per
+    query) through the tensor-core scorer, chained into expansion and sparse GQA; every row
+    validated, the chunk's first and last rows and seeded rows against the oracle."""
+    wl, cache, comp = long_cache
+    T = 8192
+    rng = np.random.default_rng(pos0 + 7)
+    rows = {pos0, pos0 + 1, pos0 + T // 2, pos0 + T - 2, pos0 + T - 1}
+    rows |= set((pos0 + rng.integers(0, T, 20)).tolist())
+    if pos0 == 0:
+        rows |= {2047, 2050, 2051, 2052, 4095}
+    _prefill_chain(Q, W, wl, cache, pos0, T, rows, pos0 + T, comp=comp[:(pos0 + T) // 4])

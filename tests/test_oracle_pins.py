@@ -315,6 +315,52 @@ def test_short_context_layer_is_dense_causal_gqa(oracle_lib, L):
     np.testing.assert_array_equal(comp[:L // 4], O.compress(raw)[:L // 4])
 
 
+def test_prefill_rows_short_context_is_dense_causal_attention(oracle_lib):
+    """Prefill rows of one sequence: row t (position t, context t + 1) with at most 512 complete blocks
+    attends to every position 0..t, i.e. textbook causal attention.  Reference: torch SDPA in FP64
+    over the whole sequence with the causal mask j <= t, per KV group.  A context off by one (t or
+    t + 2 tokens) or a row read at the wrong position fails it."""
+    T = 2051
+    wl = G.prefill_32k(seed=13, L=T)
+    idx_q, w, q = wl.idx_q(0, 0, T), wl.w(0, 0, T), wl.q(0, 0, T)
+    K, V = wl.k(0, 0, T), wl.v(0, 0, T)
+    comp = O.compress(wl.idx_keys(0, 0, T))
+    rows = np.array([0, 1, 2, 3, 4, 5, 130, 1023, 2047, 2048, 2049, 2050], dtype=np.int64)
+    out, blocks = O.prefill_rows(rows, idx_q, w, q, comp, K, V, nthreads=4)
+    qt = torch.from_numpy(f32(q[rows]).astype(np.float64)).permute(1, 0, 2).unsqueeze(0)  # [1,16,n,128]
+    kt = torch.from_numpy(f32(K).astype(np.float64)).permute(1, 0, 2).unsqueeze(0)         # [1,2,T,128]
+    vt = torch.from_numpy(f32(V).astype(np.float64)).permute(1, 0, 2).unsqueeze(0)
+    mask = torch.from_numpy(np.arange(T)[None, :] <= rows[:, None])                      # [n, T]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, enable_gqa=True)
+    ref = ref[0].permute(1, 0, 2).numpy()                                                # [n,16,128]
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+    for i, t in enumerate(rows):
+        np.testing.assert_array_equal(blocks[i], np.arange((t + 1) // 4))
+
+
+def test_prefill_rows_long_context_rows_follow_the_selection(oracle_lib):
+    """Rows with more than 512 complete blocks: each row's kept blocks are the exact top-512 of
+    brute-force scores at context t + 1 (numpy matmul, lexsort), and its output is torch SDPA over
+    those blocks' positions plus the row's own unfinished block."""
+    T = 2600
+    wl = G.prefill_32k(seed=14, L=T)
+    idx_q, w, q = wl.idx_q(0, 0, T), wl.w(0, 0, T), wl.q(0, 0, T)
+    K, V = wl.k(0, 0, T), wl.v(0, 0, T)
+    comp = O.compress(wl.idx_keys(0, 0, T))
+    rows = np.array([2051, 2052, 2310, 2599], dtype=np.int64)
+    out, blocks = O.prefill_rows(rows, idx_q, w, q, comp, K, V, nthreads=4)
+    for i, t in enumerate(rows):
+        L = int(t) + 1
+        qrot = f32(O.rotate_query(idx_q[t], L - 1)).astype(np.float64)  # rotation: pinned above
+        dots = f32(comp[:L // 4]).astype(np.float64) @ qrot.T
+        s = (np.maximum(dots, 0) * w[t].astype(np.float64)).sum(axis=1)
+        ref_blocks = np.sort(np.lexsort((np.arange(len(s)), -s))[:512])
+        np.testing.assert_array_equal(blocks[i], ref_blocks)
+        pos = np.concatenate([(4 * ref_blocks[:, None] + np.arange(4)).ravel(), np.arange(4 * (L // 4), L)])
+        ro, _ = _sdpa_ref(q[t], K, V, pos.astype(np.int32))
+        np.testing.assert_allclose(out[i], ro, rtol=1e-10, atol=1e-12)
+
+
 def test_long_context_selection_is_exact_topk_of_brute_force_scores(oracle_lib):
     wl = G.custom_decode(10, [6002])
     L = 6002
@@ -372,3 +418,28 @@ def test_indexshare_short_context_equals_normal_path(oracle_lib):
         _, pos_i, _ = O.select_query(wl.idx_q(0)[0], wl.w(0)[0], comp, L0 + i + 1)
         ro, _ = O.sparse_gqa(q[i], K, V, pos_i)
         np.testing.assert_array_equal(out[i], ro)
+
+
+# --- index projection ---------------------------------------------------------------------------
+
+def test_index_project_is_rounded_linear_map(oracle_lib):
+    """Against a numpy float64 matmul of the decoded values: query heads are features 0..511 (head h,
+    dim d at 128h + d), the key 512..639, the head weights 640..643; each bf16 output is the nearest
+    bf16 of the exact product (within half an ulp), each weight its float rounding."""
+    hidden, n = 512, 5
+    x = G.normal_bf16(15, 1, (n, hidden))
+    W = G.normal_scaled_bf16(15, 2, (O.PROJ_FEATURES, hidden), hidden ** -0.5)
+    idx_q, idx_k, w = O.index_project(x, W, nthreads=2)
+    y = f32(x).astype(np.float64) @ f32(W).astype(np.float64).T  # [n, 644]
+    yq, yk, yw = y[:, :512].reshape(n, 4, 128), y[:, 512:640], y[:, 640:]
+    for got, ref in ((idx_q, yq), (idx_k, yk)):
+        g = f32(got).astype(np.float64)
+        assert np.all(np.abs(g - ref) <= 0.5 * bf16_ulp(ref) * (1 + 1e-9) + 1e-300)
+    np.testing.assert_allclose(w, yw.astype(np.float32), rtol=1e-6, atol=0)
+    # swapping the roles of rows and features, or reading W transposed, changes the result
+    assert not np.array_equal(idx_q[0, 0], idx_q[1, 0])
+    x2 = x.copy()
+    x2[:, 0] = x[:, 1]
+    x2[:, 1] = x[:, 0]
+    q2, _, _ = O.index_project(x2, W, nthreads=1)
+    assert not np.array_equal(q2, idx_q)
