@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-scorer measurement")
     ap.add_argument("--only-prefill", action="store_true",
                     help="run only the prefill-scorer measurement and print its JSON (for profiling it alone)")
+    ap.add_argument("--no-long-prefill", action="store_true",
+                    help="with the prefill measurement, skip the 262144-token long-context prefill")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     return ap.parse_args()
 
@@ -394,14 +396,24 @@ def prefill_flops(pos0: int, T: int) -> int:
     return int(((t + 1) // 4).sum()) * 4 * 128 * 2
 
 
-def run_prefill_scorer(dev, reps: int = 20):
-    """Time the tensor-core prefill scorer on the 32768-token causal chunk (every token a query)."""
+def bf16_peak():
+    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pk):
+        return float(json.load(open(pk))["bf16_tflops"]), "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
+    return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def run_prefill_scorer(dev, reps: int = 20, long_context: bool = True):
+    """Time qsa_prefill_score_topk (rotation, tensor-core scoring with candidate filtering, exact
+    top-512) on the 32768-token causal chunk, every token a query, and on the 262144-token prefill
+    of the long-context workload in its 32 causal chunks of 8192 queries."""
     import torch
 
     import block_sparse_attention_c4_b200 as Q
     import block_sparse_attention_c4_b200.workload as W
     import qsa_gen as G
 
+    peak, src = bf16_peak()
     wl = G.prefill_32k()
     T = 32768
     cache = W.build_cache(wl, device=dev, prefix_tokens=[T])
@@ -416,6 +428,7 @@ def run_prefill_scorer(dev, reps: int = 20):
     torch.cuda.synchronize()
     if ws.device_error() != 0:
         raise RuntimeError("device error word set in the prefill scorer")
+    rescored = Q.prefill_rescored_rows(ws, T, T)
     st = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(reps)]
     for e in ev:
@@ -430,24 +443,94 @@ def run_prefill_scorer(dev, reps: int = 20):
     torch.cuda.synchronize()
     ms = [[ev[k][2 * i].elapsed_time(ev[k][2 * i + 1]) for k in range(reps)] for i in range(3)]
     total = [ev[k][0].elapsed_time(ev[k][5]) for k in range(reps)]
+    # the call without events between its kernels
+    evc = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for k in range(reps):
+        flush.zero_()
+        evc[k][0].record(st)
+        Q.prefill_score_topk(cache, idx_q, w, 0, 0, ws, blocks, nblocks)
+        evc[k][1].record(st)
+    torch.cuda.synchronize()
+    call_ms = float(np.mean([a.elapsed_time(b) for a, b in evc]))
     flops = prefill_flops(0, T)
     score_s = float(np.mean(ms[1])) * 1e-3
-    peak = 1590.0
-    src = "fallback 1.59 PFLOP/s"
-    pk = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(pk):
-        peak = float(json.load(open(pk))["bf16_tflops"])
-        src = "measured burst bf16 (MEASURED_PEAKS.json bf16_tflops)"
-    ach = flops / score_s / 1e12
-    return {
+    call_ach = flops / (call_ms * 1e-3) / 1e12
+    mma_ach = flops / score_s / 1e12
+    res = {
         "workload": "prefill_L32768 (one causal chunk of 32768 queries)",
-        "call_us": round(float(np.mean(total)) * 1e3, 2),
+        "call_us": round(call_ms * 1e3, 2),
         "kernels_us": {"rotate": round(float(np.mean(ms[0])) * 1e3, 2), "score_tcgen05": round(score_s * 1e6, 2),
-                       "finalize": round(float(np.mean(ms[2])) * 1e3, 2)},
-        "query_tok_per_s": round(T / (float(np.mean(total)) * 1e-3), 1),
-        "roofline": {"kernel": "k_prefill_score", "bound": "tensor", "achieved": round(ach, 1), "peak": peak,
-                     "peak_source": src, "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                       "select_and_rescore": round(float(np.mean(ms[2])) * 1e3, 2),
+                       "sum_with_events": round(float(np.mean(total)) * 1e3, 2)},
+        "rows_rescored_in_full": rescored,
+        "query_tok_per_s": round(T / (call_ms * 1e-3), 1),
+        "roofline": {"kernel": "qsa_prefill_score_topk (whole call)", "bound": "tensor", "achieved": round(call_ach, 1),
+                     "peak": peak, "peak_source": src, "unit": "TFLOP/s", "frac": round(call_ach / peak, 4),
                      "algorithmic_flops_per_launch": flops},
+        "roofline_mma_kernel": {"kernel": "k_prefill_score", "bound": "tensor", "achieved": round(mma_ach, 1),
+                                "peak": peak, "unit": "TFLOP/s", "frac": round(mma_ach / peak, 4),
+                                "note": "includes the sample pass (1/8 extra MMA, not in the algorithmic FLOPs)"},
+    }
+    del cache, ws, blocks, nblocks, idx_q, w
+    torch.cuda.empty_cache()
+    if long_context:
+        res["long_context_prefill"] = run_long_prefill(dev, flush)
+    return res
+
+
+def run_long_prefill(dev, flush, chunk: int = 8192, L: int = 262144):
+    """The 262144-token prefill in causal chunks of 8192 queries: every chunk's qsa_prefill_score_topk
+    timed by CUDA events (the cache holds the index keys of all 262144 tokens; a chunk's queries only
+    see the blocks before them)."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+    import qsa_gen as G
+
+    peak, src = bf16_peak()
+    wl = G.long_262k()
+    cache = W.build_cache(wl, device=dev, prefix_tokens=[0])
+    for t0 in range(0, L, chunk):
+        W.append_tokens(cache, wl, 0, t0, chunk)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, chunk, L), device=dev)
+    blocks = torch.empty(chunk, 512, dtype=torch.int32, device=dev)
+    nblocks = torch.empty(chunk, dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream()
+    chunks = []
+    for pos0 in range(0, L, chunk):
+        idx_q = W.bits_to_bf16(wl.idx_q(0, pos0, chunk), dev)
+        w = torch.from_numpy(wl.w(0, pos0, chunk)).to(dev)
+        chunks.append((pos0, idx_q, w))
+    for pos0, idx_q, w in chunks[-2:]:  # warm-up
+        Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws, blocks, nblocks)
+    torch.cuda.synchronize()
+    if ws.device_error() != 0:
+        raise RuntimeError("device error word set in the long-context prefill")
+    times, rescored = [], 0
+    for pos0, idx_q, w in chunks:
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws, blocks, nblocks)
+        b.record(st)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+        rescored += Q.prefill_rescored_rows(ws, chunk, pos0 + chunk)
+    if ws.device_error() != 0:
+        raise RuntimeError("device error word set in the long-context prefill")
+    flops = sum(prefill_flops(pos0, chunk) for pos0, _, _ in chunks)
+    total_ms = float(np.sum(times))
+    ach = flops / (total_ms * 1e-3) / 1e12
+    return {
+        "workload": f"prefill_L{L} in {len(chunks)} causal chunks of {chunk} queries",
+        "total_ms": round(total_ms, 3),
+        "chunk_ms_first_last": [round(times[0], 3), round(times[-1], 3)],
+        "rows_rescored_in_full": rescored,
+        "query_tok_per_s": round(L / (total_ms * 1e-3), 1),
+        "roofline": {"kernel": "qsa_prefill_score_topk (whole calls)", "bound": "tensor", "achieved": round(ach, 1),
+                     "peak": peak, "peak_source": src, "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                     "algorithmic_flops": flops},
     }
 
 
@@ -559,7 +642,9 @@ def main():
         build.build()
         torch.cuda.set_device(local_rank)
         if rank == 0:
-            print(json.dumps({"prefill_scorer": run_prefill_scorer(torch.device("cuda", local_rank))}), flush=True)
+            print(json.dumps({"prefill_scorer": run_prefill_scorer(torch.device("cuda", local_rank),
+                                                                   long_context=not args.no_long_prefill)}),
+                  flush=True)
         return
     res, wl = run_ours(args, rank, world, local_rank)
     if rank == 0:

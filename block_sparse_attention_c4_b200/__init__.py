@@ -28,7 +28,7 @@ MAX_DRAFT = 8
 
 OP_INDEX_SCORE_TOPK, OP_SPARSE_GQA, OP_DECODE, OP_DECODE_INDEXSHARE, OP_COMPRESS_APPEND = 1, 2, 3, 4, 5
 OP_PREFILL_SCORE_TOPK = 6
-OP_DECODE_INDEXER, OP_DECODE_ATTEND = 7, 8
+OP_DECODE_INDEXER, OP_DECODE_ATTEND, OP_SPLIT_SCORE = 7, 8, 9
 PROJ_FEATURES = INDEX_HEADS * HEAD_DIM + HEAD_DIM + INDEX_HEADS  # 644
 
 DEVERR_BITS = {1: "page", 2: "length", 4: "position", 8: "request", 16: "selection", 32: "timeout"}
@@ -53,7 +53,7 @@ EXPORTS = [
     "qsa_expand_indices", "qsa_sparse_gqa", "qsa_decode", "qsa_decode_indexshare", "qsa_device_error",
     "qsa_set_profile_events", "qsa_decode_kernel_count", "qsa_status_string", "qsa_version",
     "qsa_prefill_score_topk", "qsa_sparse_gqa_noalloc", "qsa_check_bounded_wait", "qsa_last_error_string",
-    "qsa_index_project", "qsa_decode_indexer", "qsa_decode_attend",
+    "qsa_index_project", "qsa_decode_indexer", "qsa_decode_attend", "qsa_prefill_rescored_rows",
 ]
 
 
@@ -85,6 +85,20 @@ def lib():
     L.qsa_decode_attend.argtypes = [cp, vp, vp, i32, vp, vp, f32, vp, vp, vp, sz, vp]
     for f in (L.qsa_index_project, L.qsa_decode_indexer, L.qsa_decode_attend):
         f.restype = ctypes.c_int
+    L.qsa_prefill_score_topk_varlen.argtypes = [cp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, sz, vp]
+    L.qsa_prefill_score_topk_varlen.restype = ctypes.c_int
+    L.qsa_split_score_topk.argtypes = [cp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    L.qsa_split_merge.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp]
+    L.qsa_split_positions.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, vp]
+    L.qsa_split_combine.argtypes = [vp, vp, i32, i32, vp, vp]
+    for f in (L.qsa_split_score_topk, L.qsa_split_merge, L.qsa_split_positions, L.qsa_split_combine):
+        f.restype = ctypes.c_int
+    L.qsa_sparse_gqa_fp8.argtypes = [cp, f32, f32, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    L.qsa_decode_fp8.argtypes = [cp, f32, f32, vp, vp, vp, vp, vp, i32, f32, vp, vp, vp, vp, vp, sz, vp]
+    L.qsa_sparse_gqa_fp8.restype = ctypes.c_int
+    L.qsa_decode_fp8.restype = ctypes.c_int
+    L.qsa_prefill_rescored_rows.argtypes = [vp, i32, i32, vp]
+    L.qsa_prefill_rescored_rows.restype = i32
     L.qsa_check_bounded_wait.argtypes = [cp, vp, vp, ctypes.c_uint64, vp, sz, vp]
     L.qsa_check_bounded_wait.restype = ctypes.c_int
     L.qsa_device_error.argtypes = [vp, i32, vp]
@@ -167,24 +181,28 @@ class LayerCache:
     page_table: int32 [batch, max_pages].
     kv_layout "interleaved" keeps each slot's K and V rows together (kv: [num_slots, 2, 2, 128], k and
     v its two halves), so the 4 slots of a compressed block are one 4 KiB run; "separate" allocates
-    two arrays.
+    two arrays.  kv_dtype "fp8" stores K and V as E4M3 codes (uint8 tensors of the same shapes; strides
+    counted in bytes) for the *_fp8 calls.
     """
 
     def __init__(self, num_slots: int, batch: int, max_pages: int, rope_theta: float = 1.0e7, device="cuda",
-                 page_table: torch.Tensor | None = None, kv_layout: str = "interleaved"):
+                 page_table: torch.Tensor | None = None, kv_layout: str = "interleaved", kv_dtype: str = "bf16"):
         if num_slots % PAGE_SIZE:
             raise QsaError("num_slots must be a multiple of 64")
         if kv_layout not in ("interleaved", "separate"):
             raise QsaError(f"kv_layout must be 'interleaved' or 'separate', got {kv_layout!r}")
         self.num_slots, self.batch, self.max_pages, self.rope_theta = num_slots, batch, max_pages, rope_theta
-        self.kv_layout = kv_layout
+        if kv_dtype not in ("bf16", "fp8"):
+            raise QsaError(f"kv_dtype must be 'bf16' or 'fp8', got {kv_dtype!r}")
+        self.kv_layout, self.kv_dtype = kv_layout, kv_dtype
+        dt = torch.bfloat16 if kv_dtype == "bf16" else torch.uint8
         if kv_layout == "interleaved":
-            self.kv = torch.zeros(num_slots, 2, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+            self.kv = torch.zeros(num_slots, 2, KV_HEADS, HEAD_DIM, dtype=dt, device=device)
             self.k, self.v = self.kv[:, 0], self.kv[:, 1]
             self.kv_stride = 2 * KV_HEADS * HEAD_DIM
         else:
-            self.k = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
-            self.v = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+            self.k = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=dt, device=device)
+            self.v = torch.zeros(num_slots, KV_HEADS, HEAD_DIM, dtype=dt, device=device)
             self.kv_stride = 0
         self.cidx = torch.zeros(num_slots // BLOCK, HEAD_DIM, dtype=torch.bfloat16, device=device)
         self.ring = torch.zeros(max(batch, 1), BLOCK, HEAD_DIM, dtype=torch.bfloat16, device=device)
@@ -246,6 +264,39 @@ def prefill_score_topk(cache: LayerCache, idx_q, w, req: int, pos0: int, ws: Wor
     return blocks, nblocks
 
 
+def prefill_score_topk_varlen(cache: LayerCache, idx_q, w, seg_req, seg_pos0, cu_q, max_len: int, ws: Workspace,
+                              blocks=None, nblocks=None, stream=None):
+    """Tensor-core scoring + top-512 of a ragged batch of causal chunks: segment i is request seg_req[i],
+    queries at positions seg_pos0[i] .. + (cu_q[i+1] - cu_q[i]) - 1, rows cu_q[i] .. cu_q[i+1]-1 of
+    idx_q / w / blocks / nblocks.  seg_req, seg_pos0, cu_q are host sequences."""
+    import numpy as np
+
+    nseg = len(seg_req)
+    req = np.ascontiguousarray(seg_req, dtype=np.int32)
+    pos0 = np.ascontiguousarray(seg_pos0, dtype=np.int32)
+    cu = np.ascontiguousarray(cu_q, dtype=np.int32)
+    if len(pos0) != nseg or len(cu) != nseg + 1:
+        raise QsaError("seg_req, seg_pos0 need nseg entries and cu_q nseg + 1")
+    T = int(cu[-1])
+    dev = idx_q.device
+    blocks = torch.full((T, TOPK), -1, dtype=torch.int32, device=dev) if blocks is None else blocks
+    nblocks = torch.zeros(T, dtype=torch.int32, device=dev) if nblocks is None else nblocks
+    c = cache.struct()
+    _dev(blocks, torch.int32, "blocks", (T, TOPK))
+    _dev(nblocks, torch.int32, "nblocks", (T,))
+    _check(lib().qsa_prefill_score_topk_varlen(
+        ctypes.byref(c), _ptr(_dev(idx_q, torch.bfloat16, "idx_q", (T, INDEX_HEADS, HEAD_DIM))),
+        _ptr(_dev(w, torch.float32, "w", (T, INDEX_HEADS))), nseg, req.ctypes.data_as(ctypes.c_void_p),
+        pos0.ctypes.data_as(ctypes.c_void_p), cu.ctypes.data_as(ctypes.c_void_p), int(max_len), _ptr(blocks),
+        _ptr(nblocks), ws.ptr, ws.nbytes, _stream(stream)), "qsa_prefill_score_topk_varlen")
+    return blocks, nblocks
+
+
+def prefill_rescored_rows(ws: Workspace, T: int, max_len: int, stream=None) -> int:
+    """Rows of the last prefill_score_topk call on `ws` that were re-scored in full (synchronises)."""
+    return int(lib().qsa_prefill_rescored_rows(ws.ptr, int(T), int(max_len), _stream(stream)))
+
+
 def expand_indices(blocks, nblocks, q_pos, pos=None, npos=None, stream=None):
     nq = int(q_pos.shape[0])
     dev = q_pos.device
@@ -278,6 +329,57 @@ def sparse_gqa(cache: LayerCache, q, q_req, pos, npos, max_pos: int, ws: Workspa
                                 _ptr(_dev(npos, torch.int32, "npos", (nq,))), int(pos.shape[1]), int(max_pos), nq,
                                 float(scale), _ptr(out), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)),
            "qsa_sparse_gqa")
+    return out
+
+
+def _need_fp8(cache: LayerCache, name: str):
+    if cache.kv_dtype != "fp8":
+        raise QsaError(f"{name} needs a cache with kv_dtype='fp8'")
+
+
+def sparse_gqa_fp8(cache: LayerCache, q, q_req, pos, npos, max_pos: int, ws: Workspace, k_scale: float,
+                   v_scale: float, scale: float | None = None, out=None, lse=None, stream=None):
+    """qsa_sparse_gqa over an FP8 (E4M3) K/V pool: value = code * k_scale (keys), code * v_scale (values)."""
+    _need_fp8(cache, "sparse_gqa_fp8")
+    nq = int(q.shape[0])
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    out = torch.empty(nq, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device) if out is None else out
+    c = cache.struct()
+    _dev(out, torch.bfloat16, "out", (nq, Q_HEADS, HEAD_DIM))
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (nq, Q_HEADS))
+    _check(lib().qsa_sparse_gqa_fp8(ctypes.byref(c), float(k_scale), float(v_scale),
+                                    _ptr(_dev(q, torch.bfloat16, "q", (nq, Q_HEADS, HEAD_DIM))),
+                                    _ptr(_dev(q_req, torch.int32, "q_req", (nq,))), _ptr(_dev(pos, torch.int32, "pos")),
+                                    _ptr(_dev(npos, torch.int32, "npos", (nq,))), int(pos.shape[1]), int(max_pos), nq,
+                                    float(scale), _ptr(out), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)),
+           "qsa_sparse_gqa_fp8")
+    return out
+
+
+def decode_fp8(cache: LayerCache, idx_k_new, idx_q, w, q, seq_len, max_len: int, ws: Workspace, k_scale: float,
+               v_scale: float, scale: float | None = None, out=None, lse=None, blocks_out=None, nblocks_out=None,
+               stream=None):
+    """qsa_decode over an FP8 (E4M3) K/V pool."""
+    _need_fp8(cache, "decode_fp8")
+    B = cache.batch
+    scale = HEAD_DIM ** -0.5 if scale is None else scale
+    out = torch.empty(B, Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device) if out is None else out
+    c = cache.struct()
+    _dev(out, torch.bfloat16, "out", (B, Q_HEADS, HEAD_DIM))
+    if lse is not None:
+        _dev(lse, torch.float32, "lse", (B, Q_HEADS))
+    if blocks_out is not None:
+        _dev(blocks_out, torch.int32, "blocks_out", (B, TOPK))
+        _dev(nblocks_out, torch.int32, "nblocks_out", (B,))
+    _check(lib().qsa_decode_fp8(ctypes.byref(c), float(k_scale), float(v_scale),
+                                _ptr(_dev(idx_k_new, torch.bfloat16, "idx_k_new", (B, HEAD_DIM))),
+                                _ptr(_dev(idx_q, torch.bfloat16, "idx_q", (B, INDEX_HEADS, HEAD_DIM))),
+                                _ptr(_dev(w, torch.float32, "w", (B, INDEX_HEADS))),
+                                _ptr(_dev(q, torch.bfloat16, "q", (B, Q_HEADS, HEAD_DIM))),
+                                _ptr(_dev(seq_len, torch.int32, "seq_len", (B,))), int(max_len), float(scale),
+                                _ptr(out), _ptr(lse), _ptr(blocks_out), _ptr(nblocks_out), ws.ptr, ws.nbytes,
+                                _stream(stream)), "qsa_decode_fp8")
     return out
 
 

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "qsa_common.cuh"
@@ -24,9 +25,11 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct WsLayout {
   size_t cnt_gqa = 0, qrot = 0, sel = 0, sel_n = 0, row_pages = 0, page_off = 0, pages_done = 0, cand_key = 0,
          cand_id = 0, part_o = 0, part_ml = 0, total = 0;
-  size_t pf_keys = 0, pf_ovf_n = 0, pf_ovf_list = 0;
+  size_t pf_qbase = 0, pf_cand = 0, pf_cand_n = 0, pf_fb_n = 0, pf_fb_list = 0, pf_fb_keys = 0;
   size_t ready = 0;  // decode: per-row flag, selection final (scorer -> sparse GQA)
   size_t pj_q = 0, pj_k = 0, pj_w = 0;  // decode indexer: projected index queries, keys, head weights
+  size_t sp_key = 0, sp_id = 0, sp_n = 0;  // split scoring: per-chunk candidates
+  int sp_chunks = 0;
   int ppc_min = 0;
   int seg_cap = 0;
   int splits_bound = 0;
@@ -60,7 +63,7 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
   const bool gqa = op == QSA_OP_SPARSE_GQA || op == QSA_OP_DECODE || op == QSA_OP_DECODE_INDEXSHARE ||
                    op == QSA_OP_DECODE_ATTEND;
   const bool prefill = op == QSA_OP_PREFILL_SCORE_TOPK;
-  if (!scorer && !gqa && !prefill && op != QSA_OP_COMPRESS_APPEND) return false;
+  if (!scorer && !gqa && !prefill && op != QSA_OP_COMPRESS_APPEND && op != QSA_OP_SPLIT_SCORE) return false;
   if (op == QSA_OP_DECODE_ATTEND) op = QSA_OP_DECODE;  // the decode step's attention part
   size_t off = 256;  // error word, prologue ticket, spare
   auto take = [&](size_t bytes) {
@@ -68,12 +71,24 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     off += align256(bytes);
     return at;
   };
+  if (op == QSA_OP_SPLIT_SCORE) {
+    w.sp_chunks = std::max(1, ceil_div(std::max(1, max_len / QSA_BLOCK), SPLIT_CHUNK_BLOCKS));
+    if (w.sp_chunks > SPLIT_MAX_LISTS) return false;
+    w.sp_key = take((size_t)rows * w.sp_chunks * TOPK * 4);
+    w.sp_id = take((size_t)rows * w.sp_chunks * TOPK * 4);
+    w.sp_n = take((size_t)rows * w.sp_chunks * 4);
+    w.total = off;
+    return true;
+  }
   if (prefill) {
-    w.cap = (std::max(1, max_len / QSA_BLOCK) + 127) / 128 * 128;
+    w.cap = (std::max(1, max_len / QSA_BLOCK) + 31) / 32 * 32;  // blocks of the longest row, whole words
     w.qrot = take((size_t)rows * HI * D * 2);
-    w.pf_keys = take((size_t)ceil_div(rows, 64) * 64 * w.cap * 4);
-    w.pf_ovf_n = take(4);
-    w.pf_ovf_list = take((size_t)rows * 4);
+    w.pf_qbase = take((size_t)rows * 4);
+    w.pf_cand = take((size_t)rows * 4 * PF_QCAP * 8);
+    w.pf_cand_n = take((size_t)rows * 4 * 4);
+    w.pf_fb_n = take(4);
+    w.pf_fb_list = take((size_t)rows * 4);
+    w.pf_fb_keys = take((size_t)SIZING_SMS * w.cap * 4);
     w.total = off;
     return true;
   }
@@ -133,6 +148,13 @@ qsa_status check_cache(const qsa_cache* c) {
   if (!c->cidx || !c->ring) return QSA_ERR_INVALID_ARG;
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) return QSA_ERR_INVALID_ARG;
   if (!aligned(c->cidx, 16) || !aligned(c->ring, 16)) return QSA_ERR_INVALID_ARG;
+  return QSA_OK;
+}
+
+// FP8 K/V: rows of 128 E4M3 bytes per KV head; kv_stride (bytes) 0 (= 256) or a multiple of 16, at least 256.
+qsa_status check_fp8(const qsa_cache* c, float k_scale, float v_scale) {
+  if (c->kv_stride != 0 && c->kv_stride % 16 != 0) return QSA_ERR_INVALID_ARG;
+  if (!valid_scale(k_scale) || !valid_scale(v_scale)) return QSA_ERR_INVALID_ARG;
   return QSA_OK;
 }
 
@@ -283,6 +305,16 @@ void qsa_set_profile_events(void* const* events, int32_t n_pairs) {
   g_prof_pairs = n_pairs;
 }
 
+int32_t qsa_prefill_rescored_rows(void* ws, int32_t T, int32_t max_len, void* stream) {
+  WsLayout L;
+  if (!ws || T < 1 || !layout(QSA_OP_PREFILL_SCORE_TOPK, T, max_len, L)) return -1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, at<int>(ws, L.pf_fb_n), sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return -1;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
+  return v;
+}
+
 int32_t qsa_decode_kernel_count(int32_t batch) { return batch <= SC_ROWS_SMEM ? 2 : 3; }
 
 qsa_status qsa_compress_append(const qsa_cache* cache, const void* idx_k_new, const int32_t* cu_new,
@@ -316,31 +348,65 @@ qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const
                      max_len, w, blocks, nblocks, ws, L, static_cast<cudaStream_t>(stream));
 }
 
-qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, int32_t req,
-                                  int32_t pos0, int32_t T, int32_t* blocks, int32_t* nblocks, void* ws,
-                                  size_t ws_bytes, void* stream) {
+qsa_status qsa_prefill_score_topk_varlen(const qsa_cache* cache, const void* idx_q, const float* w, int32_t nseg,
+                                         const int32_t* seg_req, const int32_t* seg_pos0, const int32_t* cu_q,
+                                         int32_t max_len, int32_t* blocks, int32_t* nblocks, void* ws,
+                                         size_t ws_bytes, void* stream) {
   qsa_status s = check_cache(cache);
   if (s != QSA_OK) return s;
-  if (T < 0 || pos0 < 0 || (int64_t)pos0 + T > QSA_MAX_CONTEXT) return QSA_ERR_INVALID_ARG;
-  if (T == 0) return QSA_OK;
-  if (req < 0 || req >= cache->batch) return QSA_ERR_INVALID_ARG;
-  if ((int64_t)pos0 + T > (int64_t)cache->max_pages * QSA_PAGE_SIZE) return QSA_ERR_INVALID_ARG;
+  if (nseg < 0 || nseg > PF_MAX_SEGS) return nseg < 0 ? QSA_ERR_INVALID_ARG : QSA_ERR_UNSUPPORTED;
+  if (nseg == 0) return QSA_OK;
+  if (!seg_req || !seg_pos0 || !cu_q || cu_q[0] != 0) return QSA_ERR_INVALID_ARG;
+  if (max_len < 1 || max_len > QSA_MAX_CONTEXT || (int64_t)max_len > (int64_t)cache->max_pages * QSA_PAGE_SIZE)
+    return QSA_ERR_INVALID_ARG;
+  PrefillParams p{};
+  int order[PF_MAX_SEGS], n_live = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const int T = cu_q[i + 1] - cu_q[i];
+    if (T < 0 || seg_pos0[i] < 0 || (int64_t)seg_pos0[i] + T > max_len) return QSA_ERR_INVALID_ARG;
+    if (seg_req[i] < 0 || seg_req[i] >= cache->batch) return QSA_ERR_INVALID_ARG;
+    if (T > 0) order[n_live++] = i;
+  }
+  const int total = cu_q[nseg];
+  if (n_live == 0) return QSA_OK;
   if (!idx_q || !w || !blocks || !nblocks) return QSA_ERR_INVALID_ARG;
   if (!aligned(idx_q, 16) || !aligned(w, 16)) return QSA_ERR_INVALID_ARG;
+  // longest contexts first: their tiles are the most expensive, so they start first
+  std::stable_sort(order, order + n_live, [&](int a, int b) {
+    return (int64_t)seg_pos0[a] + (cu_q[a + 1] - cu_q[a]) > (int64_t)seg_pos0[b] + (cu_q[b + 1] - cu_q[b]);
+  });
+  int tiles = 0, rows = 0;
+  for (int k = 0; k < n_live; ++k) {
+    const int i = order[k];
+    PfSeg& sg = p.seg[k];
+    sg.req = seg_req[i];
+    sg.pos0 = seg_pos0[i];
+    sg.T = cu_q[i + 1] - cu_q[i];
+    sg.q_off = cu_q[i];
+    sg.tile_off = tiles;
+    sg.row_off = rows;
+    tiles += ceil_div(sg.T, 64);
+    rows += sg.T;
+  }
   WsLayout L;
-  if (!layout(QSA_OP_PREFILL_SCORE_TOPK, T, pos0 + T, L)) return QSA_ERR_INVALID_ARG;
+  if (!layout(QSA_OP_PREFILL_SCORE_TOPK, total, max_len, L)) return QSA_ERR_INVALID_ARG;
   if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
-  PrefillParams p;
   p.c = view_of(cache);
-  p.req = req;
-  p.pos0 = pos0;
-  p.T = T;
+  p.nseg = n_live;
+  p.T = total;
+  p.ntiles = tiles;
   p.w = w;
   p.qrot = at<__nv_bfloat16>(ws, L.qrot);
-  p.keys = at<uint32_t>(ws, L.pf_keys);
-  p.ovf_n = at<int>(ws, L.pf_ovf_n);
-  p.ovf_list = at<int32_t>(ws, L.pf_ovf_list);
-  p.cap = L.cap;
+  p.qbase = at<int32_t>(ws, L.pf_qbase);
+  p.cand = at<unsigned long long>(ws, L.pf_cand);
+  p.cand_n = at<int32_t>(ws, L.pf_cand_n);
+  p.fb_n = at<int>(ws, L.pf_fb_n);
+  p.fb_list = at<int32_t>(ws, L.pf_fb_list);
+  p.fb_keys = at<uint32_t>(ws, L.pf_fb_keys);
+  p.fb_cap = L.cap;
+  p.fb_ctas = std::min(num_sms(), SIZING_SMS);
+  p.wait_ns = 0;
+  p.stats = nullptr;
   p.sel = blocks;
   p.sel_n = nblocks;
   p.err = at<int>(ws, WS_ERR);
@@ -348,6 +414,16 @@ qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, con
   return cuda_status(launch_prefill(p, static_cast<const __nv_bfloat16*>(idx_q), make_freqs(cache->rope_theta),
                                     num_sms(), static_cast<cudaStream_t>(stream), g_prof_pairs ? g_prof : nullptr,
                                     g_prof_pairs));
+}
+
+qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, int32_t req,
+                                  int32_t pos0, int32_t T, int32_t* blocks, int32_t* nblocks, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (T < 0 || pos0 < 0 || (int64_t)pos0 + T > QSA_MAX_CONTEXT) return QSA_ERR_INVALID_ARG;
+  if (T == 0) return check_cache(cache);
+  const int32_t cu[2] = {0, T};
+  return qsa_prefill_score_topk_varlen(cache, idx_q, w, 1, &req, &pos0, cu, pos0 + T, blocks, nblocks, ws, ws_bytes,
+                                       stream);
 }
 
 qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, const int32_t* q_pos, int32_t nq,
@@ -358,9 +434,12 @@ qsa_status qsa_expand_indices(const int32_t* blocks, const int32_t* nblocks, con
   return cuda_status(launch_expand(blocks, nblocks, q_pos, nq, pos, npos, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
-qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* q_req, const int32_t* pos,
-                          const int32_t* npos, int32_t pos_stride, int32_t max_pos, int32_t nq, float scale,
-                          void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C" (reopened below)
+
+static qsa_status sparse_gqa_impl(const qsa_cache* cache, const void* q, const int32_t* q_req, const int32_t* pos,
+                                  const int32_t* npos, int32_t pos_stride, int32_t max_pos, int32_t nq, float scale,
+                                  void* out, float* lse, void* ws, size_t ws_bytes, void* stream, int fp8,
+                                  float k_scale, float v_scale) {
   qsa_status s = check_cache(cache);
   if (s != QSA_OK) return s;
   if (nq < 0 || pos_stride < 0 || max_pos < 0 || max_pos > pos_stride || !valid_scale(scale))
@@ -382,7 +461,9 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
   p.list = pos;
   p.list_n = npos;
   p.list_stride = pos_stride;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.fp8 = fp8;
+  p.v_scale = v_scale;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.part_o = at<float>(ws, L.part_o);
@@ -392,9 +473,10 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
   return cuda_status(launch_gqa(p, nq, max_pos, num_sms(), L.splits_bound, static_cast<cudaStream_t>(stream)));
 }
 
-qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
-                      const void* q, const int32_t* seq_len, int32_t max_len, float scale, void* out, float* lse,
-                      int32_t* blocks_out, int32_t* nblocks_out, void* ws, size_t ws_bytes, void* stream) {
+static qsa_status decode_impl(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
+                              const void* q, const int32_t* seq_len, int32_t max_len, float scale, void* out,
+                              float* lse, int32_t* blocks_out, int32_t* nblocks_out, void* ws, size_t ws_bytes,
+                              void* stream, int fp8, float k_scale, float v_scale) {
   qsa_status s = check_cache(cache);
   if (s != QSA_OK) return s;
   if (max_len < 1 || max_len > QSA_MAX_CONTEXT || !valid_scale(scale))
@@ -432,7 +514,9 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   p.row_len = seq_len;
   p.len_offset = 0;
   p.max_len = max_len;
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+  p.fp8 = fp8;
+  p.v_scale = v_scale;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.part_o = at<float>(ws, L.part_o);
@@ -442,6 +526,44 @@ qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void*
   p.row_ready = ready;
   ProfScope ps(st, qsa_decode_kernel_count(B) - 1);
   return cuda_status(launch_gqa(p, B, positions_bound(QSA_OP_DECODE, max_len), num_sms(), L.splits_bound, st));
+}
+
+extern "C" {
+
+qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* q_req, const int32_t* pos,
+                          const int32_t* npos, int32_t pos_stride, int32_t max_pos, int32_t nq, float scale,
+                          void* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return sparse_gqa_impl(cache, q, q_req, pos, npos, pos_stride, max_pos, nq, scale, out, lse, ws, ws_bytes, stream,
+                         0, 1.f, 1.f);
+}
+
+qsa_status qsa_sparse_gqa_fp8(const qsa_cache* cache, float k_scale, float v_scale, const void* q,
+                              const int32_t* q_req, const int32_t* pos, const int32_t* npos, int32_t pos_stride,
+                              int32_t max_pos, int32_t nq, float scale, void* out, float* lse, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (!cache) return QSA_ERR_INVALID_ARG;
+  const qsa_status s = check_fp8(cache, k_scale, v_scale);
+  if (s != QSA_OK) return s;
+  return sparse_gqa_impl(cache, q, q_req, pos, npos, pos_stride, max_pos, nq, scale, out, lse, ws, ws_bytes, stream,
+                         1, k_scale, v_scale);
+}
+
+qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
+                      const void* q, const int32_t* seq_len, int32_t max_len, float scale, void* out, float* lse,
+                      int32_t* blocks_out, int32_t* nblocks_out, void* ws, size_t ws_bytes, void* stream) {
+  return decode_impl(cache, idx_k_new, idx_q, w, q, seq_len, max_len, scale, out, lse, blocks_out, nblocks_out, ws,
+                     ws_bytes, stream, 0, 1.f, 1.f);
+}
+
+qsa_status qsa_decode_fp8(const qsa_cache* cache, float k_scale, float v_scale, const void* idx_k_new,
+                          const void* idx_q, const float* w, const void* q, const int32_t* seq_len, int32_t max_len,
+                          float scale, void* out, float* lse, int32_t* blocks_out, int32_t* nblocks_out, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (!cache) return QSA_ERR_INVALID_ARG;
+  const qsa_status s = check_fp8(cache, k_scale, v_scale);
+  if (s != QSA_OK) return s;
+  return decode_impl(cache, idx_k_new, idx_q, w, q, seq_len, max_len, scale, out, lse, blocks_out, nblocks_out, ws,
+                     ws_bytes, stream, 1, k_scale, v_scale);
 }
 
 qsa_status qsa_index_project(const void* x, const void* w_proj, int32_t n, int32_t hidden, void* idx_q, void* idx_k,
@@ -532,6 +654,71 @@ qsa_status qsa_decode_attend(const qsa_cache* cache, const void* q, const int32_
   p.err = at<int>(ws, WS_ERR);
   return cuda_status(launch_gqa(p, B, positions_bound(QSA_OP_DECODE, max_len), num_sms(), L.splits_bound,
                                 static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_split_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, const int32_t* seq_len,
+                                const int32_t* page_lo, const int32_t* page_cnt, int32_t max_len, uint32_t* cand_key,
+                                int32_t* cand_id, int32_t* cand_n, void* ws, size_t ws_bytes, void* stream) {
+  qsa_status s = check_cache(cache);
+  if (s != QSA_OK) return s;
+  if (max_len < 1 || max_len > QSA_MAX_CONTEXT) return QSA_ERR_INVALID_ARG;
+  const int B = cache->batch;
+  if (B == 0) return QSA_OK;
+  if (!idx_q || !w || !seq_len || !page_lo || !page_cnt || !cand_key || !cand_id || !cand_n) return QSA_ERR_INVALID_ARG;
+  if (!aligned(idx_q, 16) || !aligned(w, 4)) return QSA_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!layout(QSA_OP_SPLIT_SCORE, B, max_len, L)) return QSA_ERR_INVALID_ARG;
+  if ((s = check_ws(ws, ws_bytes, L.total)) != QSA_OK) return s;
+  SplitParams p{};
+  p.c = view_of(cache);
+  p.idx_q = static_cast<const __nv_bfloat16*>(idx_q);
+  p.w = w;
+  p.seq_len = seq_len;
+  p.page_lo = page_lo;
+  p.page_cnt = page_cnt;
+  p.max_len = max_len;
+  p.fr = make_freqs(cache->rope_theta);
+  p.nchunks = L.sp_chunks;
+  p.cand_key = at<uint32_t>(ws, L.sp_key);
+  p.cand_id = at<int32_t>(ws, L.sp_id);
+  p.cand_n = at<int32_t>(ws, L.sp_n);
+  p.out_key = cand_key;
+  p.out_id = cand_id;
+  p.out_n = cand_n;
+  p.err = at<int>(ws, WS_ERR);
+  return cuda_status(launch_split_score(p, B, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_split_merge(const uint32_t* cand_key, const int32_t* cand_id, const int32_t* cand_n, int32_t world,
+                           int32_t rows, int32_t* blocks, int32_t* nblocks, void* stream) {
+  if (world < 1 || world > SPLIT_MAX_LISTS || rows < 0) return world > SPLIT_MAX_LISTS ? QSA_ERR_UNSUPPORTED
+                                                                                       : QSA_ERR_INVALID_ARG;
+  if (rows == 0) return QSA_OK;
+  if (!cand_key || !cand_id || !cand_n || !blocks || !nblocks) return QSA_ERR_INVALID_ARG;
+  return cuda_status(launch_split_merge(cand_key, cand_id, cand_n, world, rows, blocks, nblocks,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_split_positions(const int32_t* seq_len, const int32_t* page_lo, const int32_t* page_cnt,
+                               const int32_t* blocks, const int32_t* nblocks, int32_t rows, int32_t* pos,
+                               int32_t* npos, void* stream) {
+  if (rows < 0) return QSA_ERR_INVALID_ARG;
+  if (rows == 0) return QSA_OK;
+  if (!seq_len || !page_lo || !page_cnt || !blocks || !nblocks || !pos || !npos) return QSA_ERR_INVALID_ARG;
+  SplitParams p{};
+  p.seq_len = seq_len;
+  p.page_lo = page_lo;
+  p.page_cnt = page_cnt;
+  return cuda_status(launch_split_positions(p, blocks, nblocks, rows, pos, npos, static_cast<cudaStream_t>(stream)));
+}
+
+qsa_status qsa_split_combine(const void* outs, const float* lses, int32_t world, int32_t rows, void* out,
+                             void* stream) {
+  if (world < 1 || rows < 0) return QSA_ERR_INVALID_ARG;
+  if (rows == 0) return QSA_OK;
+  if (!outs || !lses || !out || !aligned(outs, 8) || !aligned(out, 8)) return QSA_ERR_INVALID_ARG;
+  return cuda_status(launch_split_combine(static_cast<const __nv_bfloat16*>(outs), lses, world, rows,
+                                          static_cast<__nv_bfloat16*>(out), static_cast<cudaStream_t>(stream)));
 }
 
 qsa_status qsa_check_bounded_wait(const qsa_cache* cache, const void* q, void* out, uint64_t limit_ns, void* ws,

@@ -122,6 +122,8 @@ struct GqaParams {
                               // through distributed shared memory (part_o, part_ml, counters unused);
                               // 0: partials go through global memory, the last split merges them
   uint64_t wait_ns;           // limit of the row-flag wait (0: WAIT_LIMIT_NS)
+  int fp8;                    // 1: K/V are E4M3 bytes (c.kv_stride in bytes), scale_log2 includes the K scale
+  float v_scale;              // fp8: scale of the V values
 };
 constexpr int GQ_CLUSTER_MAX = 8;  // splits of one row in a cluster (portable cluster size)
 
@@ -131,21 +133,39 @@ int gqa_split_bound(int rows, int max_pos);
 cudaError_t launch_gqa(const GqaParams& p, int rows, int max_pos, int num_sms, int split_bound, cudaStream_t st);
 
 // ---- prefill scorer on tcgen05 (qsa_prefill.cu) ----
+constexpr int PF_QCAP = 512;            // candidates kept per (query, TMEM quadrant) list
+constexpr int PF_EMIT_ALL = 4 * PF_QCAP - 128;  // queries with at most this many blocks emit every block
+constexpr int PF_NO_BASE = -(1 << 30);  // a query whose scores are all <= 0 (no histogram range)
+
+// One sequence of a (ragged) prefill call: request req, queries at positions pos0 .. pos0+T-1, stored
+// at rows q_off .. q_off+T-1 of the call's query arrays.  The segments are listed in the order their
+// work is scheduled (longest contexts first); tile_off / row_off are prefix sums in that order.
+constexpr int PF_MAX_SEGS = 64;
+struct PfSeg {
+  int req, pos0, T, q_off, tile_off, row_off;
+};
+
 struct PrefillParams {
   CacheView c;
-  int req;                 // request of the chunk
-  int pos0;                // position of the chunk's first query
-  int T;                   // queries (positions pos0 .. pos0+T-1)
+  int nseg;                // segments (1 .. PF_MAX_SEGS)
+  int T;                   // queries of the call (all segments)
+  int ntiles;              // work tiles of 64 queries (all segments)
+  PfSeg seg[PF_MAX_SEGS];
   const float* w;          // [T][4] head weights (16-byte aligned)
   __nv_bfloat16* qrot;     // [T*4][128] rotated index queries (written by the rotation kernel)
-  uint32_t* keys;          // [ceil(T/64)][cap/128][64][128] order-preserving score keys of the work tiles
-  int cap;                 // score slots per query: >= visible blocks of the last query, a multiple of 128
+  int32_t* qbase;          // [T] histogram base of each query (rotation kernel), or PF_NO_BASE
+  unsigned long long* cand;  // [T][4][PF_QCAP] candidates (key << 32 | ~block) per TMEM quadrant
+  int32_t* cand_n;         // [T][4] candidates emitted per list (may exceed PF_QCAP: overflow)
   int32_t* sel;            // [T][512] out
   int32_t* sel_n;          // [T] out
-  int* ovf_n;              // rows handed to the overflow selection (zeroed per call)
-  int32_t* ovf_list;       // [T]
+  int* fb_n;               // rows handed to the exact re-scoring (zeroed per call)
+  int32_t* fb_list;        // [T]
+  uint32_t* fb_keys;       // [fb_ctas][fb_cap] score keys of the rows being re-scored
+  int fb_cap;              // >= blocks visible to the chunk's last query, a multiple of 16
+  int fb_ctas;             // CTAs of the re-scoring kernel (rows of fb_keys)
   int* err;
   uint64_t wait_ns;        // limit of each mbarrier wait (0: WAIT_LIMIT_NS)
+  int* stats;              // nullable [4]: rows selected from candidates, rows re-scored, candidates, -
 };
 
 // ---- index projection (qsa_proj.cu) ----
@@ -158,6 +178,35 @@ struct ProjParams {
   float* wout;             // [n][4] out
 };
 cudaError_t launch_index_proj(const ProjParams& p, cudaStream_t st);
+
+// ---- split-context decode (qsa_split.cu) ----
+constexpr int SPLIT_MAX_LISTS = 64;  // candidate lists a merge takes: ranks, or chunks of one rank
+constexpr int SPLIT_CHUNK_BLOCKS = 8192;  // blocks one CTA of the split scorer takes
+struct SplitParams {
+  CacheView c;                 // the rank's cache (page-table rows indexed by global logical page)
+  const __nv_bfloat16* idx_q;  // [rows][4][128] unrotated index queries
+  const float* w;              // [rows][4]
+  const int32_t* seq_len;      // [rows] context length including the query token
+  const int32_t* page_lo;      // [rows] first page this rank holds
+  const int32_t* page_cnt;     // [rows] pages this rank holds
+  int max_len;
+  RopeFreqs fr;
+  int nchunks;                 // chunks of 8192 blocks per row
+  uint32_t* cand_key;          // [rows][nchunks][512]
+  int32_t* cand_id;            // [rows][nchunks][512]
+  int32_t* cand_n;             // [rows][nchunks]
+  uint32_t* out_key;           // [rows][512] the rank's best 512 (key, block), block order
+  int32_t* out_id;             // [rows][512]
+  int32_t* out_n;              // [rows]
+  int* err;
+};
+cudaError_t launch_split_score(const SplitParams& p, int rows, cudaStream_t st);
+cudaError_t launch_split_merge(const uint32_t* keys, const int32_t* ids, const int32_t* n, int world, int rows,
+                               int32_t* blocks, int32_t* nblocks, cudaStream_t st);
+cudaError_t launch_split_positions(const SplitParams& p, const int32_t* blocks, const int32_t* nblocks, int rows,
+                                   int32_t* pos, int32_t* npos, cudaStream_t st);
+cudaError_t launch_split_combine(const __nv_bfloat16* outs, const float* lses, int world, int rows,
+                                 __nv_bfloat16* out, cudaStream_t st);
 
 // ev (nullable): n_ev event pairs recorded around the rotation, scoring and finalize kernels.
 cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,

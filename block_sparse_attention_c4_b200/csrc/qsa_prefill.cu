@@ -1,5 +1,6 @@
-// Prefill scorer on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
-// followed by an exact per-query top-512.
+// Prefill scoring of a causal chunk on the 5th-generation tensor cores
+// (tcgen05 + TMEM + TMA), with the exact per-query top-512 taken from a
+// filtered candidate list instead of from every score.
 //
 // Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
 // (SGLang day-0 blog for Qwen3.8-Flash-Next): in prefill a GPU kernel computes
@@ -15,25 +16,30 @@
 // heads (B, the rotated queries of one work tile, resident in shared memory),
 // accumulators double-buffered in TMEM (2 x 256 of the 512 columns).  Keys on
 // the M side put the 4 heads of one (block, query) pair in 4 adjacent TMEM
-// columns of one lane, so one thread combines them without shuffles.
+// columns of one lane, so one thread combines them without shuffles.  Warp
+// roles (one CTA per SM, persistent): warp 0 issues TMA, warp 1 owns TMEM and
+// issues the MMAs, 16 epilogue warps read the accumulators.  Work tiles are
+// ordered longest first (causal imbalance) and dealt to CTAs in a snake.
 //
-// Warp roles (one CTA per SM, persistent): warp 0 issues TMA, warp 1 owns TMEM
-// and issues the MMAs (one elected thread), the other warps are the epilogue:
-// each reads its 32-lane TMEM quadrant (32 blocks) for a group of queries,
-// combines the heads and writes the score of every visible (query, block) pair
-// as an order-preserving 32-bit key, 32 consecutive blocks of one query per
-// warp store (one 128-byte line).  Writing every score costs the same HBM
-// bytes as a filtered candidate list (key + block id) of the usual size, and
-// keeps the epilogue to a few instructions per score so that it hides under
-// the MMAs.  Work tiles are ordered longest first (causal imbalance) and dealt
-// to CTAs in a snake.
-//
-// Selection (k_prefill_select): one warp per query row, longest rows first:
-// a lower bound from a sample of the row's keys, one pass collecting the keys
-// at or above it, the exact cut among those (score desc, block asc), and the
-// kept blocks written in ascending order.  Rows that do not fit that path
-// (longer than 8192 blocks, heavy ties, a bound that keeps too few or too
-// many) go to k_prefill_select_overflow: an exact CTA-wide selection.
+// Scores never go to memory as a whole.  Per work tile the M-tiles run in two
+// phases:
+//   (1) sample: every 8th M-tile of the tile's visible range (a stratified
+//       sample, 1/8 of the blocks) fills, per query, a log-scale histogram of
+//       its score keys in shared memory (1/16 octave per bin, the range fixed
+//       per query by an upper bound of its scores from the rotation kernel).
+//       From it each query gets a threshold tau expected to pass about
+//       2 x 512 of its blocks;
+//   (2) main: every M-tile (the sampled ones again); a score key >= tau is
+//       written as a candidate (key << 32 | ~block, so a larger word ranks
+//       first under (score desc, block asc)) to the query's list for the TMEM
+//       quadrant of the block; each epilogue warp owns its lists' counters.
+// Exactness does not rest on the sample: if a query's candidates number at
+// least 512, its top-512 is among them (every block below tau has 512 blocks
+// at or above it, ties at tau included), and k_prefill_select takes the exact
+// cut among the candidates.  A query whose lists hold fewer than 512 or
+// overflowed (an unlucky sample, heavily tied scores) is re-scored in full by
+// k_prefill_rescore (mma.sync over its pages, exact radix top-k).  Queries
+// with at most PF_EMIT_ALL blocks skip the sample and emit every block.
 #include <mutex>
 
 #include "qsa_common.cuh"
@@ -44,29 +50,38 @@ namespace qsa {
 constexpr int PF_QT = 64;              // queries per work tile
 constexpr int PF_N = PF_QT * HI;       // 256 MMA columns
 constexpr int PF_M = 128;              // compressed keys per M-tile
-#ifndef QSA_PF_STAGES
-#define QSA_PF_STAGES 3
-#endif
-#ifndef QSA_PF_EPI_WARPS
-#define QSA_PF_EPI_WARPS 16
-#endif
-constexpr int PF_STAGES = QSA_PF_STAGES;       // A ring depth
-constexpr int PF_EPI_WARPS = QSA_PF_EPI_WARPS;  // 8 or 16
+constexpr int PF_STAGES = 3;           // A ring depth
+constexpr int PF_EPI_WARPS = 16;
 constexpr int PF_THREADS = (2 + PF_EPI_WARPS) * 32;
-constexpr int PF_QPW = PF_QT * 4 / PF_EPI_WARPS;  // queries per epilogue warp (32 or 16)
+constexpr int PF_QPW = PF_QT * 4 / PF_EPI_WARPS;  // queries per epilogue warp (16)
 constexpr int PF_A_BYTES = PF_M * D * 2;  // 32 KiB
 constexpr int PF_B_BYTES = PF_N * D * 2;  // 64 KiB
 constexpr uint32_t PF_TMEM_COLS = 512;
+constexpr int PF_PAGES = PF_M / PAGE_BLOCKS;  // 8 pages per M-tile
+constexpr int PF_SAMPLE = 8;              // one M-tile in PF_SAMPLE is scored first, as the sample
+constexpr float PF_SAMPLE_KEEP = 0.5f;    // tau passes about 512 / PF_SAMPLE_KEEP blocks
+constexpr int PF_BINS = 128;              // histogram bins per query: 8 octaves below the bound
+constexpr int PF_BIN_SHIFT = 19;          // key >> 19 = sign, exponent, 4 mantissa bits (1/16 octave)
+constexpr int PF_HIST_STRIDE = PF_BINS + 1;  // padded rows: conflict-free per-query scans
 static_assert(PF_EPI_WARPS % 4 == 0 && PF_QPW % 8 == 0, "epilogue warps cover the four TMEM quadrants evenly");
+static_assert(PF_QPW <= 32, "one lane per query of an epilogue warp holds its list counter");
 
 struct __align__(1024) PfSmem {
   uint8_t a[PF_STAGES][2][PF_A_BYTES / 2];  // [stage][K half][128 rows x 128 B], 128B-swizzled
   uint8_t b[2][PF_B_BYTES / 2];              // [K half][256 rows x 128 B]
-  float4 w[2][PF_QT];                        // halved head weights of the work tile's queries (by tile parity)
+  float4 w[PF_QT];                           // halved head weights of the work tile's queries
+  uint32_t hist[PF_QT * PF_HIST_STRIDE];     // sample histograms of the work tile's queries
+  float tau[PF_QT];                          // emission thresholds (scores; -inf: every block)
+  int32_t base[PF_QT];                       // histogram bases (bin 0 = key >> 19 at or below base)
   uint64_t full_a[PF_STAGES], empty_a[PF_STAGES], full_b, empty_b, tfull[2], tempty[2];
   uint32_t tmem_base;
   int abort;  // set by the first role whose wait gives up: every role then stops issuing work
 };
+
+// Histogram bin of a score key for a query whose bins start at `base` (monotone in the key).
+__device__ __forceinline__ int pf_bin(uint32_t key, int base) {
+  return min(PF_BINS - 1, max(0, (int)(key >> PF_BIN_SHIFT) - base));
+}
 
 // Wait of one role: bounded, and it stops as soon as any role of the CTA has given up, so that one
 // barrier that never completes ends the whole CTA instead of costing a full limit per later wait.
@@ -143,31 +158,82 @@ __host__ __device__ constexpr uint32_t pf_idesc() {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PF_N >> 3) << 17) | ((uint32_t)(PF_M >> 4) << 24);
 }
 
-// ---- work schedule: tiles longest first, dealt in a snake ----
-struct PfSched {
-  int ntiles, grid, pos0, T;
-  __device__ int tile_at(int k) const {  // k-th tile in descending cost order
-    return ntiles - 1 - k;
-  }
-  // j-th tile of CTA c, or -1
-  __device__ int nth(int c, int j) const {
-    const int k = j * grid + ((j & 1) ? (grid - 1 - c) : c);
-    return k < ntiles ? tile_at(k) : -1;
-  }
+
+// ---- work schedule: tiles longest first, dealt in a snake; per tile the sample M-tiles first ----
+// A work tile: 64 consecutive queries of one segment.  Local query index t (0 .. T-1 within the
+// segment), global row q_off + t of the call's arrays.
+struct PfTile {
+  int req, pos0, T, q_off, qt;
   __device__ int nbv_of(int t) const { return (pos0 + t + 1) >> 2; }
-  __device__ int mtiles(int qt) const {  // M-tiles of a work tile (0: every query keeps all its blocks)
-    const int tl = min(T, (qt + 1) * PF_QT) - 1;
-    const int nb = nbv_of(tl);
+  __device__ int nbv_hi() const { return nbv_of(min(T, (qt + 1) * PF_QT) - 1); }
+  // M-tiles of the main phase (0: every query keeps all its blocks, nothing to score)
+  __device__ int mtiles() const {
+    const int nb = nbv_hi();
     return nb <= TOPK ? 0 : ceil_div(nb, PF_M);
+  }
+  // M-tiles of the sample phase (0: every query of the tile emits all its blocks)
+  __device__ int stiles() const {
+    const int nb = nbv_hi();
+    return nb <= PF_EMIT_ALL ? 0 : ceil_div(ceil_div(nb, PF_M), PF_SAMPLE);
   }
 };
 
+// M-tile of step k of a tile with ns sample steps
+__device__ __forceinline__ int pf_mt_of(int k, int ns) { return k < ns ? k * PF_SAMPLE : k - ns; }
+
+// The k-th tile in schedule order: segments in their listed order, each segment's tiles from its last
+// (longest context) down.
+__device__ __forceinline__ PfTile pf_tile(const PrefillParams& p, int k) {
+  int lo = 0, hi = p.nseg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seg[mid].tile_off <= k) lo = mid;
+    else hi = mid - 1;
+  }
+  const PfSeg& s = p.seg[lo];
+  return PfTile{s.req, s.pos0, s.T, s.q_off, ceil_div(s.T, PF_QT) - 1 - (k - s.tile_off)};
+}
+
+// j-th tile of CTA c, dealt in a snake over the schedule, or false
+__device__ __forceinline__ bool pf_nth(const PrefillParams& p, int c, int j, PfTile& tile) {
+  const int grid = (int)gridDim.x;
+  const int k = j * grid + ((j & 1) ? (grid - 1 - c) : c);
+  if (k >= p.ntiles) return false;
+  tile = pf_tile(p, k);
+  return true;
+}
+
+// Segment holding global row g (rows of one warp or CTA share it: uniform lookups).
+__device__ __forceinline__ const PfSeg& pf_seg_of_row(const PrefillParams& p, int g) {
+  int s = 0;
+  while (s + 1 < p.nseg && (unsigned)(g - p.seg[s].q_off) >= (unsigned)p.seg[s].T) ++s;
+  return p.seg[s];
+}
+
+// Emission threshold of one query from its sample histogram: the lower edge of the highest bin at
+// which the sample holds R keys, R = (512 / PF_SAMPLE_KEEP) x (sampled blocks / visible blocks), so
+// that about 512 / PF_SAMPLE_KEEP of the query's blocks pass.  0 (emit every
+// visible block) for queries with few blocks, no histogram range, or too small a sample.
+__device__ __forceinline__ uint32_t pf_threshold(const uint32_t* hist_row, int base, int nbv, int ns) {
+  if (nbv <= PF_EMIT_ALL || base == PF_NO_BASE) return 0u;
+  int ns_q = 0;
+  for (int i = 0; i < ns; ++i) ns_q += min(PF_M, max(0, nbv - i * PF_SAMPLE * PF_M));
+  const int R = max(1, (int)((float)TOPK / PF_SAMPLE_KEEP * (float)ns_q / (float)nbv));
+  int acc = 0;
+  for (int b = PF_BINS - 1; b > 0; --b) {
+    acc += (int)hist_row[b];
+    if (acc >= R) return base + b > 0 ? (uint32_t)(base + b) << PF_BIN_SHIFT : 0u;
+  }
+  return 0u;
+}
+
+// 576 threads (18 warps), one CTA per SM: two of the SM's four register-file quarters hold five warps,
+// so the kernel gets at most 96 registers per thread
 __global__ void __launch_bounds__(PF_THREADS, 1)
     k_prefill_score(PrefillParams p, const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap) {
   extern __shared__ uint8_t smem_raw[];
   PfSmem& S = *reinterpret_cast<PfSmem*>(smem_aligned<1024>(smem_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  PfSched sch{ceil_div(p.T, PF_QT), (int)gridDim.x, p.pos0, p.T};
   const uint64_t lim = p.wait_ns ? p.wait_ns : WAIT_LIMIT_NS;
   volatile int* abort = &S.abort;
 
@@ -197,18 +263,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
   if (warp == 0) {
     // =============================== TMA producer ===============================
-    // The whole warp walks the schedule: lane i fetches the physical page of
-    // logical page 32g + i for the group g of four M-tiles (32 pages) ahead of
-    // use, so no page-table load sits on the path of a copy; lane 0 waits for
-    // the stage and expects its bytes, then 16 lanes issue one copy each.
+    // Lane i < 8 looks up the physical page of page i of the next step's M-tile one step ahead, so
+    // no page-table load sits on the path of a copy; lane 0 waits for the stage and expects its
+    // bytes, then 16 lanes issue one copy each (a 64-dim half of one page of 16 keys).
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&qmap);
     }
-    const int32_t* pt = p.c.page_table + (int64_t)p.req * p.c.max_pages;
     const int oob_row = (int)(p.c.num_pages * PAGE_BLOCKS);  // a row past the cache: TMA fills zeros
-    constexpr int GROUP = 32 / (PF_M / PAGE_BLOCKS);         // M-tiles per page group (4)
-    auto page_row = [&](int lp, int nbv_hi) {                // lane's page -> first cache row
+    const int32_t* pt = p.c.page_table;
+    auto page_row = [&](int lp, int nbv_hi) {                // logical page of the tile's request -> first cache row
       int row = oob_row;
       if (lp < p.c.max_pages) {
         const int phys = __ldg(pt + lp);
@@ -219,27 +283,29 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     };
     int a_it = 0, wt = 0;
     bool ok = true;
-    for (int j = 0; ok; ++j) {
-      const int qt = sch.nth(blockIdx.x, j);
-      if (qt < 0) break;
-      const int nm = sch.mtiles(qt);
+    PfTile tl;
+    for (int j = 0; ok && pf_nth(p, blockIdx.x, j, tl); ++j) {
+      const int nm = tl.mtiles();
       if (nm == 0) continue;
-      const int nbv_hi = sch.nbv_of(min(p.T, (qt + 1) * PF_QT) - 1);
+      const int ns = tl.stiles(), nk = ns + nm;
+      const int nbv_hi = tl.nbv_hi();
+      pt = p.c.page_table + (int64_t)tl.req * p.c.max_pages;
       int go = 1;
       if (lane == 0) {
         go = wt == 0 || pf_wait(&S.empty_b, (wt - 1) & 1, p.err, lim, abort);
-        if (go) {
+        if (go) {  // the tile's 64 queries x 4 heads of rotated index queries (rows past the call's end: zeros)
+          const int qrow = (tl.q_off + tl.qt * PF_QT) * HI;
           mbar_arrive_expect_tx(&S.full_b, PF_B_BYTES);
-          tma_load_2d(S.b[0], &qmap, 0, qt * PF_N, &S.full_b);
-          tma_load_2d(S.b[1], &qmap, 64, qt * PF_N, &S.full_b);
+          tma_load_2d(S.b[0], &qmap, 0, qrow, &S.full_b);
+          tma_load_2d(S.b[1], &qmap, 64, qrow, &S.full_b);
         }
       }
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
       ++wt;
-      int rows_cur = page_row(lane, nbv_hi), rows_nxt = oob_row;
-      for (int mt = 0; mt < nm; ++mt, ++a_it) {
-        const int g = mt / GROUP, r = mt % GROUP;
-        if (r == 0 && (g + 1) * GROUP < nm) rows_nxt = page_row((g + 1) * 32 + lane, nbv_hi);
+      int rows_cur = lane < PF_PAGES ? page_row(pf_mt_of(0, ns) * PF_PAGES + lane, nbv_hi) : oob_row;
+      for (int k = 0; k < nk; ++k, ++a_it) {
+        const int rows_nxt =
+            (k + 1 < nk && lane < PF_PAGES) ? page_row(pf_mt_of(k + 1, ns) * PF_PAGES + lane, nbv_hi) : oob_row;
         const int s = a_it % PF_STAGES;
         if (lane == 0) {
           go = a_it < PF_STAGES || pf_wait(&S.empty_a[s], ((a_it / PF_STAGES) - 1) & 1, p.err, lim, abort);
@@ -250,14 +316,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           ok = false;
           break;
         }
-        // 16 lanes issue the M-tile's 16 copies at once: lane 2*pg + half copies the 64-dim half
-        // `half` of page pg (16 keys)
-        constexpr int PAGES = PF_M / PAGE_BLOCKS;  // 8 pages per M-tile
-        const int pg = (lane >> 1) & (PAGES - 1), half = lane & 1;
-        const int row = __shfl_sync(0xffffffffu, rows_cur, r * PAGES + pg);
-        if (lane < 2 * PAGES)
+        const int pg = (lane >> 1) & (PF_PAGES - 1), half = lane & 1;
+        const int row = __shfl_sync(0xffffffffu, rows_cur, pg);
+        if (lane < 2 * PF_PAGES)
           tma_load_2d(S.a[s][half] + pg * PAGE_BLOCKS * 128, &kmap, half * 64, row, &S.full_a[s]);
-        if (r == GROUP - 1) rows_cur = rows_nxt;
+        rows_cur = rows_nxt;
       }
     }
     // drain: every copy issued above has landed before the CTA may exit (in the normal case these
@@ -275,14 +338,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       const uint32_t idesc = pf_idesc();
       int a_it = 0, m_it = 0, wt = 0, b_commits = 0;
       bool ok = true;
-      for (int j = 0; ok; ++j) {
-        const int qt = sch.nth(blockIdx.x, j);
-        if (qt < 0) break;
-        const int nm = sch.mtiles(qt);
+      PfTile tl;
+      for (int j = 0; ok && pf_nth(p, blockIdx.x, j, tl); ++j) {
+        const int nm = tl.mtiles();
         if (nm == 0) continue;
+        const int nk = tl.stiles() + nm;
         if (!pf_wait(&S.full_b, wt & 1, p.err, lim, abort)) break;
         ++wt;
-        for (int mt = 0; mt < nm; ++mt, ++a_it, ++m_it) {
+        for (int k = 0; k < nk; ++k, ++a_it, ++m_it) {
           const int s = a_it % PF_STAGES;
           const int buf = m_it & 1;
           if (!pf_wait(&S.full_a[s], (a_it / PF_STAGES) & 1, p.err, lim, abort) ||
@@ -314,70 +377,116 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
   } else {
     // =============================== epilogue ===============================
+    // Thread = one block of the M-tile (TMEM lane 32*quad + lane), registers = the 4 heads of the
+    // warp's 16 queries.  Lane jl < 16 of a warp keeps the candidate count of query jl's list for
+    // the warp's quadrant, so a list is never shared between warps.
     const int e = warp - 2;           // 0 .. PF_EPI_WARPS-1
     const int quad = warp & 3;        // TMEM lanes 32*quad .. +31 = blocks of the M-tile
     const int qg = e >> 2;            // query group: queries qg*PF_QPW .. +PF_QPW-1 of the tile
     const int etid = tid - 64;        // 0 .. 32*PF_EPI_WARPS-1
-    const int nmax = p.cap / PF_M;    // M-tile slots per work tile in the score array
-    int m_it = 0, wt = 0;
-    for (int j = 0;; ++j) {
-      const int qt = sch.nth(blockIdx.x, j);
-      if (qt < 0) break;
-      const int nm = sch.mtiles(qt);
+    const uint32_t lt = (1u << lane) - 1u;
+    int m_it = 0;
+    PfTile tl;
+    for (int j = 0; pf_nth(p, blockIdx.x, j, tl); ++j) {
+      const int nm = tl.mtiles();
       if (nm == 0) continue;
-      const int par = wt & 1;
-      ++wt;
-      // this tile's head weights, halved (see below); the other parity's copy
-      // may still be read by warps finishing the previous tile, so a barrier
-      // is needed only after writing
-      if (etid < PF_QT) {
-        const int t = qt * PF_QT + etid;
-        float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < p.T) w4 = __ldg(reinterpret_cast<const float4*>(p.w) + t);
-        S.w[par][etid] = make_float4(0.5f * w4.x, 0.5f * w4.y, 0.5f * w4.z, 0.5f * w4.w);
-      }
+      const int ns = tl.stiles(), nk = ns + nm;
+      // every epilogue warp is done with the previous tile's shared state before it is replaced
       asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
-      const float4* wq = &S.w[par][qg * PF_QPW];
-      // score-key tile (qt, mt): [64 queries][128 blocks]; this thread writes column quad*32+lane
-      uint32_t* col = p.keys + (int64_t)qt * nmax * (PF_QT * PF_M) + qg * PF_QPW * PF_M + quad * 32 + lane;
+      if (etid < PF_QT) {
+        const int t = tl.qt * PF_QT + etid;
+        float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        int bs = PF_NO_BASE;
+        if (t < tl.T) {
+          w4 = __ldg(reinterpret_cast<const float4*>(p.w) + tl.q_off + t);
+          bs = __ldg(p.qbase + tl.q_off + t);
+        }
+        S.w[etid] = make_float4(0.5f * w4.x, 0.5f * w4.y, 0.5f * w4.z, 0.5f * w4.w);
+        S.base[etid] = bs;
+        S.tau[etid] = -INFINITY;
+      }
+      if (ns > 0)
+        for (int i = etid; i < PF_QT * PF_HIST_STRIDE; i += PF_EPI_WARPS * 32) S.hist[i] = 0u;
+      asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
+      const int q0 = qg * PF_QPW;          // first query of this warp's group, in the tile
+      const int t0 = tl.qt * PF_QT + q0;   // ... in the segment
+      int cnt = 0;                         // lane jl < PF_QPW: candidates of query q0 + jl, this quadrant
 
-      for (int mt = 0; mt < nm; ++mt, ++m_it) {
+      for (int k = 0; k < nk; ++k, ++m_it) {
+        const int mt = pf_mt_of(k, ns);
         const int buf = m_it & 1;
-        // after a timeout anywhere in the CTA the loops still run to their end (no work, no waits), so
+        // after a timeout anywhere in the CTA the loop still runs to its end (no work, no waits), so
         // that every epilogue warp meets the same named barriers
-        if (!pf_wait(&S.tfull[buf], (m_it >> 1) & 1, p.err, lim, abort)) continue;
-        tc_fence_after();
-        uint32_t r[PF_QPW / 8][32];
-        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * PF_N + qg * PF_QPW * 4);
+        if (pf_wait(&S.tfull[buf], (m_it >> 1) & 1, p.err, lim, abort)) {
+          tc_fence_after();
+          const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * PF_N + q0 * 4);
+          const int b = mt * PF_M + quad * 32 + lane;  // this thread's block
+          // which of the warp's 16 queries see this thread's block (all of them except in a tile's last
+          // M-tiles), as a mask computed once per M-tile
+          uint32_t vmask = 0xFFFFu;
+          if (!((mt + 1) * PF_M <= tl.nbv_of(t0) && t0 + PF_QPW <= tl.T)) {
+            vmask = 0u;
 #pragma unroll
-        for (int g = 0; g < PF_QPW / 8; ++g) tc_ld32(taddr + 32u * g, r[g]);
-        tc_wait_ld();
+            for (int jl = 0; jl < PF_QPW; ++jl)
+              vmask |= (t0 + jl < tl.T && b < tl.nbv_of(t0 + jl)) ? (1u << jl) : 0u;
+          }
+          // the 16 queries' 4 heads in two loads of 8 queries (32 columns each); the TMEM buffer goes back
+          // to the MMA warp once both are in registers
 #pragma unroll
-        for (int g = 0; g < PF_QPW / 8; ++g) tc_after_wait(r[g]);
-        // the accumulators are in registers: hand the TMEM buffer back at once
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.tempty[buf]);
-
-        // w * max(x, 0) == (w/2) * (x + |x|) exactly (doubling and halving are
-        // exact), which keeps the ReLU on the FMA pipe.  Every column of the
-        // tile is written: the blocks past a query's visible range are never
-        // read back.
-        uint32_t* out = col + (int64_t)mt * (PF_QT * PF_M);
+          for (int half = 0; half < PF_QPW / 8; ++half) {
+            uint32_t r[32];
+            tc_ld32(taddr + 32u * half, r);
+            tc_wait_ld();
+            tc_after_wait(r);
+            if (half == PF_QPW / 8 - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&S.tempty[buf]);
+            }
 #pragma unroll
-        for (int jl = 0; jl < PF_QPW; ++jl) {
-          const float4 w4 = wq[jl];
-          const uint32_t* rr = &r[jl >> 3][4 * (jl & 7)];
-          const float x0 = __uint_as_float(rr[0]), x1 = __uint_as_float(rr[1]);
-          const float x2 = __uint_as_float(rr[2]), x3 = __uint_as_float(rr[3]);
-          float sc = fmaf(w4.x, x0 + fabsf(x0), 0.f);
-          sc = fmaf(w4.y, x1 + fabsf(x1), sc);
-          sc = fmaf(w4.z, x2 + fabsf(x2), sc);
-          sc = fmaf(w4.w, x3 + fabsf(x3), sc) + 0.f;  // + 0: an underflowed -0 becomes +0
-          const uint32_t u = __float_as_uint(sc);
-          out[jl * PF_M] = u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);  // order-preserving key
+            for (int jj = 0; jj < 8; ++jj) {
+              const int jl = half * 8 + jj;
+              // w * max(x, 0) == (w/2) * (x + |x|) exactly (doubling and halving are exact), which keeps
+              // the ReLU on the FMA pipe; + 0 turns an underflowed -0 into +0
+              const float4 w4 = S.w[q0 + jl];
+              const float x0 = __uint_as_float(r[4 * jj]), x1 = __uint_as_float(r[4 * jj + 1]);
+              const float x2 = __uint_as_float(r[4 * jj + 2]), x3 = __uint_as_float(r[4 * jj + 3]);
+              float sc = fmaf(w4.x, x0 + fabsf(x0), 0.f);
+              sc = fmaf(w4.y, x1 + fabsf(x1), sc);
+              sc = fmaf(w4.z, x2 + fabsf(x2), sc);
+              sc = fmaf(w4.w, x3 + fabsf(x3), sc) + 0.f;
+              const uint32_t u = __float_as_uint(sc);
+              const uint32_t key = u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);  // order-preserving
+              if (k < ns) {
+                if ((vmask >> jl) & 1u)
+                  atomicAdd(&S.hist[(q0 + jl) * PF_HIST_STRIDE + pf_bin(key, S.base[q0 + jl])], 1u);
+              } else {
+                const bool emit = sc >= S.tau[q0 + jl] && ((vmask >> jl) & 1u);
+                const unsigned m = __ballot_sync(0xffffffffu, emit);
+                if (m) {  // warp-uniform
+                  const int c = __shfl_sync(0xffffffffu, cnt, jl);
+                  const int slot = c + __popc(m & lt);
+                  if (emit && slot < PF_QCAP)
+                    p.cand[((int64_t)(tl.q_off + t0 + jl) * 4 + quad) * PF_QCAP + slot] =
+                        ((unsigned long long)key << 32) | (uint32_t)~(uint32_t)b;
+                  if (lane == jl) cnt += __popc(m);
+                }
+              }
+            }
+          }
+        }
+        if (k == ns - 1) {  // the sample is complete: each query's threshold
+          asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
+          if (etid < PF_QT) {
+            const int t = tl.qt * PF_QT + etid;
+            const uint32_t tk =
+                t < tl.T ? pf_threshold(S.hist + etid * PF_HIST_STRIDE, S.base[etid], tl.nbv_of(t), ns) : 0u;
+            S.tau[etid] = tk == 0u ? -INFINITY : key_score(tk);
+          }
+          asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
         }
       }
+      if (lane < PF_QPW && t0 + lane < tl.T) p.cand_n[(int64_t)(tl.q_off + t0 + lane) * 4 + quad] = cnt;
     }
   }
   tc_fence_before();
@@ -389,115 +498,41 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Selection: one warp per query row, longest rows first.  Row t's keys are the
-// 128-key chunks (t & 63) of its work tile's M-tiles, 32 KiB apart; a chunk is
-// one 16-byte load per lane (lane l: blocks 4l .. 4l+3).
-//
-// (1) A bound L below the cut: rows of at most PW_ALL_N blocks take L = 0.
-//     Longer rows sample every 8th chunk; L is the smallest sample key in
-//     the bin (256 bins linear in the score) that holds the sample's R-th
-//     largest key, R set for about 1.5 x 512 row keys at or above L.
-// (2) One streaming pass appends every key >= L (with its block) to
-//     lane-private lists; a lane keeps its blocks in ascending order.
-// (3) The exact cut (key T, block I of the 512th element in (key desc, block
-//     asc) order) is found on the lists: a histogram of the list's scores
-//     (256 linear bins) gives the bin holding the cut, and that bin's few keys are
-//     ranked among themselves.
-// (4) The kept list entries set their bits in a block bitmap, which is
-//     written out in ascending order.
-// A row that does not fit (a lane list overflows, fewer than 512 keys reach
-// L, heavily tied keys, or a row longer than PW_FAST_N) goes to the overflow
-// list, which k_prefill_select_overflow resolves with a CTA-wide exact
-// selection.
+// Selection from the candidates: one warp per query row, longest rows first.
+// (1) a histogram of the candidates' bins (the scorer's log-scale bins of the
+//     query) gives the bin D holding the 512th candidate;
+// (2) one pass marks the blocks of every candidate above bin D in a block
+//     bitmap and gathers bin D's candidates;
+// (3) bin D's candidates are ranked by their whole word (key, then lower
+//     block first; words are distinct), the best `need` marked;
+// (4) the bitmap is written out in ascending block order.
+// Rows with fewer than 512 candidates, an overflowed list, or more ties in
+// bin D than the warp holds go to the re-scoring list.
 // ----------------------------------------------------------------------------
-#ifndef QSA_PW_WARPS
-#define QSA_PW_WARPS 4
-#endif
-#ifndef QSA_PW_UNROLL
-#define QSA_PW_UNROLL 8
-#endif
-constexpr int PW_WARPS = QSA_PW_WARPS;    // rows in flight per CTA
-constexpr int PW_UNROLL = QSA_PW_UNROLL;  // chunks loaded back to back
-constexpr int PW_LIST = 48;               // list entries per lane
-constexpr int PW_FAST_N = 8192;           // longer rows take the CTA-wide path
-constexpr int PW_ALL_N = PW_LIST * 32;    // rows this short keep every key as a candidate
-constexpr int PW_SAMPLE = 8;              // sample chunks at most (every 8th of <= 64)
-constexpr int PW_BINS = 256;
-constexpr int PW_L3 = 64;
+constexpr int PS_MAX_WARPS = 8;
+constexpr int PS_TIE_CAP = 256;
 
-struct __align__(16) PwWarp {
-  uint32_t lkey[(PW_LIST + 1) * 32];  // [slot][lane]; slot PW_LIST is a spare for writes past a full list
-  uint16_t lidx[(PW_LIST + 1) * 32];
-  uint32_t hist[PW_BINS];
-  uint32_t bitmap[PW_FAST_N / 32];
-  uint32_t k3[PW_L3];
-  int i3[PW_L3];
-};
-
-// Bin D of hist[0..256) counted from the top: count(> D) < k <= count(>= D);
-// `above` = count(> D).  Returns false when the histogram holds fewer than k.
-__device__ __forceinline__ bool pw_top_bin(const uint32_t* hist, int k, int& D, int& above) {
-  const int lane = threadIdx.x & 31;
-  const int lo = PW_BINS - 8 * (lane + 1);
-  const uint4 h0 = *reinterpret_cast<const uint4*>(hist + lo);
-  const uint4 h1 = *reinterpret_cast<const uint4*>(hist + lo + 4);
-  const int local = (int)(h0.x + h0.y + h0.z + h0.w + h1.x + h1.y + h1.z + h1.w);
-  int x = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  const uint32_t hit = __ballot_sync(0xffffffffu, x - local < k && x >= k);
-  if (!hit) return false;
-  const int L = __ffs(hit) - 1;
-  int c = __shfl_sync(0xffffffffu, x - local, L);
-  const int topL = PW_BINS - 1 - 8 * L;
-  int d = topL - 7;
-  for (int i = 0; i < 8; ++i) {
-    const int h = (int)hist[topL - i];
-    if (c + h >= k) {
-      d = topL - i;
-      break;
-    }
-    c += h;
-  }
-  D = d;
-  above = c;
-  return true;
+__host__ __device__ constexpr int ps_warp_bytes(int bm_words) {
+  return PF_BINS * 4 + PS_TIE_CAP * 8 + ((bm_words + 3) / 4) * 16;
 }
 
-// Bins linear in the score between the scores of keys kmin and kmax.
-// Monotone in the key: decoding, subtraction, scaling by a positive factor
-// and truncation all preserve order.
-struct PwBins {
-  float smin, scale;
-  __device__ int operator()(uint32_t k) const { return min(PW_BINS - 1, (int)((key_score(k) - smin) * scale)); }
-};
-
-__device__ __forceinline__ PwBins pw_bins(uint32_t kmin, uint32_t kmax) {
-  PwBins b;
-  b.smin = key_score(kmin);
-  const float span = key_score(kmax) - b.smin;
-  b.scale = span > 0.f && span < 3.0e38f ? (float)PW_BINS / (span * 1.0001f) : 0.f;
-  return b;
-}
-
-__device__ __forceinline__ void pw_zero(uint32_t* a, int words) {  // words: a multiple of 4
-  const int lane = threadIdx.x & 31;
-  for (int i = lane; i < words / 4; i += 32) reinterpret_cast<uint4*>(a)[i] = make_uint4(0u, 0u, 0u, 0u);
-}
-
-__global__ void __launch_bounds__(PW_WARPS * 32) k_prefill_select(PrefillParams p) {
-  extern __shared__ uint8_t pw_raw[];
+__global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillParams p, int bm_words) {
+  extern __shared__ __align__(16) uint8_t ps_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  PwWarp& W = reinterpret_cast<PwWarp*>(pw_raw)[warp];
-  const int nmax = p.cap / PF_M;
+  uint8_t* mine = ps_raw + warp * ps_warp_bytes(bm_words);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(mine);
+  unsigned long long* tie = reinterpret_cast<unsigned long long*>(mine + PF_BINS * 4);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(mine + PF_BINS * 4 + PS_TIE_CAP * 8);
   const uint32_t lt = (1u << lane) - 1u;
-  const int gw = blockIdx.x * PW_WARPS + warp, nw = gridDim.x * PW_WARPS;
+  const int wpb = blockDim.x >> 5;
+  const int gw = blockIdx.x * wpb + warp, nw = gridDim.x * wpb;
   for (int k = gw; k < p.T; k += nw) {
-    const int t = p.T - 1 - k;
-    const int n = (p.pos0 + t + 1) >> 2;
+    // k-th row in schedule order: segments in listed order, each from its last (longest) row down
+    int si = 0;
+    while (si + 1 < p.nseg && p.seg[si + 1].row_off <= k) ++si;
+    const PfSeg& sg = p.seg[si];
+    const int t = sg.q_off + (sg.T - 1 - (k - sg.row_off));  // global row
+    const int n = (sg.pos0 + (t - sg.q_off) + 1) >> 2;
     int32_t* sel = p.sel + (int64_t)t * TOPK;
     __syncwarp();  // the previous row's shared data is no longer read
     if (n <= TOPK) {
@@ -505,217 +540,176 @@ __global__ void __launch_bounds__(PW_WARPS * 32) k_prefill_select(PrefillParams 
       if (lane == 0) p.sel_n[t] = n;
       continue;
     }
-    bool overflow = n > PW_FAST_N;
-    if (!overflow) {
-      const uint32_t* row = p.keys + ((int64_t)(t >> 6) * nmax * PF_QT + (t & 63)) * PF_M + 4 * lane;
-      auto chunk = [&](int c) { return __ldcg(reinterpret_cast<const uint4*>(row + (int64_t)c * (PF_QT * PF_M))); };
-      const int nch = ceil_div(n, PF_M);
-      // ---- (1) the bound L ----
-      uint32_t L = 0u;
-      if (n > PW_ALL_N) {
-        const int ns_ch = max(2, nch / 8);
-        uint32_t sk[PW_SAMPLE][4];
-        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    const int cl = lane < 4 ? p.cand_n[(int64_t)t * 4 + lane] : 0;
+    const int total = __reduce_add_sync(0xffffffffu, (unsigned)cl);
+    bool rescore = __reduce_max_sync(0xffffffffu, (unsigned)cl) > (unsigned)PF_QCAP || total < TOPK;
+    if (!rescore) {
+      const int base = p.qbase[t];
+      const unsigned long long* lists = p.cand + (int64_t)t * 4 * PF_QCAP;
+      // ---- (1) histogram ----
+      for (int i = lane; i < PF_BINS; i += 32) hist[i] = 0u;
+      __syncwarp();
+      for (int q = 0; q < 4; ++q) {
+        const int cn = __shfl_sync(0xffffffffu, cl, q);
+        for (int i = lane; i < cn; i += 32)
+          atomicAdd(&hist[pf_bin((uint32_t)(__ldcg(lists + q * PF_QCAP + i) >> 32), base)], 1u);
+      }
+      __syncwarp();
+      // bin D from the top: count(> D) < 512 <= count(>= D); lane l owns bins 127-4l .. 124-4l
+      const uint4 h4 = reinterpret_cast<const uint4*>(hist)[PF_BINS / 4 - 1 - lane];
+      const int local = (int)(h4.x + h4.y + h4.z + h4.w);
+      int x = local;
 #pragma unroll
-        for (int i = 0; i < PW_SAMPLE; ++i) {
-          const int c = (i * nch) / ns_ch;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (i < ns_ch) v = chunk(c);
-          const uint32_t kk[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const bool valid = i < ns_ch && c * PF_M + 4 * lane + e < n;
-            sk[i][e] = kk[e];
-            if (valid) {
-              mn = min(mn, kk[e]);
-              mx = max(mx, kk[e]);
-            }
-          }
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const uint32_t hit = __ballot_sync(0xffffffffu, x - local < TOPK && x >= TOPK);
+      const int L = __ffs(hit) - 1;  // total >= 512, so some lane holds the crossing
+      int above = __shfl_sync(0xffffffffu, x - local, L);
+      const int topL = PF_BINS - 1 - 4 * L;
+      int D = topL - 3;
+      for (int i = 0; i < 4; ++i) {
+        const int h = (int)hist[topL - i];
+        if (above + h >= TOPK) {
+          D = topL - i;
+          break;
         }
-        mn = __reduce_min_sync(0xffffffffu, mn);
-        mx = __reduce_max_sync(0xffffffffu, mx);
-        const PwBins bin = pw_bins(mn, mx);
-        pw_zero(W.hist, PW_BINS);
-        __syncwarp();
-        int ns = 0;
-#pragma unroll
-        for (int i = 0; i < PW_SAMPLE; ++i) {
-          const int c = (i * nch) / ns_ch;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (i < ns_ch && c * PF_M + 4 * lane + e < n) {
-              atomicAdd(&W.hist[bin(sk[i][e])], 1u);
-              ++ns;
-            }
+        above += h;
+      }
+      const int need = TOPK - above;  // taken from bin D, >= 1
+      // ---- (2) bitmap of the blocks above bin D; bin D gathered ----
+      const int words = (n + 31) >> 5;
+      for (int i = lane; i < words; i += 32) bitmap[i] = 0u;
+      __syncwarp();
+      int nt = 0;
+      for (int q = 0; q < 4; ++q) {
+        const int cn = __shfl_sync(0xffffffffu, cl, q);
+        for (int i0 = 0; i0 < cn; i0 += 32) {
+          const int i = i0 + lane;
+          unsigned long long e = 0ull;
+          int bn = -1;
+          if (i < cn) {
+            e = __ldcg(lists + q * PF_QCAP + i);
+            bn = pf_bin((uint32_t)(e >> 32), base);
           }
-        }
-        ns = __reduce_add_sync(0xffffffffu, ns);
-        __syncwarp();
-        const int R = min(ns, (3 * TOPK / 2 * ns) / n + 8);
-        int Ds = 0, as = 0;
-        if (pw_top_bin(W.hist, R, Ds, as)) {
-          uint32_t lm = 0xFFFFFFFFu;
-#pragma unroll
-          for (int i = 0; i < PW_SAMPLE; ++i) {
-            const int c = (i * nch) / ns_ch;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (i < ns_ch && c * PF_M + 4 * lane + e < n && bin(sk[i][e]) >= Ds) lm = min(lm, sk[i][e]);
+          if (bn > D) {
+            const uint32_t blk = ~(uint32_t)e;
+            atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
           }
-          L = __reduce_min_sync(0xffffffffu, lm);
+          const unsigned tm = __ballot_sync(0xffffffffu, bn == D);
+          if (bn == D) {
+            const int slot = nt + __popc(tm & lt);
+            if (slot < PS_TIE_CAP) tie[slot] = e;
+          }
+          nt += __popc(tm);
         }
       }
-      // ---- (2) candidates: every key >= L ----
-      int lc = 0;
-      const int nfull = n / PF_M;
-      for (int c0 = 0; c0 < nch; c0 += PW_UNROLL) {
-        uint4 v[PW_UNROLL];
-#pragma unroll
-        for (int u = 0; u < PW_UNROLL; ++u)
-          if (c0 + u < nch) v[u] = chunk(c0 + u);
-#pragma unroll
-        for (int u = 0; u < PW_UNROLL; ++u) {
-          const int c = c0 + u;
-          if (c >= nch) break;
-          const int b0 = c * PF_M + 4 * lane;
-          const uint32_t kk[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-          // branch-free: every key is written to the lane's next slot, which advances only for a
-          // key >= L; past a full list the writes go to a spare slot (the row then overflows)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int slot = min(lc, PW_LIST) * 32 + lane;
-            W.lkey[slot] = kk[e];
-            W.lidx[slot] = (uint16_t)(b0 + e);
-            lc += (kk[e] >= L && (c < nfull || b0 + e < n)) ? 1 : 0;
+      __syncwarp();
+      rescore = nt > PS_TIE_CAP || need > nt;
+      if (!rescore) {
+        // ---- (3) the best `need` of bin D ----
+        for (int j = lane; j < nt; j += 32) {
+          const unsigned long long ej = tie[j];
+          int rank = 0;
+          for (int m = 0; m < nt; ++m) rank += tie[m] > ej;
+          if (rank < need) {
+            const uint32_t blk = ~(uint32_t)ej;
+            atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
           }
         }
-      }
-      const int ln = __reduce_add_sync(0xffffffffu, (unsigned)lc);
-      overflow = __any_sync(0xffffffffu, lc > PW_LIST) || ln < TOPK;
-      if (!overflow) {
         __syncwarp();
-        // ---- (3) the cut ----
-        uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-        for (int j = 0; j < lc; ++j) {
-          const uint32_t kk = W.lkey[j * 32 + lane];
-          mn = min(mn, kk);
-          mx = max(mx, kk);
-        }
-        mn = __reduce_min_sync(0xffffffffu, mn);
-        mx = __reduce_max_sync(0xffffffffu, mx);
-        const PwBins bin = pw_bins(mn, mx);
-        pw_zero(W.hist, PW_BINS);
-        __syncwarp();
-        for (int j = 0; j < lc; ++j) atomicAdd(&W.hist[bin(W.lkey[j * 32 + lane])], 1u);
-        __syncwarp();
-        int D = 0, above = 0;
-        bool ok = pw_top_bin(W.hist, TOPK, D, above);
-        const int need = TOPK - above;
-        int n3 = 0;
-        const int lmax = __reduce_max_sync(0xffffffffu, (unsigned)lc);
-        for (int j = 0; j < lmax; ++j) {
-          const bool have = j < lc;
-          const uint32_t kk = have ? W.lkey[j * 32 + lane] : 0u;
-          const bool in = have && bin(kk) == D;
-          const uint32_t mm = __ballot_sync(0xffffffffu, in);
-          const int slot = n3 + __popc(mm & lt);
-          if (in && slot < PW_L3) {
-            W.k3[slot] = kk;
-            W.i3[slot] = W.lidx[j * 32 + lane];
-          }
-          n3 += __popc(mm);
-        }
-        __syncwarp();
-        overflow = !ok || n3 > PW_L3 || need < 1 || need > n3;
-        if (!overflow) {
-          uint32_t T = 0u;
-          int I = -1;
-          for (int j0 = 0; j0 < n3; j0 += 32) {
-            const int j = j0 + lane;
-            bool hit = false;
-            uint32_t kj = 0u;
-            int ij = 0;
-            if (j < n3) {
-              kj = W.k3[j];
-              ij = W.i3[j];
-              int rank = 0;
-              for (int q = 0; q < n3; ++q) {
-                const uint32_t kq = W.k3[q];
-                rank += (kq > kj) || (kq == kj && W.i3[q] < ij);
-              }
-              hit = rank == need - 1;
-            }
-            const uint32_t hm = __ballot_sync(0xffffffffu, hit);
-            if (hm) {
-              const int src = __ffs(hm) - 1;
-              T = __shfl_sync(0xffffffffu, kj, src);
-              I = __shfl_sync(0xffffffffu, ij, src);
-            }
-          }
-          // ---- (4) bitmap of the kept blocks, written out in order ----
-          const int words = ceil_div(n, 128) * 4;
-          pw_zero(W.bitmap, words);
-          __syncwarp();
-          for (int j = 0; j < lc; ++j) {
-            const uint32_t kk = W.lkey[j * 32 + lane];
-            const int b = W.lidx[j * 32 + lane];
-            if (kk > T || (kk == T && b <= I)) atomicOr(&W.bitmap[b >> 5], 1u << (b & 31));
-          }
-          __syncwarp();
-          int out = 0;
-          for (int w0 = 0; w0 < words; w0 += 32) {
-            const int wi = w0 + lane;
-            uint32_t bits = wi < words ? W.bitmap[wi] : 0u;
-            const int cn = __popc(bits);
-            int x = cn;
+        // ---- (4) ascending output ----
+        int out = 0;
+        for (int w0 = 0; w0 < words; w0 += 32) {
+          const int wi = w0 + lane;
+          uint32_t bits = wi < words ? bitmap[wi] : 0u;
+          const int cn = __popc(bits);
+          int xx = cn;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(0xffffffffu, x, o);
-              if (lane >= o) x += y;
-            }
-            int o = out + x - cn;
-            while (bits) {
-              const int bit = __ffs(bits) - 1;
-              bits &= bits - 1u;
-              if (o < TOPK) sel[o] = wi * 32 + bit;
-              ++o;
-            }
-            out += __shfl_sync(0xffffffffu, x, 31);
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, xx, o);
+            if (lane >= o) xx += y;
           }
-          if (lane == 0) {
-            if (out != TOPK) set_error(p.err, QSA_DEVERR_SELECTION);
-            p.sel_n[t] = min(out, TOPK);
+          int o = out + xx - cn;
+          while (bits) {
+            const int bit = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (o < TOPK) sel[o] = wi * 32 + bit;
+            ++o;
           }
+          out += __shfl_sync(0xffffffffu, xx, 31);
+        }
+        if (lane == 0) {
+          if (out != TOPK) set_error(p.err, QSA_DEVERR_SELECTION);
+          p.sel_n[t] = min(out, TOPK);
         }
       }
     }
-    if (overflow && lane == 0) {
-      const int slot = atomicAdd(p.ovf_n, 1);
-      p.ovf_list[slot] = t;
-    }
+    if (rescore && lane == 0) p.fb_list[atomicAdd(p.fb_n, 1)] = t;
   }
 }
 
-// Overflow rows: exact CTA-wide selection over the row's keys in L2.
-__global__ void __launch_bounds__(256) k_prefill_select_overflow(PrefillParams p) {
+// ----------------------------------------------------------------------------
+// Exact re-scoring of the rows the candidates could not settle: one CTA per
+// row, its warps stream the row's pages (16 compressed keys each) through
+// mma.sync into order-preserving score keys in global scratch, then an exact
+// CTA-wide top-512 (radix refinement for heavy ties) emits the kept blocks in
+// ascending order.
+// ----------------------------------------------------------------------------
+constexpr int PB_WARPS = 8;
+
+__global__ void __launch_bounds__(PB_WARPS * 32) k_prefill_rescore(PrefillParams p) {
   __shared__ FastTopScratch fs;
-  using All = Group<256, 0>;
-  const int nmax = p.cap / PF_M;
-  const int nov = *p.ovf_n;
-  for (int o = blockIdx.x; o < nov; o += gridDim.x) {
-    const int t = p.ovf_list[o];
-    const int n = (p.pos0 + t + 1) >> 2;
-    const uint32_t* row = p.keys + ((int64_t)(t >> 6) * nmax * PF_QT + (t & 63)) * PF_M;
+  using All = Group<PB_WARPS * 32, 0>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g8 = lane >> 2, cq = lane & 3;
+  const int nfb = *p.fb_n;
+  uint32_t* keys = p.fb_keys + (int64_t)blockIdx.x * p.fb_cap;
+  const uint4* cidx = reinterpret_cast<const uint4*>(p.c.cidx);
+  for (int o = blockIdx.x; o < nfb; o += gridDim.x) {
+    const int t = p.fb_list[o];  // global row
+    const PfSeg& sg = pf_seg_of_row(p, t);
+    const int n = (sg.pos0 + (t - sg.q_off) + 1) >> 2;
+    const int32_t* pt = p.c.page_table + (int64_t)sg.req * p.c.max_pages;
+    // B fragments of the rotated query (permuted like the page loads) and the lane's head weights
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.qrot + (int64_t)t * HI * D);
+    uint32_t bq[8][2];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int d0 = 8 * (cq + 4 * (j >> 1)) + 4 * (j & 1);
+      bq[j][0] = g8 < HI ? __ldg(q32 + ((g8 * D + d0) >> 1)) : 0u;
+      bq[j][1] = g8 < HI ? __ldg(q32 + ((g8 * D + d0 + 2) >> 1)) : 0u;
+    }
+    const float wa = cq < 2 ? __ldg(p.w + (int64_t)t * HI + 2 * cq) : 0.f;
+    const float wb = cq < 2 ? __ldg(p.w + (int64_t)t * HI + 2 * cq + 1) : 0.f;
+    const int np = ceil_div(n, PAGE_BLOCKS);
+    for (int lp = warp; lp < np; lp += PB_WARPS) {
+      int phys = lp < p.c.max_pages ? __ldg(pt + lp) : -1;
+      if (phys >= p.c.num_pages) phys = -1;  // flagged by the scorer already
+      PageRegs pr;
+      if (phys >= 0) load_page(pr, cidx + (int64_t)phys * (PAGE_BLOCKS * D / 8), g8, cq);
+      float lo = 0.f, hi = 0.f;
+      if (phys >= 0) score_page(pr, bq, wa, wb, lo, hi);
+      if (cq < 2) {
+        const int local = lp * PAGE_BLOCKS + g8 + 8 * cq;
+        if (local < n) keys[local] = score_key(cq ? hi : lo);
+      }
+    }
+    __syncthreads();
     int32_t* sel = p.sel + (int64_t)t * TOPK;
-    auto key_at = [&](int i) { return __ldcg(row + (int64_t)(i >> 7) * (PF_QT * PF_M) + (i & (PF_M - 1))); };
-    fast_topk<All>(key_at, n, TOPK, [&](int i, int out) { sel[out] = i; }, &fs);
-    if (threadIdx.x == 0) p.sel_n[t] = TOPK;
+    fast_topk<All>([&](int i) { return keys[i]; }, n, TOPK, [&](int i, int out) { sel[out] = i; }, &fs);
+    if (tid == 0) p.sel_n[t] = TOPK;
     __syncthreads();
   }
 }
 
 // ----------------------------------------------------------------------------
-// Rotation of the chunk's index queries (bf16, [T*4][128] rows for TMA).
+// Rotation of the chunk's index queries (bf16, [T*4][128] rows for TMA), and
+// each query's histogram base: an upper bound of its scores,
+//   s <= sum_h max(w_h, 0) * |q~_h| * |k^|,  |k^| <= 1 + 2^-8 (a bf16 unit vector),
+// taken with 2% of slack, sets the top bin; the 127 bins below it cover
+// eight octaves at 1/16 octave each.
 // ----------------------------------------------------------------------------
 // One warp per query: lane i owns the rotation pairs (i, i+64) and (i+32, i+96)
 // of all four heads; the angles pos * inv_freq_i are taken once per query in
@@ -726,23 +720,42 @@ __global__ void __launch_bounds__(PR_WARPS * 32) k_prefill_rotate(PrefillParams 
                                                                  RopeFreqs fr) {
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * PR_WARPS + (threadIdx.x >> 5);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.fb_n = 0;  // the re-scoring list of this call starts empty
   if (t >= p.T) return;
-  const double pos = (double)(p.pos0 + t);
+  const PfSeg& sg = pf_seg_of_row(p, t);
+  const double pos = (double)(sg.pos0 + (t - sg.q_off));
   double sn[2], cs[2];
 #pragma unroll
   for (int e = 0; e < 2; ++e) sincos(pos * fr.f[lane + 32 * e], &sn[e], &cs[e]);
   const uint16_t* qin = reinterpret_cast<const uint16_t*>(idx_q + (int64_t)t * HI * D);
   uint16_t* qo = reinterpret_cast<uint16_t*>(p.qrot + (int64_t)t * HI * D);
+  float nrm2[HI];
 #pragma unroll
   for (int h = 0; h < HI; ++h) {
+    nrm2[h] = 0.f;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int i = h * D + lane + 32 * e;
       const double x0 = (double)bf16_bits_to_f32(__ldg(qin + i));
       const double x1 = (double)bf16_bits_to_f32(__ldg(qin + i + D / 2));
-      qo[i] = f64_to_bf16_bits(x0 * cs[e] - x1 * sn[e]);
-      qo[i + D / 2] = f64_to_bf16_bits(x0 * sn[e] + x1 * cs[e]);
+      const uint16_t y0 = f64_to_bf16_bits(x0 * cs[e] - x1 * sn[e]);
+      const uint16_t y1 = f64_to_bf16_bits(x0 * sn[e] + x1 * cs[e]);
+      qo[i] = y0;
+      qo[i + D / 2] = y1;
+      const float f0 = bf16_bits_to_f32(y0), f1 = bf16_bits_to_f32(y1);
+      nrm2[h] = fmaf(f0, f0, fmaf(f1, f1, nrm2[h]));
     }
+  }
+#pragma unroll
+  for (int h = 0; h < HI; ++h)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) nrm2[h] += __shfl_xor_sync(0xffffffffu, nrm2[h], o);
+  if (lane == 0) {
+    const float4 w4 = __ldg(reinterpret_cast<const float4*>(p.w) + t);
+    const float bound = 1.02f * (fmaxf(w4.x, 0.f) * sqrtf(nrm2[0]) + fmaxf(w4.y, 0.f) * sqrtf(nrm2[1]) +
+                                 fmaxf(w4.z, 0.f) * sqrtf(nrm2[2]) + fmaxf(w4.w, 0.f) * sqrtf(nrm2[3]));
+    p.qbase[t] = bound > 0.f && bound < 3.0e38f ? (int)(score_key(bound) >> PF_BIN_SHIFT) - (PF_BINS - 1)
+                                                : PF_NO_BASE;
   }
 }
 
@@ -777,6 +790,10 @@ static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint32_t
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+
+// Warps per CTA of the selection: 8, fewer when each warp's block bitmap is large.
+static int select_warps(int bm_words) { return std::max(1, std::min(8, (200 * 1024) / ps_warp_bytes(bm_words))); }
+
 cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,
                            cudaStream_t st, const cudaEvent_t* ev, int n_ev) {
   auto mark = [&](int i) {
@@ -786,15 +803,16 @@ cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, c
   int dev = 0;
   cudaGetDevice(&dev);
   const size_t smem = sizeof(PfSmem) + 1024;
-  const size_t pw_smem = sizeof(PwWarp) * PW_WARPS;
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k_prefill_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_prefill_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pw_smem);
+      e = cudaFuncSetAttribute(k_prefill_select, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  if (p.cap % PF_M != 0) return cudaErrorInvalidValue;  // whole M-tile slots per work tile
+  if (p.fb_cap % 32 != 0 || p.fb_ctas < 1 || p.nseg < 1 || p.nseg > PF_MAX_SEGS) return cudaErrorInvalidValue;
+  for (int i = 0; i < p.nseg; ++i)
+    if (p.fb_cap < ((p.seg[i].pos0 + p.seg[i].T) >> 2)) return cudaErrorInvalidValue;
   CUtensorMap kmap, qmap;
   if (!make_map(&kmap, p.c.cidx, (uint64_t)p.c.num_pages * PAGE_BLOCKS, PAGE_BLOCKS)) return cudaErrorInvalidValue;
   if (!make_map(&qmap, p.qrot, (uint64_t)p.T * HI, PF_N)) return cudaErrorInvalidValue;
@@ -803,20 +821,23 @@ cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, c
   mark(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int tiles = ceil_div(p.T, PF_QT);
+  const int tiles = p.ntiles;
   mark(2);
   k_prefill_score<<<std::min(num_sms, tiles), PF_THREADS, smem, st>>>(p, kmap, qmap);
   mark(3);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark(4);
-  if ((e = cudaMemsetAsync(p.ovf_n, 0, sizeof(int), st)) != cudaSuccess) return e;
+  const int bm_words = p.fb_cap / 32;
+  const int warps = select_warps(bm_words);
+  const size_t ps_smem = (size_t)warps * ps_warp_bytes(bm_words);
   int per_sm = 0;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_prefill_select, PW_WARPS * 32, pw_smem)) !=
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_prefill_select, warps * 32, ps_smem)) !=
       cudaSuccess)
     return e;
-  k_prefill_select<<<std::min(ceil_div(p.T, PW_WARPS), std::max(1, per_sm) * num_sms), PW_WARPS * 32, pw_smem, st>>>(p);
+  k_prefill_select<<<std::min(ceil_div(p.T, warps), std::max(1, per_sm) * num_sms), warps * 32, ps_smem, st>>>(
+      p, bm_words);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_prefill_select_overflow<<<std::min(p.T, 2 * num_sms), 256, 0, st>>>(p);
+  k_prefill_rescore<<<p.fb_ctas, PB_WARPS * 32, 0, st>>>(p);
   mark(5);
   return cudaGetLastError();
 }

@@ -116,76 +116,6 @@ __device__ __forceinline__ int for_each_segment(int rs, int re, int ppc, F f) {
   return j;
 }
 
-#ifndef QSA_SC_L2_PROMOTE
-#define QSA_SC_L2_PROMOTE 0
-#endif
-__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
-  uint4 v;
-#if QSA_SC_L2_PROMOTE == 256
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-#elif QSA_SC_L2_PROMOTE == 128
-  asm volatile("ld.global.nc.L1::no_allocate.L2::128B.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-#else
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-#endif
-  return v;
-}
-
-// One page of 16 keys: lane (g, c) holds 16-byte chunks c, c+4, c+8, c+12 of
-// keys g and g+8.  Chunk u of key g, read as four bf16 pairs x, y, z, w,
-// supplies the A fragment of k-steps 2u (pairs x, y) and 2u+1 (pairs z, w):
-// logical k {2c, 2c+1} -> first pair, {2c+8, 2c+9} -> second pair.
-struct PageRegs {
-  uint4 lo[4], hi[4];  // keys g and g + 8
-};
-
-__device__ __forceinline__ void load_page(PageRegs& r, const uint4* page, int g, int c) {
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    r.lo[u] = ldg_stream(page + g * 16 + c + 4 * u);
-    r.hi[u] = ldg_stream(page + (g + 8) * 16 + c + 4 * u);
-  }
-}
-
-// The same with coherent loads, for the one page this kernel has just written a compressed key to.
-__device__ __forceinline__ void load_page_fresh(PageRegs& r, const uint4* page, int g, int c) {
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    r.lo[u] = __ldcg(page + g * 16 + c + 4 * u);
-    r.hi[u] = __ldcg(page + (g + 8) * 16 + c + 4 * u);
-  }
-}
-
-__device__ __forceinline__ void score_page(const PageRegs& r, const uint32_t (&bq)[8][2], float wa, float wb,
-                                           float& lo_score, float& hi_score) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int u = j >> 1;
-    uint32_t a[4];
-    a[0] = (j & 1) ? r.lo[u].z : r.lo[u].x;
-    a[1] = (j & 1) ? r.hi[u].z : r.hi[u].x;
-    a[2] = (j & 1) ? r.lo[u].w : r.lo[u].y;
-    a[3] = (j & 1) ? r.hi[u].w : r.hi[u].y;
-    mma_bf16_16816(acc, a, bq[j][0], bq[j][1]);
-  }
-  // acc: rows g / g+8 (keys), columns 2c, 2c+1 (heads); sum the heads over the quad
-  float lo = wa * fmaxf(acc[0], 0.f) + wb * fmaxf(acc[1], 0.f);
-  float hi = wa * fmaxf(acc[2], 0.f) + wb * fmaxf(acc[3], 0.f);
-  lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-  hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-  lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-  hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-  lo_score = lo;
-  hi_score = hi;
-}
-
 __global__ void __launch_bounds__(SC_THREADS, QSA_SC_CTAS_PER_SM) k_score_topk(ScoreParams p) {
   extern __shared__ uint8_t smem_raw[];
   ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(smem_aligned<128>(smem_raw));

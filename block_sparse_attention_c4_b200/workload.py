@@ -26,14 +26,15 @@ def slots_of(page_table_row: np.ndarray, n_tok: int, tok0: int = 0) -> np.ndarra
 
 
 def build_cache(wl, device="cuda", prefix_tokens=None, chunk_tokens: int = 1 << 16,
-                kv_layout: str = "interleaved") -> LayerCache:
+                kv_layout: str = "interleaved", kv_dtype: str = "bf16") -> LayerCache:
     """Allocate the cache of `wl`, fill K/V for every stored token, and append the raw index keys of
     the first `prefix_tokens[r]` tokens of each request (default: lens[r] - 1, the state before a
-    decode step) through qsa_compress_append."""
+    decode step) through qsa_compress_append.  kv_dtype "fp8" fills K/V with the workload's E4M3
+    codes (wl.k8 / wl.v8)."""
     pt = wl.page_table()
     B = wl.batch
     cache = LayerCache(wl.total_pages * PAGE_SIZE, B, pt.shape[1], rope_theta=wl.rope_theta, device=device,
-                       page_table=torch.from_numpy(pt).to(device), kv_layout=kv_layout)
+                       page_table=torch.from_numpy(pt).to(device), kv_layout=kv_layout, kv_dtype=kv_dtype)
     if prefix_tokens is None:
         prefix_tokens = [int(wl.lens[r]) - 1 for r in range(B)]
     for r in range(B):
@@ -41,8 +42,12 @@ def build_cache(wl, device="cuda", prefix_tokens=None, chunk_tokens: int = 1 << 
         for t0 in range(0, n, chunk_tokens):
             m = min(chunk_tokens, n - t0)
             slots = torch.from_numpy(slots_of(pt[r], m, t0)).to(device)
-            cache.k.index_copy_(0, slots, bits_to_bf16(wl.k(r, t0, m), device))
-            cache.v.index_copy_(0, slots, bits_to_bf16(wl.v(r, t0, m), device))
+            if kv_dtype == "fp8":
+                cache.k.index_copy_(0, slots, torch.from_numpy(wl.k8(r, t0, m)).to(device))
+                cache.v.index_copy_(0, slots, torch.from_numpy(wl.v8(r, t0, m)).to(device))
+            else:
+                cache.k.index_copy_(0, slots, bits_to_bf16(wl.k(r, t0, m), device))
+                cache.v.index_copy_(0, slots, bits_to_bf16(wl.v(r, t0, m), device))
         append_tokens(cache, wl, r, 0, int(prefix_tokens[r]), chunk_tokens)
     return cache
 

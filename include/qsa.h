@@ -118,7 +118,8 @@ typedef enum {
   QSA_OP_COMPRESS_APPEND = 5,
   QSA_OP_PREFILL_SCORE_TOPK = 6,
   QSA_OP_DECODE_INDEXER = 7, /* qsa_decode_indexer: rows = batch, max_len = longest context */
-  QSA_OP_DECODE_ATTEND = 8   /* qsa_decode_attend:  rows = batch, max_len = longest context */
+  QSA_OP_DECODE_ATTEND = 8,  /* qsa_decode_attend:  rows = batch, max_len = longest context */
+  QSA_OP_SPLIT_SCORE = 9     /* qsa_split_score_topk: rows = batch, max_len = longest context */
 } qsa_op;
 
 /*
@@ -179,7 +180,10 @@ qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const
  * positions pos0 .. pos0+T-1 of request `req` each score their complete
  * blocks b < floor((pos+1)/4) and keep the top 512.  Same result as
  * qsa_index_score_topk on those queries; built for long chunks, where the
- * chunk's queries share every compressed-key tile.
+ * chunk's queries share every compressed-key tile.  Scores do not go to
+ * memory: a sampled threshold per query lets only likely members of its top
+ * 512 through as candidates, the exact top 512 is taken among them, and a row
+ * the candidates cannot settle is re-scored in full (exact either way).
  * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
  * (prefill: a GPU kernel computes the index scores, a fast top-k selects).
  *   idx_q     bf16 [T][4][128] unrotated index queries
@@ -192,6 +196,31 @@ qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const
 qsa_status qsa_prefill_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, int32_t req,
                                   int32_t pos0, int32_t T, int32_t* blocks, int32_t* nblocks, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/*
+ * Prefill scoring of a ragged batch of causal chunks in one call (chunked
+ * prefill of several sequences at once: the aik8s.run deployment page runs
+ * chunked prefill of 8192 tokens over concurrent requests).  Segment i is the
+ * queries at positions seg_pos0[i] .. seg_pos0[i]+T_i-1 of request seg_req[i],
+ * T_i = cu_q[i+1] - cu_q[i], stored at rows cu_q[i] .. cu_q[i+1]-1 of idx_q,
+ * w, blocks and nblocks.  Each segment's result equals a
+ * qsa_prefill_score_topk call on it alone.  Requests may share pages: when
+ * two page tables map a shared prefix to the same physical pages, the
+ * compressed keys of that prefix are one copy (block b of a request lives at
+ * its own physical slot / 4, blog section "Qwen Sparse Attention: Retrieve
+ * Coarsely, Attend Precisely", page-aligned full_slot / 4 addressing), and
+ * both requests' queries score it.
+ *   nseg         1 .. 64 (host); seg_req, seg_pos0 int32 [nseg] and cu_q int32 [nseg+1]
+ *                are HOST arrays, cu_q[0] = 0, non-decreasing
+ *   max_len      host bound of seg_pos0[i] + T_i
+ *   idx_q        bf16 [cu_q[nseg]][4][128]; w f32 [cu_q[nseg]][4] (16-byte aligned)
+ *   blocks, nblocks   int32 [cu_q[nseg]][512], [cu_q[nseg]] out
+ *   ws           workspace of qsa_workspace_bytes(QSA_OP_PREFILL_SCORE_TOPK, cu_q[nseg], max_len)
+ */
+qsa_status qsa_prefill_score_topk_varlen(const qsa_cache* cache, const void* idx_q, const float* w, int32_t nseg,
+                                         const int32_t* seg_req, const int32_t* seg_pos0, const int32_t* cu_q,
+                                         int32_t max_len, int32_t* blocks, int32_t* nblocks, void* ws,
+                                         size_t ws_bytes, void* stream);
 
 /*
  * Expand kept blocks to token positions: block b -> 4b..4b+3 in block order,
@@ -247,6 +276,30 @@ qsa_status qsa_sparse_gqa(const qsa_cache* cache, const void* q, const int32_t* 
 qsa_status qsa_decode(const qsa_cache* cache, const void* idx_k_new, const void* idx_q, const float* w,
                       const void* q, const int32_t* seq_len, int32_t max_len, float scale, void* out, float* lse,
                       int32_t* blocks_out, int32_t* nblocks_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * FP8 K/V variants of qsa_sparse_gqa and qsa_decode.  The pages run FP8
+ * checkpoints and an FP8 KV cache (the aik8s.run deployment page and the
+ * ailone.io model page) but do not state its format; the reading used here:
+ * the raw attention keys and values are E4M3 bytes with one FP32 scale for K
+ * and one for V (value = code * scale); everything else, the compressed index
+ * keys and the ring included, stays as in the bf16 calls.
+ *   cache->k, cache->v   E4M3 bytes: slot s holds its two KV heads' 128-byte rows at
+ *                        k + s * kv_stride (bytes; 0 means 256, separate arrays; 512 with
+ *                        v = k + 256 interleaves K and V); kv_stride a multiple of 16
+ *   k_scale, v_scale     positive, finite
+ * Every other argument is that of qsa_sparse_gqa / qsa_decode (same workspaces).
+ * Attention is computed on the exact dequantized values (each E4M3 value is a
+ * bf16 value; the K scale joins the softmax scale and the V scale the output).
+ */
+qsa_status qsa_sparse_gqa_fp8(const qsa_cache* cache, float k_scale, float v_scale, const void* q,
+                              const int32_t* q_req, const int32_t* pos, const int32_t* npos, int32_t pos_stride,
+                              int32_t max_pos, int32_t nq, float scale, void* out, float* lse, void* ws,
+                              size_t ws_bytes, void* stream);
+qsa_status qsa_decode_fp8(const qsa_cache* cache, float k_scale, float v_scale, const void* idx_k_new,
+                          const void* idx_q, const float* w, const void* q, const int32_t* seq_len, int32_t max_len,
+                          float scale, void* out, float* lse, int32_t* blocks_out, int32_t* nblocks_out, void* ws,
+                          size_t ws_bytes, void* stream);
 
 /*
  * IndexShare draft step: attention only, the indexer is skipped.
@@ -317,6 +370,48 @@ qsa_status qsa_decode_attend(const qsa_cache* cache, const void* q, const int32_
                              void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Split-context decode: a request's context divided over several GPUs (ranks)
+ * by page ranges, for one very long request that one GPU would decode slowly.
+ * The pages describe no such split (the layer runs on one GPU there); this is
+ * the plainest exact split of the decode step of blog section "Qwen Sparse
+ * Attention: Retrieve Coarsely, Attend Precisely".  Each rank holds pages
+ * [page_lo[r], page_lo[r] + page_cnt[r]) of request r in a cache of its own
+ * whose page-table row is indexed by the request's logical page (only those
+ * pages mapped), so positions and block numbers are the request's own
+ * everywhere.  A step, on every rank:
+ *   1. the rank holding position L-1 appends the new index key
+ *      (qsa_compress_append at len_before = L-1);
+ *   2. qsa_split_score_topk: its best min(512, its blocks) (score key, block)
+ *      in block order, the index query rotated at L-1;
+ *   3. an all-gather of the candidates in rank order (ranks hold increasing
+ *      page ranges), then qsa_split_merge: the exact top 512 of the request,
+ *      the same on every rank;
+ *   4. qsa_split_positions: the kept positions the rank holds (plus the tail
+ *      on the rank holding L-1), then qsa_sparse_gqa with lse;
+ *   5. an all-gather of (out, lse) and qsa_split_combine.
+ * qsa_split_score_topk:
+ *   seq_len, page_lo, page_cnt   int32 [batch] (device)
+ *   cand_key uint32 [batch][512], cand_id int32 [batch][512], cand_n int32 [batch] out
+ *   ws  workspace of qsa_workspace_bytes(QSA_OP_SPLIT_SCORE, batch, max_len)
+ * qsa_split_merge: cand_key / cand_id [world][rows][512], cand_n [world][rows]
+ *   (the ranks' outputs stacked in rank order) -> blocks [rows][512] ascending,
+ *   nblocks [rows]; world <= 64.
+ * qsa_split_positions: -> pos int32 [rows][2051], npos int32 [rows].
+ * qsa_split_combine: outs bf16 [world][rows][16][128], lses f32 [world][rows][16]
+ *   (natural-log LSE; -inf for a rank without positions) -> out bf16 [rows][16][128].
+ */
+qsa_status qsa_split_score_topk(const qsa_cache* cache, const void* idx_q, const float* w, const int32_t* seq_len,
+                                const int32_t* page_lo, const int32_t* page_cnt, int32_t max_len, uint32_t* cand_key,
+                                int32_t* cand_id, int32_t* cand_n, void* ws, size_t ws_bytes, void* stream);
+qsa_status qsa_split_merge(const uint32_t* cand_key, const int32_t* cand_id, const int32_t* cand_n, int32_t world,
+                           int32_t rows, int32_t* blocks, int32_t* nblocks, void* stream);
+qsa_status qsa_split_positions(const int32_t* seq_len, const int32_t* page_lo, const int32_t* page_cnt,
+                               const int32_t* blocks, const int32_t* nblocks, int32_t rows, int32_t* pos,
+                               int32_t* npos, void* stream);
+qsa_status qsa_split_combine(const void* outs, const float* lses, int32_t world, int32_t rows, void* out,
+                             void* stream);
+
+/*
  * Sparse GQA without a workspace: the same computation as qsa_sparse_gqa
  * (same arguments minus ws / ws_bytes), for callers that cannot allocate
  * device memory or pass the library scratch space -- e.g. a plugin whose host
@@ -385,6 +480,14 @@ int32_t qsa_device_error(void* ws, int32_t clear, void* stream);
  * Not thread-safe with concurrent qsa_decode calls from several host threads.
  */
 void qsa_set_profile_events(void* const* events, int32_t n_pairs);
+
+/*
+ * Measurement hook of qsa_prefill_score_topk: how many rows of the last call
+ * made with workspace `ws` (sized for T queries and contexts up to max_len)
+ * could not be settled from their filtered candidates and were re-scored in
+ * full.  Synchronises `stream`.  Returns -1 on error.
+ */
+int32_t qsa_prefill_rescored_rows(void* ws, int32_t T, int32_t max_len, void* stream);
 
 /* Number of kernels qsa_decode launches per call for `batch` requests: 2 up to
  * 512 requests (the scorer runs the indexer front end itself, then the sparse

@@ -65,6 +65,10 @@ def lib():
                                           ctypes.c_int]
         L.oracle_prefill_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, f64, f64, vp, vp, vp, vp, ctypes.c_int]
         L.oracle_indexshare.argtypes = [vp, i32, i64, i32, vp, vp, vp, f64, vp]
+        L.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_to_f64.restype = f64
+        L.oracle_sparse_gqa_fp8.argtypes = [vp, vp, vp, f64, f64, vp, i32, f64, vp, vp]
+        L.oracle_sparse_gqa_fp8.restype = None
         L.oracle_index_project.argtypes = [vp, vp, i64, i64, vp, vp, vp, ctypes.c_int]
         for name in ("oracle_rope_f64", "oracle_compress_block", "oracle_compress", "oracle_append",
                      "oracle_rotate_query", "oracle_block_scores", "oracle_sparse_gqa", "oracle_decode_batch",
@@ -159,6 +163,24 @@ def sparse_gqa(q: np.ndarray, K: np.ndarray, V: np.ndarray, pos: np.ndarray, sca
     out = np.empty((HQ, D), dtype=np.float64)
     lse = np.empty(HQ, dtype=np.float64)
     lib().oracle_sparse_gqa(_p(q), _p(K), _p(V), _p(pos), len(pos), scale, _p(out), _p(lse))
+    return out, lse
+
+
+def e4m3_to_f64(b: int) -> float:
+    return float(lib().oracle_e4m3_to_f64(int(b)))
+
+
+def sparse_gqa_fp8(q: np.ndarray, K8: np.ndarray, V8: np.ndarray, k_scale: float, v_scale: float, pos: np.ndarray,
+                   scale: float = SCALE):
+    """q [16,128] bf16 bits; K8, V8 [T,2,128] E4M3 bytes (uint8, logical); pos int32 -> (out [16,128] f64, lse [16])."""
+    q = _u16(q).reshape(HQ, D)
+    K8 = np.ascontiguousarray(K8, dtype=np.uint8)
+    V8 = np.ascontiguousarray(V8, dtype=np.uint8)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    out = np.empty((HQ, D), dtype=np.float64)
+    lse = np.empty(HQ, dtype=np.float64)
+    lib().oracle_sparse_gqa_fp8(_p(q), _p(K8), _p(V8), float(k_scale), float(v_scale), _p(pos), len(pos), scale,
+                                _p(out), _p(lse))
     return out, lse
 
 

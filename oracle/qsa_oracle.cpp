@@ -250,6 +250,48 @@ void oracle_sparse_gqa(const uint16_t* q, const uint16_t* K, const uint16_t* V, 
   }
 }
 
+// E4M3 byte -> value, from the format's definition: sign bit, 4 exponent bits (bias 7), 3 mantissa
+// bits; exponent 0 is subnormal (m/8 * 2^-6); exponent 15 with mantissa 7 is NaN (no infinities).
+double e4m3_to_f64(uint8_t b) {
+  const int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e ? std::ldexp(1.0 + m / 8.0, e - 7) : std::ldexp(m / 8.0, -6);
+  return sgn ? -mag : mag;
+}
+
+double oracle_e4m3_to_f64(uint8_t b) { return e4m3_to_f64(b); }
+
+// Sparse GQA over FP8 K/V (reading: E4M3 codes with one scale for K and one for V, value = code *
+// scale), FP64: head h uses KV head h/8; o_h = softmax_j(scale * q_h . K[pos_j]) V[pos_j].
+// K8, V8: [token][2][128] E4M3 bytes.  out: [16][128] FP64; lse: [16] (natural log), may be null.
+void oracle_sparse_gqa_fp8(const uint16_t* q, const uint8_t* K8, const uint8_t* V8, double k_scale, double v_scale,
+                           const int32_t* pos, int32_t npos, double scale, double* out, double* lse) {
+  std::vector<double> logit(npos > 0 ? npos : 1);
+  for (int h = 0; h < HQ; ++h) {
+    const int g = h / (HQ / HKV);
+    double qh[D];
+    for (int d = 0; d < D; ++d) qh[d] = bf16_to_f64(q[h * D + d]);
+    double mx = -INFINITY;
+    for (int32_t j = 0; j < npos; ++j) {
+      const uint8_t* kr = K8 + (static_cast<int64_t>(pos[j]) * HKV + g) * D;
+      double dot = 0.0;
+      for (int d = 0; d < D; ++d) dot += qh[d] * (e4m3_to_f64(kr[d]) * k_scale);
+      logit[j] = dot * scale;
+      mx = std::max(mx, logit[j]);
+    }
+    double den = 0.0;
+    double acc[D] = {0.0};
+    for (int32_t j = 0; j < npos; ++j) {
+      const double p = std::exp(logit[j] - mx);
+      den += p;
+      const uint8_t* vr = V8 + (static_cast<int64_t>(pos[j]) * HKV + g) * D;
+      for (int d = 0; d < D; ++d) acc[d] += p * (e4m3_to_f64(vr[d]) * v_scale);
+    }
+    for (int d = 0; d < D; ++d) out[h * D + d] = npos > 0 ? acc[d] / den : 0.0;
+    if (lse) lse[h] = npos > 0 ? mx + std::log(den) : -INFINITY;
+  }
+}
+
 // Selection of one query: rotate, score complete blocks, keep the top-512,
 // expand with the tail.  comp must hold at least floor(L/4) blocks.
 // Returns the number of positions; writes blocks (<=512), nblocks, pos (<=2051).

@@ -32,7 +32,7 @@ PAGE = 64
 
 # stream kinds
 K_IDXQ, K_W, K_IDXK, K_BIAS, K_Q, K_K, K_V, K_PAGES, K_LENS = 1, 2, 3, 4, 5, 6, 7, 8, 9
-K_HIDDEN, K_WPROJ = 10, 11
+K_HIDDEN, K_WPROJ, K_K8, K_V8 = 10, 11, 12, 13
 
 
 def _threads() -> int:
@@ -94,6 +94,15 @@ def normal_scaled_bf16(seed: int, strm: int, shape, std: float, offset: int = 0)
     out = np.empty(shape, dtype=np.uint16)
     lib().qsa_gen_normal_scaled_bf16(seed, strm, offset, out.size, float(std), _ptr(out), _threads())
     return out
+
+
+def normal_fp8_e4m3(seed: int, strm: int, shape, std: float = 1.0, offset: int = 0) -> np.ndarray:
+    """N(0, std^2) values of the stream (bf16 first), converted to E4M3 codes by torch's float8_e4m3fn
+    conversion; raw uint8 codes."""
+    import torch
+
+    f = bf16_bits_to_f32(normal_scaled_bf16(seed, strm, shape, std, offset=offset))
+    return torch.from_numpy(np.ascontiguousarray(f)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
 def uniform_f32(seed: int, strm: int, shape, lo: float = 0.0, hi: float = 1.0, offset: int = 0) -> np.ndarray:
@@ -194,6 +203,18 @@ class Workload:
         index projection."""
         n = self.n_queries(r) if n is None else n
         return normal_bf16(self.seed, stream(K_HIDDEN, r), (n, hidden), offset=q0 * hidden)
+
+    def k8(self, r: int, tok0: int = 0, n: int | None = None, std: float = 2.0) -> np.ndarray:
+        """FP8 (E4M3) attention keys [n, 2, 128] of request r, N(0, std^2) in code units."""
+        n = self.tokens(r) - tok0 if n is None else n
+        return normal_fp8_e4m3(self.seed, stream(K_K8, r), (n, KV_HEADS, HEAD_DIM), std,
+                               offset=tok0 * KV_HEADS * HEAD_DIM)
+
+    def v8(self, r: int, tok0: int = 0, n: int | None = None, std: float = 4.0) -> np.ndarray:
+        """FP8 (E4M3) attention values [n, 2, 128] of request r, N(0, std^2) in code units."""
+        n = self.tokens(r) - tok0 if n is None else n
+        return normal_fp8_e4m3(self.seed, stream(K_V8, r), (n, KV_HEADS, HEAD_DIM), std,
+                               offset=tok0 * KV_HEADS * HEAD_DIM)
 
     def bias_direction(self, r: int) -> np.ndarray:
         nq = self.n_queries(r)

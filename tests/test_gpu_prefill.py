@@ -39,6 +39,7 @@ def _run(Q, W, wl, pos0, T, rows=None):
                                            pos0, ws)
     torch.cuda.synchronize()
     assert ws.device_error() == 0
+    print(f"prefill pos0={pos0} T={T}: {Q.prefill_rescored_rows(ws, T, pos0 + T)} rows re-scored in full")
     bl, nbl = blocks.cpu().numpy(), nblocks.cpu().numpy()
     comp = O.compress(wl.idx_keys(0, 0, pos0 + T))
     rows = range(T) if rows is None else rows
@@ -137,3 +138,41 @@ def test_prefill_heavy_ties(Q, W):
             ob, _, s = O.select_query(idx_q[i], w[i], keys[:(t + 1) // 4], t + 1)
             assert len(np.unique(s)) <= 2 and nbl[i] == 512
             np.testing.assert_array_equal(bl[i], ob)
+
+
+def test_prefill_rows_the_candidates_cannot_settle(Q, W):
+    """Blocks of the sampled M-tiles (every 8th run of 128 blocks) score high and every other block
+    low, so each query's sampled threshold lets far fewer than 512 blocks through: every such row is
+    re-scored in full, and the result is still the exact top 512."""
+    nb = 8192
+    L = 4 * nb
+    T = 96
+    wl = G.custom_decode(33, [L])
+    cache = W.build_cache(wl, prefix_tokens=[0])
+    rng = np.random.default_rng(9)
+    a = rng.standard_normal(128)
+    bdir = -a + 0.1 * rng.standard_normal(128)
+    blk = np.arange(nb)
+    sampled = (blk // 128) % 8 == 0
+    vecs = np.where(sampled[:, None], a[None, :], bdir[None, :]) + 0.3 * rng.standard_normal((nb, 128))
+    vecs /= np.linalg.norm(vecs, axis=1, keepdims=True)
+    keys = torch.from_numpy(vecs.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    pt = wl.page_table()[0]
+    entries = (pt[(4 * blk) // 64].astype(np.int64) * 64 + (4 * blk) % 64) // 4
+    cache.cidx[torch.from_numpy(entries).cuda()] = W.bits_to_bf16(keys, "cuda")
+    qa = torch.from_numpy((a / np.linalg.norm(a)).astype(np.float32)).to(torch.bfloat16)
+    qa = qa.view(torch.int16).numpy().view(np.uint16)
+    idx_q = np.repeat(np.repeat(qa[None, :], 4, axis=0)[None], T, axis=0)
+    w = np.tile(np.array([[1.0, 0.5, 0.25, 0.125]], dtype=np.float32), (T, 1))
+    pos0 = L - T
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, L))
+    blocks, nblocks = Q.prefill_score_topk(cache, W.bits_to_bf16(idx_q, "cuda"), torch.from_numpy(w).cuda(), 0,
+                                           pos0, ws)
+    torch.cuda.synchronize()
+    assert ws.device_error() == 0
+    assert Q.prefill_rescored_rows(ws, T, L) == T  # every row took the full re-scoring path
+    bl, nbl = blocks.cpu().numpy(), nblocks.cpu().numpy()
+    for i in range(0, T, 5):
+        t = pos0 + i
+        ob, _, s = O.select_query(idx_q[i], w[i], keys[:(t + 1) // 4], t + 1)
+        check_selection(bl[i, :nbl[i]], ob, s, (t + 1) // 4, what=f"re-scored row {t}")

@@ -1,7 +1,8 @@
 """Index projection and the two-phase decode (indexer on a second stream) against the CPU oracle.
 
-* qsa_index_project: projected index queries and keys within one bf16 ulp of the oracle's FP64
-  projection (and almost all bit-exact), head weights within FP32 accumulation error.
+* qsa_index_project: projected index queries and keys within half a bf16 ulp of the exact projection
+  plus a bound of the FP32 accumulation error (and at least 99% bit-equal to the oracle's), head
+  weights within FP32 accumulation error.
 * qsa_decode_indexer + qsa_decode_attend: the GPU's projections (the same kernel, read back through
   qsa_index_project) are checked against the oracle's; from those values on, the oracle appends the
   key, selects and attends, and the GPU's kept blocks and outputs must match it under the usual
@@ -42,21 +43,26 @@ def W():
     return W
 
 
-def _ulps(a_bits, b_bits):
-    """Distance in bf16 ulps between two arrays of bf16 bits of the same sign (finite values)."""
-    a = a_bits.astype(np.int32)
-    b = b_bits.astype(np.int32)
-    sa = np.where(a & 0x8000, -(a & 0x7FFF), a)
-    sb = np.where(b & 0x8000, -(b & 0x7FFF), b)
-    return np.abs(sa - sb)
-
-
-def _check_projection(got_q, got_k, got_w, ref_q, ref_k, ref_w, what=""):
-    for g, r, name in ((got_q, ref_q, "idx_q"), (got_k, ref_k, "idx_k")):
-        u = _ulps(g, r)
-        assert u.max() <= 1, f"{what} {name}: {int(u.max())} ulps"
-        assert np.mean(u == 0) >= 0.995, f"{what} {name}: only {np.mean(u == 0):.4f} bit-exact"
-    np.testing.assert_allclose(got_w, ref_w, rtol=1e-4, atol=1e-5, err_msg=f"{what} w")
+def _check_projection(got_q, got_k, got_w, x, Wp, what=""):
+    """Each GPU output against the exact (FP64) projection: within half a bf16 ulp of it plus the FP32
+    accumulation error, bounded by 2^-18 * sum_j |x_j W_fj| (several dozen FP32 roundings of partial
+    sums no larger than that); and at least 99% of the bf16 outputs bit-equal to the oracle's."""
+    xf = G.bf16_bits_to_f32(x).astype(np.float64)
+    wf = G.bf16_bits_to_f32(Wp).astype(np.float64)
+    y = xf @ wf.T                                  # [n, 644] exact up to FP64 rounding
+    bound = 2.0 ** -18 * (np.abs(xf) @ np.abs(wf).T)
+    rq, rk, rw = O.index_project(x, Wp)
+    n = x.shape[0]
+    for got, ref, sl, name in ((got_q, rq, slice(0, 512), "idx_q"), (got_k, rk, slice(512, 640), "idx_k")):
+        g = G.bf16_bits_to_f32(got.reshape(n, -1)).astype(np.float64)
+        ye = y[:, sl]
+        ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ye), 1e-30))) - 7)
+        err = np.abs(g - ye)
+        assert np.all(err <= 0.5 * ulp + bound[:, sl]), f"{what} {name}: max excess {np.max(err - 0.5 * ulp - bound[:, sl])}"
+        assert np.mean(got.reshape(n, -1) == ref.reshape(n, -1)) >= 0.99, f"{what} {name}: too few bit-exact"
+    np.testing.assert_array_less(np.abs(got_w.astype(np.float64) - y[:, 640:]),
+                                 np.abs(y[:, 640:]) * 2.0 ** -23 + bound[:, 640:] + 1e-30)
+    np.testing.assert_allclose(got_w, rw, rtol=1e-4, atol=1e-5, err_msg=f"{what} w")
 
 
 @pytest.mark.parametrize("n,hidden", [(1, 128), (70, 4096), (33, 2560)])
@@ -65,8 +71,7 @@ def test_index_project_matches_oracle(Q, W, n, hidden):
     Wp = G.projection_weights(71, hidden)
     iq, ik, w = Q.index_project(W.bits_to_bf16(x, "cuda"), W.bits_to_bf16(Wp, "cuda"))
     torch.cuda.synchronize()
-    rq, rk, rw = O.index_project(x, Wp)
-    _check_projection(bf16_tensor_to_bits(iq), bf16_tensor_to_bits(ik), w.cpu().numpy(), rq, rk, rw,
+    _check_projection(bf16_tensor_to_bits(iq), bf16_tensor_to_bits(ik), w.cpu().numpy(), x, Wp,
                       what=f"n={n} hidden={hidden}")
 
 
@@ -94,8 +99,7 @@ def test_decode_indexer_and_attend_match_oracle(Q, W):
     torch.cuda.synchronize()
     assert ws_i.device_error() == 0 and ws_a.device_error() == 0
     iq, ik, w = bf16_tensor_to_bits(iq), bf16_tensor_to_bits(ik), w.cpu().numpy()
-    rq, rk, rw = O.index_project(x, Wp)
-    _check_projection(iq, ik, w, rq, rk, rw, what="decode projection")
+    _check_projection(iq, ik, w, x, Wp, what="decode projection")
     bl, nbl = blocks.cpu().numpy(), nblocks.cpu().numpy()
     got = bf16_tensor_to_f32(out)
     for r, L in enumerate(lens):

@@ -443,3 +443,43 @@ def test_index_project_is_rounded_linear_map(oracle_lib):
     x2[:, 1] = x[:, 0]
     q2, _, _ = O.index_project(x2, W, nthreads=1)
     assert not np.array_equal(q2, idx_q)
+
+
+# --- FP8 K/V ------------------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_on_every_code(oracle_lib):
+    """The oracle's E4M3 decode, written from the format's definition, against torch's
+    float8_e4m3fn -> float32 conversion for all 256 codes (NaN codes included)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float32).numpy().astype(np.float64)
+    got = np.array([O.e4m3_to_f64(b) for b in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_sparse_gqa_fp8_matches_torch_sdpa_on_dequantized_values(oracle_lib):
+    rng = np.random.default_rng(16)
+    T = 2500
+    K8 = G.normal_fp8_e4m3(16, 1, (T, 2, 128), 2.0)
+    V8 = G.normal_fp8_e4m3(16, 2, (T, 2, 128), 4.0)
+    q = G.normal_bf16(16, 3, (16, 128))
+    ks, vs = 0.5, 0.25
+    Kd = torch.from_numpy(K8).view(torch.float8_e4m3fn).to(torch.float64).numpy() * ks
+    Vd = torch.from_numpy(V8).view(torch.float8_e4m3fn).to(torch.float64).numpy() * vs
+    for n in (1, 9, 2051):
+        pos = np.sort(rng.choice(T, size=n, replace=False)).astype(np.int32)
+        out, lse = O.sparse_gqa_fp8(q, K8, V8, ks, vs, pos)
+        qt = torch.from_numpy(f32(q).astype(np.float64)).view(1, 16, 1, 128)
+        kt = torch.from_numpy(Kd[pos]).permute(1, 0, 2).unsqueeze(0)
+        vt = torch.from_numpy(Vd[pos]).permute(1, 0, 2).unsqueeze(0)
+        ro = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, enable_gqa=True).view(16, 128).numpy()
+        np.testing.assert_allclose(out, ro, rtol=1e-10, atol=1e-12)
+        s = (qt @ kt.repeat_interleave(8, dim=1).transpose(-1, -2)) / np.sqrt(128.0)
+        np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).view(16).numpy(), rtol=1e-12, atol=1e-12)
+    # the K scale and the V scale act where they should: swapping them changes the output
+    pos = np.arange(64, dtype=np.int32)
+    a, _ = O.sparse_gqa_fp8(q, K8, V8, ks, vs, pos)
+    b, _ = O.sparse_gqa_fp8(q, K8, V8, vs, ks, pos)
+    assert np.max(np.abs(a - b)) > 1e-3
