@@ -49,8 +49,13 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-scorer measurement")
     ap.add_argument("--only-prefill", action="store_true",
                     help="run only the prefill-scorer measurement and print its JSON (for profiling it alone)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the secondary measurements (FP8 K/V, index projection, varlen prefill, split decode)")
     ap.add_argument("--no-long-prefill", action="store_true",
                     help="with the prefill measurement, skip the 262144-token long-context prefill")
+    ap.add_argument("--prefill-chunk", type=int, default=-1, metavar="POS0",
+                    help="run only the 8192-query prefill chunk at POS0 of the 262144-token context, 3 times "
+                         "(for profiling one chunk)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU work of the oracle baseline")
     return ap.parse_args()
 
@@ -379,15 +384,255 @@ def run_ours(args, rank, world, local_rank):
             "wall_s_timed_region": round(wall, 3),
             "setup_s": round(setup_s, 1),
         }
-    # free device memory before the secondary measurement and the CPU baseline
-    del cache, ws, flush, sess
+    # free device memory before the secondary measurements and the CPU baseline
+    del ws, sess
+    if rank == 0 and not args.no_extras:
+        res["extras"] = {}
+        extra(res["extras"], "index_projection_two_stream", run_projection_decode, cache, inp, wl, dev, flush)
+        extra(res["extras"], "fp8_kv_decode", run_fp8_decode, cache, inp, wl, dev, flush, score_b, gqa_b)
+        extra(res["extras"], "varlen_prefill", run_varlen_prefill, cache, wl, dev, flush)
+    del cache, flush
     torch.cuda.empty_cache()
     if rank == 0 and not args.no_prefill:
         res["prefill_scorer"] = run_prefill_scorer(dev)
         torch.cuda.empty_cache()
+    if rank == 0 and not args.no_extras:
+        extra(res["extras"], "split_context_decode_262k", run_split_decode, dev)
+        torch.cuda.empty_cache()
     if world > 1:
         dist.destroy_process_group()
     return res, wl
+
+
+def extra(out: dict, name: str, fn, *args):
+    """A secondary measurement: its result under `name`, or the error it raised (the headline number
+    above does not depend on it)."""
+    import torch
+
+    try:
+        out[name] = fn(*args)
+    except Exception as e:  # reported in the JSON line, not hidden
+        out[name] = {"error": f"{type(e).__name__}: {e}"[:500]}
+    torch.cuda.synchronize()
+
+
+def time_calls(fn, reps: int, flush=None):
+    """Mean CUDA-event time (ms) of `fn` on the current stream over `reps` calls (L2 flushed before each
+    when `flush` is given, outside the events)."""
+    import torch
+
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for k in range(reps):
+        if flush is not None:
+            flush.zero_()
+        ev[k][0].record(st)
+        fn()
+        ev[k][1].record(st)
+    torch.cuda.synchronize()
+    return float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+
+def run_projection_decode(cache, inp, wl, dev, flush, hidden: int = 4096, reps: int = 200):
+    """The decode step from hidden states: qsa_decode_indexer (index projection, append, scoring,
+    top-512) and qsa_decode_attend, on one stream; and with the indexer on a second stream while the
+    main stream runs a stand-in for the caller's Q/K/V projection (a bf16 GEMM [B, hidden] x
+    [hidden, (16 + 2 + 2) x 128]), joined by an event before the attention."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+    import qsa_gen as G
+
+    B, max_len = wl.batch, int(max(wl.lens))
+    x = W.bits_to_bf16(np.stack([wl.hidden(r, hidden)[0] for r in range(B)]), dev)
+    wp = W.bits_to_bf16(G.projection_weights(wl.seed, hidden), dev)
+    w_qkv = torch.randn(hidden, 20 * 128, device=dev, dtype=torch.bfloat16) * hidden ** -0.5
+    ws_i = Q.Workspace(Q.workspace_bytes(Q.OP_DECODE_INDEXER, B, max_len), device=dev)
+    ws_a = Q.Workspace(Q.workspace_bytes(Q.OP_DECODE_ATTEND, B, max_len), device=dev)
+    blocks = torch.empty(B, 512, dtype=torch.int32, device=dev)
+    nblocks = torch.empty(B, dtype=torch.int32, device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.bfloat16, device=dev)
+    main, side = torch.cuda.current_stream(), torch.cuda.Stream(device=dev)
+    done = torch.cuda.Event()
+
+    def one_stream():
+        Q.decode_indexer(cache, x, wp, inp["seq_len"], max_len, ws_i, blocks, nblocks)
+        Q.decode_attend(cache, inp["q"], inp["seq_len"], max_len, blocks, nblocks, ws_a, out=out)
+
+    def proj_only():
+        Q.index_project(x, wp)
+
+    def qkv():
+        return x @ w_qkv
+
+    def serial():
+        qkv()
+        one_stream()
+
+    def overlapped():
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            Q.decode_indexer(cache, x, wp, inp["seq_len"], max_len, ws_i, blocks, nblocks, stream=side)
+        done.record(side)
+        qkv()
+        main.wait_event(done)
+        Q.decode_attend(cache, inp["q"], inp["seq_len"], max_len, blocks, nblocks, ws_a, out=out)
+
+    for f in (one_stream, proj_only, qkv, serial, overlapped):
+        for _ in range(3):
+            f()
+    torch.cuda.synchronize()
+    if ws_i.device_error() != 0 or ws_a.device_error() != 0:
+        raise RuntimeError("device error word set in the two-phase decode")
+    t = {name: time_calls(f, reps, flush) for name, f in
+         (("indexer_plus_attend_us", one_stream), ("projection_alone_us", proj_only), ("qkv_gemm_alone_us", qkv),
+          ("qkv_then_decode_us", serial), ("decode_overlapping_qkv_us", overlapped))}
+    wbytes = (4 * 128 + 128 + 4) * hidden * 2
+    res = {k: round(v * 1e3, 2) for k, v in t.items()}
+    res.update({"hidden": hidden, "batch": B, "projection_weight_bytes": wbytes,
+                "projection_hbm_gbs": round((wbytes + B * hidden * 2) / (t["projection_alone_us"] * 1e-3) / 1e9, 1),
+                "note": "indexer on a second stream while the main stream runs the caller's Q/K/V projection "
+                        "stand-in (torch matmul, not part of this library); joined by an event"})
+    return res
+
+
+def run_fp8_decode(cache, inp, wl, dev, flush, score_b, gqa_b, reps: int = 400):
+    """qsa_decode_fp8 on the headline workload: the same cache with its K/V as E4M3 codes (the bf16 pool
+    divided by the scale and converted on the device), the same index cache."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+
+    B, max_len = wl.batch, int(max(wl.lens))
+    scale = 0.25
+    c8 = Q.LayerCache(cache.num_slots, B, cache.max_pages, rope_theta=cache.rope_theta, device=dev,
+                      page_table=cache.page_table, kv_dtype="fp8")
+    c8.cidx, c8.ring = cache.cidx, cache.ring
+    step = 1 << 20
+    for s0 in range(0, cache.num_slots, step):
+        src = cache.kv[s0:s0 + step].float() / scale
+        c8.kv[s0:s0 + step].copy_(src.to(torch.float8_e4m3fn).view(torch.uint8))
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_DECODE, B, max_len), device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.bfloat16, device=dev)
+
+    def step_fn():
+        Q.decode_fp8(c8, inp["idx_k_new"], inp["idx_q"], inp["w"], inp["q"], inp["seq_len"], max_len, ws, scale,
+                     scale, out=out)
+
+    for _ in range(5):
+        step_fn()
+    torch.cuda.synchronize()
+    if ws.device_error() != 0:
+        raise RuntimeError("device error word set in the FP8 decode")
+    ms = time_calls(step_fn, reps, flush)
+    total = score_b + gqa_b // 2  # K/V rows halve: 512 B per position
+    hbm, _ = measured_peaks()
+    del c8
+    return {"ms_per_step": round(ms, 5), "query_tok_per_s": round(B / (ms * 1e-3), 1),
+            "step_bytes_algorithmic": int(total), "step_hbm_gbs": round(total / (ms * 1e-3) / 1e9, 1),
+            "step_frac_of_hbm": round(total / (ms * 1e-3) / 1e9 / hbm, 4),
+            "note": "E4M3 K/V with one scale each for K and V; index path unchanged (bf16 compressed keys)"}
+
+
+def run_varlen_prefill(cache, wl, dev, flush, reps: int = 20):
+    """qsa_prefill_score_topk_varlen: one call over a ragged batch of causal chunks of four requests at
+    different depths (8192 queries in all), against one qsa_prefill_score_topk call per chunk."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+
+    segs = [(0, 0, 4096), (1, 60000, 2048), (2, 110000, 1024), (3, 8000, 1024)]
+    idx_q = W.bits_to_bf16(np.concatenate([wl.idx_q(r, q0=p0, n=T) for r, p0, T in segs]), dev)
+    w = torch.from_numpy(np.concatenate([wl.w(r, q0=p0, n=T) for r, p0, T in segs])).to(dev)
+    cu = np.concatenate([[0], np.cumsum([T for _, _, T in segs])]).astype(np.int32)
+    Tall, max_len = int(cu[-1]), max(p0 + T for _, p0, T in segs)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, Tall, max_len), device=dev)
+    blocks = torch.empty(Tall, 512, dtype=torch.int32, device=dev)
+    nblocks = torch.empty(Tall, dtype=torch.int32, device=dev)
+    ws1 = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, 4096, max_len), device=dev)
+
+    def varlen():
+        Q.prefill_score_topk_varlen(cache, idx_q, w, [s[0] for s in segs], [s[1] for s in segs], cu, max_len, ws,
+                                    blocks, nblocks)
+
+    def separate():
+        for i, (r, p0, T) in enumerate(segs):
+            Q.prefill_score_topk(cache, idx_q[cu[i]:cu[i + 1]], w[cu[i]:cu[i + 1]], r, p0, ws1,
+                                 blocks[cu[i]:cu[i + 1]], nblocks[cu[i]:cu[i + 1]])
+
+    for f in (varlen, separate):
+        for _ in range(3):
+            f()
+    torch.cuda.synchronize()
+    if ws.device_error() != 0 or ws1.device_error() != 0:
+        raise RuntimeError("device error word set in the varlen prefill")
+    t_v, t_s = time_calls(varlen, reps, flush), time_calls(separate, reps, flush)
+    flops = sum(prefill_flops(p0, T) for _, p0, T in segs)
+    peak, _ = bf16_peak()
+    return {"segments": [{"req": r, "pos0": p0, "queries": T} for r, p0, T in segs],
+            "call_us": round(t_v * 1e3, 2), "one_call_per_chunk_us": round(t_s * 1e3, 2),
+            "query_tok_per_s": round(Tall / (t_v * 1e-3), 1),
+            "tflops": round(flops / (t_v * 1e-3) / 1e12, 1), "frac_of_bf16_peak": round(flops / (t_v * 1e-3) / 1e12 / peak, 4)}
+
+
+def run_split_decode(dev, reps: int = 50):
+    """Split-context decode of the 262,147-token request over 2 and 4 ranks, run as virtual ranks one after
+    another on this GPU (exchanges by stacking): each rank's compute time (scoring its pages, the merge, its
+    attention, the combine) and the bytes each exchange moves, next to qsa_decode of the whole context on one
+    GPU.  No NVLink is involved here: the exchange time is not measured."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+    from block_sparse_attention_c4_b200 import split as SP
+    import qsa_gen as G
+
+    wl = G.long_262k()
+    L = 262144
+    t = L - 1
+    raw = wl.idx_keys(0, 0, L)
+    full = W.build_cache(wl, device=dev, prefix_tokens=[L - 1])
+    knew = W.bits_to_bf16(raw[t:t + 1], dev)
+    idx_q = W.bits_to_bf16(wl.idx_q(0, q0=t, n=1), dev)
+    w = torch.from_numpy(wl.w(0, q0=t, n=1)).to(dev)
+    q = W.bits_to_bf16(wl.q(0, q0=t, n=1), dev)
+    seq_len = torch.tensor([L], dtype=torch.int32, device=dev)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_DECODE, 1, L), device=dev)
+    single = time_calls(lambda: Q.decode(full, knew, idx_q, w, q, seq_len, L, ws), reps)
+    res = {"context": L, "single_gpu_decode_us": round(single * 1e3, 2)}
+    n_pages = (L + 63) // 64
+    for world in (2, 4):
+        lo, cnt = SP.partition_pages(n_pages, world)
+        ranks = []
+        for r in range(world):
+            pt = torch.full((1, full.max_pages), -1, dtype=torch.int32, device=dev)
+            pt[0, lo[r]:lo[r] + cnt[r]] = full.page_table[0, lo[r]:lo[r] + cnt[r]]
+            # a view of the one pool whose page table maps only this rank's pages (no copy)
+            view = Q.LayerCache(full.num_slots, 1, full.max_pages, rope_theta=full.rope_theta, device="meta",
+                                page_table=pt)
+            view.kv, view.k, view.v, view.cidx, view.ring = full.kv, full.k, full.v, full.cidx, full.ring
+            view.kv_stride = full.kv_stride
+            ranks.append(SP.SplitRank(view, [lo[r]], [cnt[r]], L, device=dev))
+        cands = [rk.score(idx_q, w, seq_len) for rk in ranks]
+        stack = [torch.stack([c[i] for c in cands]) for i in range(3)]
+        blocks, nblocks = SP.merge(*stack)
+        parts = [rk.attend(q, seq_len, blocks, nblocks) for rk in ranks]
+        outs, lses = torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts])
+        torch.cuda.synchronize()
+        per_rank = []
+        for rk in ranks:
+            per_rank.append(time_calls(lambda: rk.score(idx_q, w, seq_len), reps) +
+                            time_calls(lambda: SP.merge(*stack), reps) +
+                            time_calls(lambda: rk.attend(q, seq_len, blocks, nblocks), reps) +
+                            time_calls(lambda: SP.combine(outs, lses), reps))
+        res[f"world{world}"] = {"per_rank_compute_us_max": round(max(per_rank) * 1e3, 2),
+                                "per_rank_compute_us": [round(x * 1e3, 2) for x in per_rank],
+                                "exchange_bytes_per_rank": {"candidates": 512 * 8 + 4, "attention": 16 * 128 * 2 + 16 * 4}}
+    res["note"] = ("virtual ranks on one GPU sharing one pool (each rank's page table maps only its pages); "
+                   "per-rank time = its kernels timed separately; the two all-gathers are not timed")
+    return res
 
 
 def prefill_flops(pos0: int, T: int) -> int:
@@ -478,6 +723,28 @@ def run_prefill_scorer(dev, reps: int = 20, long_context: bool = True):
     return res
 
 
+def run_prefill_chunk(dev, pos0: int, chunk: int = 8192, L: int = 262144, reps: int = 3):
+    """One causal chunk of the long-context prefill (the cache holds every index key), called `reps` times."""
+    import torch
+
+    import block_sparse_attention_c4_b200 as Q
+    import block_sparse_attention_c4_b200.workload as W
+    import qsa_gen as G
+
+    wl = G.long_262k()
+    cache = W.build_cache(wl, device=dev, prefix_tokens=[0])
+    W.append_tokens(cache, wl, 0, 0, L)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, chunk, pos0 + chunk), device=dev)
+    idx_q = W.bits_to_bf16(wl.idx_q(0, pos0, chunk), dev)
+    w = torch.from_numpy(wl.w(0, pos0, chunk)).to(dev)
+    torch.cuda.synchronize()
+    ms = time_calls(lambda: Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws), reps)
+    if ws.device_error() != 0:
+        raise RuntimeError("device error word set in the prefill chunk")
+    return {"pos0": pos0, "queries": chunk, "call_ms_mean": round(ms, 4),
+            "rows_rescored_in_full": Q.prefill_rescored_rows(ws, chunk, pos0 + chunk)}
+
+
 def run_long_prefill(dev, flush, chunk: int = 8192, L: int = 262144):
     """The 262144-token prefill in causal chunks of 8192 queries: every chunk's qsa_prefill_score_topk
     timed by CUDA events (the cache holds the index keys of all 262144 tokens; a chunk's queries only
@@ -507,7 +774,7 @@ def run_long_prefill(dev, flush, chunk: int = 8192, L: int = 262144):
     torch.cuda.synchronize()
     if ws.device_error() != 0:
         raise RuntimeError("device error word set in the long-context prefill")
-    times, rescored = [], 0
+    times, rescored, split = [], 0, np.zeros(3)
     for pos0, idx_q, w in chunks:
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -517,6 +784,16 @@ def run_long_prefill(dev, flush, chunk: int = 8192, L: int = 262144):
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
         rescored += Q.prefill_rescored_rows(ws, chunk, pos0 + chunk)
+    for pos0, idx_q, w in chunks:  # the kernel split, on separate calls (events between the kernels)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for x in ev:
+            x.record(st)
+        flush.zero_()
+        Q.set_profile_events(ev)
+        Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws, blocks, nblocks)
+        Q.set_profile_events(None)
+        torch.cuda.synchronize()
+        split += [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(3)]
     if ws.device_error() != 0:
         raise RuntimeError("device error word set in the long-context prefill")
     flops = sum(prefill_flops(pos0, chunk) for pos0, _, _ in chunks)
@@ -526,6 +803,8 @@ def run_long_prefill(dev, flush, chunk: int = 8192, L: int = 262144):
         "workload": f"prefill_L{L} in {len(chunks)} causal chunks of {chunk} queries",
         "total_ms": round(total_ms, 3),
         "chunk_ms_first_last": [round(times[0], 3), round(times[-1], 3)],
+        "kernels_ms_total": {"rotate": round(float(split[0]), 3), "score_tcgen05": round(float(split[1]), 3),
+                             "select_and_rescore": round(float(split[2]), 3)},
         "rows_rescored_in_full": rescored,
         "query_tok_per_s": round(L / (total_ms * 1e-3), 1),
         "roofline": {"kernel": "qsa_prefill_score_topk (whole calls)", "bound": "tensor", "achieved": round(ach, 1),
@@ -633,6 +912,17 @@ def main():
         res = run_reference(args, rank, world)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+    if args.prefill_chunk >= 0:
+        import torch
+
+        from block_sparse_attention_c4_b200 import build
+
+        build.build()
+        torch.cuda.set_device(local_rank)
+        if rank == 0:
+            print(json.dumps({"prefill_chunk": run_prefill_chunk(torch.device("cuda", local_rank),
+                                                                 args.prefill_chunk)}), flush=True)
         return
     if args.only_prefill:
         import torch

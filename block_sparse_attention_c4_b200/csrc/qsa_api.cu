@@ -29,7 +29,7 @@ struct WsLayout {
   size_t ready = 0;  // decode: per-row flag, selection final (scorer -> sparse GQA)
   size_t pj_q = 0, pj_k = 0, pj_w = 0;  // decode indexer: projected index queries, keys, head weights
   size_t sp_key = 0, sp_id = 0, sp_n = 0;  // split scoring: per-chunk candidates
-  int sp_chunks = 0;
+  int sp_chunks = 0, sp_chunk = 0;
   int ppc_min = 0;
   int seg_cap = 0;
   int splits_bound = 0;
@@ -72,8 +72,9 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     return at;
   };
   if (op == QSA_OP_SPLIT_SCORE) {
-    w.sp_chunks = std::max(1, ceil_div(std::max(1, max_len / QSA_BLOCK), SPLIT_CHUNK_BLOCKS));
-    if (w.sp_chunks > SPLIT_MAX_LISTS) return false;
+    w.sp_chunk = split_chunk(max_len);
+    if (w.sp_chunk == 0) return false;
+    w.sp_chunks = ceil_div(std::max(1, max_len / QSA_BLOCK), w.sp_chunk);
     w.sp_key = take((size_t)rows * w.sp_chunks * TOPK * 4);
     w.sp_id = take((size_t)rows * w.sp_chunks * TOPK * 4);
     w.sp_n = take((size_t)rows * w.sp_chunks * 4);
@@ -678,6 +679,7 @@ qsa_status qsa_split_score_topk(const qsa_cache* cache, const void* idx_q, const
   p.page_cnt = page_cnt;
   p.max_len = max_len;
   p.fr = make_freqs(cache->rope_theta);
+  p.chunk = L.sp_chunk;
   p.nchunks = L.sp_chunks;
   p.cand_key = at<uint32_t>(ws, L.sp_key);
   p.cand_id = at<int32_t>(ws, L.sp_id);

@@ -30,11 +30,10 @@
 
 namespace qsa {
 
-#ifndef QSA_GQ_STAGES
-#define QSA_GQ_STAGES 4
-#endif
+
 constexpr int GQ_TILE = 16;
-constexpr int GQ_STAGES = QSA_GQ_STAGES;
+constexpr int GQ_STAGES = 4;      // bf16 ring: 3 tiles of 16 KB in flight
+constexpr int GQ_STAGES_F8 = 8;   // fp8 ring: 7 tiles of 8 KB in flight (the gather is bound by bytes in flight)
 constexpr int GQ_ROW_BYTES = D * 2;                             // 256 B: one head of one position
 constexpr int GQ_KV_BYTES = GQ_TILE * HKV * GQ_ROW_BYTES;       // 8 KiB: K (or V) of a tile
 constexpr int GQ_STAGE_BYTES = 2 * GQ_KV_BYTES;                 // 16 KiB
@@ -53,23 +52,24 @@ constexpr int GQ_MAX_TILES = (QSA_MAX_SEL + QSA_MAX_DRAFT + GQ_TILE - 1) / GQ_TI
 template <int MT, bool F8>
 struct GqaSmem {
   static constexpr int STAGE = F8 ? GQ_STAGE_BYTES / 2 : GQ_STAGE_BYTES;  // a tile's K and V as gathered
+  static constexpr int STAGES = F8 ? GQ_STAGES_F8 : GQ_STAGES;
   static constexpr int CVT = F8 ? GQ_STAGE_BYTES : 128;
   static constexpr int QBYTES = HKV * MT * 16 * GQ_ROW_BYTES;
   static constexpr bool Q_IN_RING = QBYTES <= GQ_STAGE_BYTES;
-  alignas(128) uint8_t kv[GQ_STAGES][STAGE];  // [K|V][group][pos][row], bf16 rows swizzled
+  alignas(128) uint8_t kv[STAGES][STAGE];  // [K|V][group][pos][row], bf16 rows swizzled
   alignas(128) uint8_t cvt[2][CVT];           // fp8: converted tiles (bf16 stage layout)
   alignas(128) uint8_t qsep[Q_IN_RING ? 16 : QBYTES];
   int is_last;
-  int32_t slot[1];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
+  alignas(16) int32_t slot[4];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
   // split merge: the O partial (up to 32*MT heads x 128 fp32) in the ring area, (m, l) after it or in qsep
-  static constexpr int AREA = GQ_STAGES * STAGE + (F8 ? 2 * CVT : 0);
+  static constexpr int AREA = STAGES * STAGE + (F8 ? 2 * CVT : 0);
   static constexpr int PO_BYTES = 32 * MT * D * 4, PML_BYTES = 32 * MT * 2 * 4;
   static constexpr bool ML_IN_RING = PO_BYTES + PML_BYTES <= AREA;
   static constexpr bool CLUSTER_FITS =
       PO_BYTES <= AREA && (ML_IN_RING || (Q_IN_RING ? 16 : QBYTES) >= PML_BYTES);
   __device__ __forceinline__ uint8_t* area() { return kv[0]; }
   __device__ __forceinline__ uint8_t* qrow(int g, int rho) {
-    uint8_t* q = Q_IN_RING ? (F8 ? cvt[1] : kv[GQ_STAGES - 1]) : qsep;
+    uint8_t* q = Q_IN_RING ? (F8 ? cvt[1] : kv[STAGES - 1]) : qsep;
     return q + (g * MT * 16 + rho) * GQ_ROW_BYTES;
   }
 };
@@ -180,9 +180,34 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   };
 
   // ---- physical slots of this CTA's positions, resolved once up front ----
-  for (int j = tid; j < ntl * GQ_TILE; j += THREADS) {
-    const int jj = t_begin * GQ_TILE + j;
-    S.slot[j] = jj < ntot ? (int32_t)slot_of(p.c, req, position(jj), p.err) : -1;
+  if (p.mode == 0 && !p.extra_base) {
+    // kept blocks: the 4 positions of a block are 4 consecutive slots of one page (a page holds 16
+    // whole blocks), so one thread per block makes one selection read and one page-table read
+    // (a tile of 16 positions is 4 blocks; the tail positions 4 * floor(L/4) .. L-1 follow the blocks)
+    const int nsel = nsel4 >> 2;
+    for (int i = tid; i < ntl * (GQ_TILE / 4); i += THREADS) {
+      const int bi = t_begin * (GQ_TILE / 4) + i;  // block slot in the row's position order
+      int32_t s4[4] = {-1, -1, -1, -1};
+      if (bi < nsel) {
+        const int64_t s0 = slot_of(p.c, req, __ldcg(sel + bi) * CBLK, p.err);
+        if (s0 >= 0) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s4[e] = (int32_t)(s0 + e);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int jj = 4 * bi + e;
+          if (jj < ntot) s4[e] = (int32_t)slot_of(p.c, req, tail0 + (jj - nsel4), p.err);
+        }
+      }
+      *reinterpret_cast<int4*>(S.slot + 4 * i) = make_int4(s4[0], s4[1], s4[2], s4[3]);
+    }
+  } else {
+    for (int j = tid; j < ntl * GQ_TILE; j += THREADS) {
+      const int jj = t_begin * GQ_TILE + j;
+      S.slot[j] = jj < ntot ? (int32_t)slot_of(p.c, req, position(jj), p.err) : -1;
+    }
   }
   __syncthreads();
 
@@ -221,8 +246,9 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   };
 
   // prologue of the pipeline
+  constexpr int NST = Smem::STAGES;
 #pragma unroll
-  for (int k = 0; k < GQ_STAGES - 1; ++k) {
+  for (int k = 0; k < NST - 1; ++k) {
     if (k < ntl) issue_tile(t_begin + k, k);
     cp_async_commit();
   }
@@ -246,12 +272,12 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
   for (int it = 0; it < ntl; ++it) {
-    cp_async_wait<GQ_STAGES - 2>();
+    cp_async_wait<NST - 2>();
     __syncthreads();
-    if (it + GQ_STAGES - 1 < ntl) issue_tile(t_begin + it + GQ_STAGES - 1, (it + GQ_STAGES - 1) % GQ_STAGES);
+    if (it + NST - 1 < ntl) issue_tile(t_begin + it + NST - 1, (it + NST - 1) % NST);
     cp_async_commit();
 
-    const int stage = it % GQ_STAGES;
+    const int stage = it % NST;
     const int t = t_begin + it;
     const uint8_t* tile = S.kv[stage];
     if constexpr (F8) {  // the gathered fp8 tile -> bf16, laid out like a bf16 stage

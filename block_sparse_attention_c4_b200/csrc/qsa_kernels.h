@@ -181,7 +181,18 @@ cudaError_t launch_index_proj(const ProjParams& p, cudaStream_t st);
 
 // ---- split-context decode (qsa_split.cu) ----
 constexpr int SPLIT_MAX_LISTS = 64;  // candidate lists a merge takes: ranks, or chunks of one rank
-constexpr int SPLIT_CHUNK_BLOCKS = 8192;  // blocks one CTA of the split scorer takes
+constexpr int SPLIT_CHUNK_BLOCKS = 8192;  // most blocks one CTA of the split scorer takes
+constexpr int SPLIT_CHUNK_MIN = 1024;     // fewest
+// Blocks per CTA of the split scorer for contexts up to max_len: the smallest multiple of 16 (at least
+// SPLIT_CHUNK_MIN) that keeps a row's chunks within SPLIT_MAX_LISTS, so a rank's blocks spread over
+// many CTAs; 0 when even SPLIT_CHUNK_BLOCKS per CTA leaves too many chunks.
+inline int split_chunk(int max_len) {
+  const int nb = max_len / QSA_BLOCK > 1 ? max_len / QSA_BLOCK : 1;
+  int c = (nb + SPLIT_MAX_LISTS - 1) / SPLIT_MAX_LISTS;
+  c = (c + 15) / 16 * 16;
+  if (c < SPLIT_CHUNK_MIN) c = SPLIT_CHUNK_MIN;
+  return c <= SPLIT_CHUNK_BLOCKS ? c : 0;
+}
 struct SplitParams {
   CacheView c;                 // the rank's cache (page-table rows indexed by global logical page)
   const __nv_bfloat16* idx_q;  // [rows][4][128] unrotated index queries
@@ -191,7 +202,8 @@ struct SplitParams {
   const int32_t* page_cnt;     // [rows] pages this rank holds
   int max_len;
   RopeFreqs fr;
-  int nchunks;                 // chunks of 8192 blocks per row
+  int chunk;                   // blocks per chunk (one CTA), a multiple of 16, <= SPLIT_CHUNK_BLOCKS
+  int nchunks;                 // chunks per row
   uint32_t* cand_key;          // [rows][nchunks][512]
   int32_t* cand_id;            // [rows][nchunks][512]
   int32_t* cand_n;             // [rows][nchunks]

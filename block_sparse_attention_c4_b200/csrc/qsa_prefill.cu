@@ -385,6 +385,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const int qg = e >> 2;            // query group: queries qg*PF_QPW .. +PF_QPW-1 of the tile
     const int etid = tid - 64;        // 0 .. 32*PF_EPI_WARPS-1
     const uint32_t lt = (1u << lane) - 1u;
+    auto to_key = [](float sc) {  // order-preserving score key
+      const uint32_t u = __float_as_uint(sc);
+      return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+    };
     int m_it = 0;
     PfTile tl;
     for (int j = 0; pf_nth(p, blockIdx.x, j, tl); ++j) {
@@ -410,7 +414,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
       const int q0 = qg * PF_QPW;          // first query of this warp's group, in the tile
       const int t0 = tl.qt * PF_QT + q0;   // ... in the segment
-      int cnt = 0;                         // lane jl < PF_QPW: candidates of query q0 + jl, this quadrant
+      int cntq[PF_QPW];                    // every lane: candidates of query q0 + j in this quadrant's list
+#pragma unroll
+      for (int j2 = 0; j2 < PF_QPW; ++j2) cntq[j2] = 0;
+      // this quadrant's list of the warp's first query; query q0 + jl's list is 4 * PF_QCAP further on
+      unsigned long long* list0 = p.cand + ((int64_t)(tl.q_off + t0) * 4 + quad) * PF_QCAP;
 
       for (int k = 0; k < nk; ++k, ++m_it) {
         const int mt = pf_mt_of(k, ns);
@@ -421,6 +429,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           tc_fence_after();
           const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * PF_N + q0 * 4);
           const int b = mt * PF_M + quad * 32 + lane;  // this thread's block
+          const uint32_t nb_word = ~(uint32_t)b;       // low word of its candidates: lower block ranks first
           // which of the warp's 16 queries see this thread's block (all of them except in a tile's last
           // M-tiles), as a mask computed once per M-tile
           uint32_t vmask = 0xFFFFu;
@@ -443,33 +452,43 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
               __syncwarp();
               if (lane == 0) mbar_arrive(&S.tempty[buf]);
             }
+            // the 8 scores first (independent chains); w * max(x, 0) == (w/2) * (x + |x|) exactly (doubling
+            // and halving are exact), which keeps the ReLU on the FMA pipe; + 0 turns an underflowed -0 into +0
+            float sc[8];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
-              const int jl = half * 8 + jj;
-              // w * max(x, 0) == (w/2) * (x + |x|) exactly (doubling and halving are exact), which keeps
-              // the ReLU on the FMA pipe; + 0 turns an underflowed -0 into +0
-              const float4 w4 = S.w[q0 + jl];
+              const float4 w4 = S.w[q0 + half * 8 + jj];
               const float x0 = __uint_as_float(r[4 * jj]), x1 = __uint_as_float(r[4 * jj + 1]);
               const float x2 = __uint_as_float(r[4 * jj + 2]), x3 = __uint_as_float(r[4 * jj + 3]);
-              float sc = fmaf(w4.x, x0 + fabsf(x0), 0.f);
-              sc = fmaf(w4.y, x1 + fabsf(x1), sc);
-              sc = fmaf(w4.z, x2 + fabsf(x2), sc);
-              sc = fmaf(w4.w, x3 + fabsf(x3), sc) + 0.f;
-              const uint32_t u = __float_as_uint(sc);
-              const uint32_t key = u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);  // order-preserving
-              if (k < ns) {
-                if ((vmask >> jl) & 1u)
-                  atomicAdd(&S.hist[(q0 + jl) * PF_HIST_STRIDE + pf_bin(key, S.base[q0 + jl])], 1u);
-              } else {
-                const bool emit = sc >= S.tau[q0 + jl] && ((vmask >> jl) & 1u);
-                const unsigned m = __ballot_sync(0xffffffffu, emit);
-                if (m) {  // warp-uniform
-                  const int c = __shfl_sync(0xffffffffu, cnt, jl);
-                  const int slot = c + __popc(m & lt);
-                  if (emit && slot < PF_QCAP)
-                    p.cand[((int64_t)(tl.q_off + t0 + jl) * 4 + quad) * PF_QCAP + slot] =
-                        ((unsigned long long)key << 32) | (uint32_t)~(uint32_t)b;
-                  if (lane == jl) cnt += __popc(m);
+              float a = fmaf(w4.x, x0 + fabsf(x0), 0.f);
+              a = fmaf(w4.y, x1 + fabsf(x1), a);
+              a = fmaf(w4.z, x2 + fabsf(x2), a);
+              sc[jj] = fmaf(w4.w, x3 + fabsf(x3), a) + 0.f;
+            }
+            const uint32_t vis8 = (vmask >> (8 * half)) & 0xFFu;
+            if (k < ns) {
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj)
+                if ((vis8 >> jj) & 1u)
+                  atomicAdd(&S.hist[(q0 + half * 8 + jj) * PF_HIST_STRIDE + pf_bin(to_key(sc[jj]), S.base[q0 + half * 8 + jj])], 1u);
+            } else {
+              uint32_t em = 0u;  // queries this thread's block is a candidate of
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj) em |= (sc[jj] >= S.tau[q0 + half * 8 + jj] ? 1u : 0u) << jj;
+              em &= vis8;
+              const uint32_t qm = __reduce_or_sync(0xffffffffu, em);  // queries with a candidate in this warp
+              if (qm) {
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                  if ((qm >> jj) & 1u) {  // warp-uniform
+                    const int jl = half * 8 + jj;
+                    const bool e = (em >> jj) & 1u;
+                    const unsigned m = __ballot_sync(0xffffffffu, e);
+                    const int slot = cntq[jl] + __popc(m & lt);
+                    if (e && slot < PF_QCAP)
+                      list0[(int64_t)jl * 4 * PF_QCAP + slot] = ((unsigned long long)to_key(sc[jj]) << 32) | nb_word;
+                    cntq[jl] += __popc(m);
+                  }
                 }
               }
             }
@@ -486,7 +505,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
         }
       }
-      if (lane < PF_QPW && t0 + lane < tl.T) p.cand_n[(int64_t)(tl.q_off + t0 + lane) * 4 + quad] = cnt;
+      int mine = 0;
+#pragma unroll
+      for (int j2 = 0; j2 < PF_QPW; ++j2) mine = lane == j2 ? cntq[j2] : mine;
+      if (lane < PF_QPW && t0 + lane < tl.T) p.cand_n[(int64_t)(tl.q_off + t0 + lane) * 4 + quad] = mine;
     }
   }
   tc_fence_before();
@@ -511,9 +533,44 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 // ----------------------------------------------------------------------------
 constexpr int PS_MAX_WARPS = 8;
 constexpr int PS_TIE_CAP = 256;
+constexpr int PS_SUB_BINS = 256;   // second level: the 8 key bits below a first-level bin
+constexpr int PS_SUB_SHIFT = 11;
 
 __host__ __device__ constexpr int ps_warp_bytes(int bm_words) {
-  return PF_BINS * 4 + PS_TIE_CAP * 8 + ((bm_words + 3) / 4) * 16;
+  return PS_SUB_BINS * 4 + PS_TIE_CAP * 8 + ((bm_words + 3) / 4) * 16;
+}
+
+// Bin D of hist[0 .. NB) counted from the top: count(> D) < k <= count(>= D); `above` = count(> D).
+// The caller guarantees count(all) >= k.  One warp; lane l owns the NB/32 bins below the top NB/32*l.
+template <int NB>
+__device__ __forceinline__ void ps_top_bin(const uint32_t* hist, int k, int& D, int& above) {
+  constexpr int PER = NB / 32;
+  const int lane = threadIdx.x & 31;
+  const int top = NB - 1 - PER * lane;
+  int local = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) local += (int)hist[top - i];
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const uint32_t hit = __ballot_sync(0xffffffffu, x - local < k && x >= k);
+  const int L = __ffs(hit) - 1;
+  int c = __shfl_sync(0xffffffffu, x - local, L);
+  const int topL = NB - 1 - PER * L;
+  int d = topL - (PER - 1);
+  for (int i = 0; i < PER; ++i) {
+    const int h = (int)hist[topL - i];
+    if (c + h >= k) {
+      d = topL - i;
+      break;
+    }
+    c += h;
+  }
+  D = d;
+  above = c;
 }
 
 __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillParams p, int bm_words) {
@@ -521,8 +578,8 @@ __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillPar
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* mine = ps_raw + warp * ps_warp_bytes(bm_words);
   uint32_t* hist = reinterpret_cast<uint32_t*>(mine);
-  unsigned long long* tie = reinterpret_cast<unsigned long long*>(mine + PF_BINS * 4);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(mine + PF_BINS * 4 + PS_TIE_CAP * 8);
+  unsigned long long* tie = reinterpret_cast<unsigned long long*>(mine + PS_SUB_BINS * 4);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(mine + PS_SUB_BINS * 4 + PS_TIE_CAP * 8);
   const uint32_t lt = (1u << lane) - 1u;
   const int wpb = blockDim.x >> 5;
   const int gw = blockIdx.x * wpb + warp, nw = gridDim.x * wpb;
@@ -555,57 +612,64 @@ __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillPar
           atomicAdd(&hist[pf_bin((uint32_t)(__ldcg(lists + q * PF_QCAP + i) >> 32), base)], 1u);
       }
       __syncwarp();
-      // bin D from the top: count(> D) < 512 <= count(>= D); lane l owns bins 127-4l .. 124-4l
-      const uint4 h4 = reinterpret_cast<const uint4*>(hist)[PF_BINS / 4 - 1 - lane];
-      const int local = (int)(h4.x + h4.y + h4.z + h4.w);
-      int x = local;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, x - local < TOPK && x >= TOPK);
-      const int L = __ffs(hit) - 1;  // total >= 512, so some lane holds the crossing
-      int above = __shfl_sync(0xffffffffu, x - local, L);
-      const int topL = PF_BINS - 1 - 4 * L;
-      int D = topL - 3;
-      for (int i = 0; i < 4; ++i) {
-        const int h = (int)hist[topL - i];
-        if (above + h >= TOPK) {
-          D = topL - i;
-          break;
-        }
-        above += h;
-      }
-      const int need = TOPK - above;  // taken from bin D, >= 1
+      int D, above;
+      ps_top_bin<PF_BINS>(hist, TOPK, D, above);
+      int need = TOPK - above;  // taken from bin D, >= 1
       // ---- (2) bitmap of the blocks above bin D; bin D gathered ----
       const int words = (n + 31) >> 5;
       for (int i = lane; i < words; i += 32) bitmap[i] = 0u;
       __syncwarp();
-      int nt = 0;
-      for (int q = 0; q < 4; ++q) {
-        const int cn = __shfl_sync(0xffffffffu, cl, q);
-        for (int i0 = 0; i0 < cn; i0 += 32) {
-          const int i = i0 + lane;
-          unsigned long long e = 0ull;
-          int bn = -1;
-          if (i < cn) {
-            e = __ldcg(lists + q * PF_QCAP + i);
-            bn = pf_bin((uint32_t)(e >> 32), base);
+      auto sweep = [&](auto in_above, auto in_tie) {  // one pass: bits for in_above, in_tie gathered
+        int cnt_t = 0;
+        for (int q = 0; q < 4; ++q) {
+          const int cn = __shfl_sync(0xffffffffu, cl, q);
+          for (int i0 = 0; i0 < cn; i0 += 32) {
+            const int i = i0 + lane;
+            unsigned long long e = 0ull;
+            bool up = false, tie_e = false;
+            if (i < cn) {
+              e = __ldcg(lists + q * PF_QCAP + i);
+              up = in_above(e);
+              tie_e = in_tie(e);
+            }
+            if (up) {
+              const uint32_t blk = ~(uint32_t)e;
+              atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
+            }
+            const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
+            if (tie_e) {
+              const int slot = cnt_t + __popc(tm & lt);
+              if (slot < PS_TIE_CAP) tie[slot] = e;
+            }
+            cnt_t += __popc(tm);
           }
-          if (bn > D) {
-            const uint32_t blk = ~(uint32_t)e;
-            atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
-          }
-          const unsigned tm = __ballot_sync(0xffffffffu, bn == D);
-          if (bn == D) {
-            const int slot = nt + __popc(tm & lt);
-            if (slot < PS_TIE_CAP) tie[slot] = e;
-          }
-          nt += __popc(tm);
         }
-      }
+        return cnt_t;
+      };
+      auto bin1 = [&](unsigned long long e) { return pf_bin((uint32_t)(e >> 32), base); };
+      int nt = sweep([&](unsigned long long e) { return bin1(e) > D; },
+                     [&](unsigned long long e) { return bin1(e) == D; });
       __syncwarp();
+      if (nt > PS_TIE_CAP) {
+        // a crowded cut bin: split it by the next 8 key bits and keep only the cut sub-bin's ties
+        for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
+        __syncwarp();
+        auto sub = [](unsigned long long e) { return (int)((uint32_t)(e >> 32) >> PS_SUB_SHIFT) & (PS_SUB_BINS - 1); };
+        for (int q = 0; q < 4; ++q) {
+          const int cn = __shfl_sync(0xffffffffu, cl, q);
+          for (int i = lane; i < cn; i += 32) {
+            const unsigned long long e = __ldcg(lists + q * PF_QCAP + i);
+            if (bin1(e) == D) atomicAdd(&hist[sub(e)], 1u);
+          }
+        }
+        __syncwarp();
+        int D2, above2;
+        ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
+        need -= above2;
+        nt = sweep([&](unsigned long long e) { return bin1(e) == D && sub(e) > D2; },
+                   [&](unsigned long long e) { return bin1(e) == D && sub(e) == D2; });
+        __syncwarp();
+      }
       rescore = nt > PS_TIE_CAP || need > nt;
       if (!rescore) {
         // ---- (3) the best `need` of bin D ----

@@ -18,14 +18,16 @@
 // MMAs; A (rows) and B (features) are both read with 16-byte loads and fed to
 // the MMA in the same permuted order of the hidden dimension, so no shuffle
 // or shared-memory staging is needed.  The warps of a CTA split the hidden
-// dimension and add their tiles in shared memory in a fixed order (the result
-// does not depend on timing).
+// dimension (32 warps: one 128-dim slice each at hidden 4096, so the whole
+// product is one round of loads) and add their tiles in shared memory in a
+// fixed order (the result does not depend on timing).
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 
 namespace qsa {
 
-constexpr int PJ_WARPS = 8;        // hidden-dimension slices per CTA
+constexpr int PJ_WARPS = 32;       // hidden-dimension slices per CTA: at hidden 4096 one 128-dim load round
+                                   // per warp, so every load of the CTA is in flight at once
 constexpr int PJ_ROWS = 16;        // rows of a tile (MMA M)
 constexpr int PJ_FEAT = 8;         // features of a tile (MMA N)
 constexpr int PJ_KCHUNK = 128;     // hidden dims per load round of a warp (8 MMA k-steps)

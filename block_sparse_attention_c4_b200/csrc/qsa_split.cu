@@ -26,7 +26,7 @@ namespace qsa {
 
 constexpr int SP_WARPS = 16;
 constexpr int SP_THREADS = SP_WARPS * 32;
-constexpr int SP_CHUNK = SPLIT_CHUNK_BLOCKS;          // blocks a CTA scores (512 pages)
+constexpr int SP_CHUNK = SPLIT_CHUNK_BLOCKS;          // most blocks a CTA scores (512 pages)
 using SpCta = Group<SP_THREADS, 0>;
 
 struct SpSmem {
@@ -52,7 +52,7 @@ __device__ __forceinline__ SpRow sp_row(const SplitParams& p, int r) {
   return g;
 }
 
-// grid = (chunks, rows): chunk c of row r scores the rank's blocks [b_lo + c * SP_CHUNK, ...) and writes
+// grid = (chunks, rows): chunk c of row r scores the rank's blocks [b_lo + c * chunk, ...) and writes
 // its best min(512, n) (key, block) to slot c of the row's candidate list, in block order.
 __global__ void __launch_bounds__(SP_THREADS) k_split_score(SplitParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(SP_THREADS) k_split_score(SplitParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = blockIdx.y, c = blockIdx.x;
   const SpRow g = sp_row(p, r);
-  const int b0 = g.b_lo + c * SP_CHUNK;
-  const int n = min(SP_CHUNK, g.b_hi - b0);
+  const int b0 = g.b_lo + c * p.chunk;
+  const int n = min(p.chunk, g.b_hi - b0);
   int* slot_n = p.cand_n + (int64_t)r * p.nchunks + c;
   if (g.L < 1 || g.L > p.max_len || __ldg(p.page_lo + r) < 0 || __ldg(p.page_cnt + r) < 0) {
     if (tid == 0) {
