@@ -418,11 +418,15 @@ def extra(out: dict, name: str, fn, *args):
 
 def time_calls(fn, reps: int, flush=None):
     """Mean CUDA-event time (ms) of `fn` on the current stream over `reps` calls (L2 flushed before each
-    when `flush` is given, outside the events)."""
+    when `flush` is given, outside the events).  Without a flush the stream is first held by a device-side
+    sleep long enough for the host to enqueue every call, so that the events time the GPU's work and not
+    the host's launch cost of short calls."""
     import torch
 
     st = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    if flush is None:
+        torch.cuda._sleep(min(200_000_000, 200_000 * reps))  # ~0.1 ms of host time per call at ~2 GHz
     for k in range(reps):
         if flush is not None:
             flush.zero_()

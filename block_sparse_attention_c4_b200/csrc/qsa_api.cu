@@ -85,7 +85,7 @@ bool layout(int op, int rows, int max_len, WsLayout& w) {
     w.cap = (std::max(1, max_len / QSA_BLOCK) + 31) / 32 * 32;  // blocks of the longest row, whole words
     w.qrot = take((size_t)rows * HI * D * 2);
     w.pf_qbase = take((size_t)rows * 4);
-    w.pf_cand = take((size_t)rows * 4 * PF_QCAP * 8);
+    w.pf_cand = take((size_t)rows * PF_ROW_WORDS * 8);
     w.pf_cand_n = take((size_t)rows * 4 * 4);
     w.pf_fb_n = take(4);
     w.pf_fb_list = take((size_t)rows * 4);

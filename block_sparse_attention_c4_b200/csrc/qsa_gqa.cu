@@ -25,6 +25,8 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
 
@@ -33,7 +35,8 @@ namespace qsa {
 
 constexpr int GQ_TILE = 16;
 constexpr int GQ_STAGES = 4;      // bf16 ring: 3 tiles of 16 KB in flight
-constexpr int GQ_STAGES_F8 = 8;   // fp8 ring: 7 tiles of 8 KB in flight (the gather is bound by bytes in flight)
+constexpr int GQ_STAGES_F8 = 7;   // fp8 ring: 6 tiles of 8 KB in flight, the bf16 ring's bytes in flight (the
+                                  // gather is bound by them) at the same 3 CTAs per SM
 constexpr int GQ_ROW_BYTES = D * 2;                             // 256 B: one head of one position
 constexpr int GQ_KV_BYTES = GQ_TILE * HKV * GQ_ROW_BYTES;       // 8 KiB: K (or V) of a tile
 constexpr int GQ_STAGE_BYTES = 2 * GQ_KV_BYTES;                 // 16 KiB
@@ -57,19 +60,20 @@ struct GqaSmem {
   static constexpr int QBYTES = HKV * MT * 16 * GQ_ROW_BYTES;
   static constexpr bool Q_IN_RING = QBYTES <= GQ_STAGE_BYTES;
   alignas(128) uint8_t kv[STAGES][STAGE];  // [K|V][group][pos][row], bf16 rows swizzled
-  alignas(128) uint8_t cvt[2][CVT];           // fp8: converted tiles (bf16 stage layout)
+  alignas(128) uint8_t cvt[1][CVT];           // fp8: the converted tile (bf16 stage layout); one buffer is
+                                              // enough, the loop's first barrier ends the previous tile's reads
   alignas(128) uint8_t qsep[Q_IN_RING ? 16 : QBYTES];
   int is_last;
   alignas(16) int32_t slot[4];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
   // split merge: the O partial (up to 32*MT heads x 128 fp32) in the ring area, (m, l) after it or in qsep
-  static constexpr int AREA = STAGES * STAGE + (F8 ? 2 * CVT : 0);
+  static constexpr int AREA = STAGES * STAGE + (F8 ? CVT : 0);
   static constexpr int PO_BYTES = 32 * MT * D * 4, PML_BYTES = 32 * MT * 2 * 4;
   static constexpr bool ML_IN_RING = PO_BYTES + PML_BYTES <= AREA;
   static constexpr bool CLUSTER_FITS =
       PO_BYTES <= AREA && (ML_IN_RING || (Q_IN_RING ? 16 : QBYTES) >= PML_BYTES);
   __device__ __forceinline__ uint8_t* area() { return kv[0]; }
   __device__ __forceinline__ uint8_t* qrow(int g, int rho) {
-    uint8_t* q = Q_IN_RING ? (F8 ? cvt[1] : kv[STAGES - 1]) : qsep;
+    uint8_t* q = Q_IN_RING ? (F8 ? cvt[0] : kv[STAGES - 1]) : qsep;
     return q + (g * MT * 16 + rho) * GQ_ROW_BYTES;
   }
 };
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
     const int t = t_begin + it;
     const uint8_t* tile = S.kv[stage];
     if constexpr (F8) {  // the gathered fp8 tile -> bf16, laid out like a bf16 stage
-      uint8_t* dst0 = S.cvt[it & 1];
+      uint8_t* dst0 = S.cvt[0];
       constexpr int PER = 1024 / THREADS;
 #pragma unroll
       for (int k = 0; k < PER; ++k) {
@@ -620,37 +624,52 @@ static void choose_splits(int rows, int max_pos, int num_sms, int bound, int& sp
   tps = tiles;
 }
 
-// Clusters of `splits` CTAs that can be resident at once (device query, cached per device and
-// cluster size; the shared memory of the longest split, so an upper bound on what a launch uses).
+// Clusters of `splits` CTAs, each with `smem` bytes of dynamic shared memory, that can be resident at
+// once (device query, cached per device for a few (splits, smem) pairs).
 #ifndef QSA_GQA_CLUSTER_SLACK
 #define QSA_GQA_CLUSTER_SLACK 0  // percent of the cluster slots left free
 #endif
 template <int MT, bool F8>
-static int active_clusters(int splits) {
-  static int cache[64][GQ_CLUSTER_MAX + 1] = {};
+static int active_clusters(int splits, size_t smem) {
+  struct Entry {
+    int splits;
+    size_t smem;
+    int n;
+  };
+  constexpr int CAP = 32;
+  static Entry cache[64][CAP] = {};
+  static std::mutex mu;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || splits < 1 || splits > GQ_CLUSTER_MAX) return 0;
-  if (cache[dev][splits] == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(splits, 1);
-    cfg.blockDim = dim3(MT * 128);
-    cfg.dynamicSmemBytes = gqa_smem_bytes<MT, F8>(GQ_MAX_TILES);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_sparse_gqa<MT, F8>, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      n = 0;
-    }
-    cache[dev][splits] = n > 0 ? n : -1;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (const Entry& e : cache[dev])
+      if (e.splits == splits && e.smem == smem) return e.n;
   }
-  return max(cache[dev][splits], 0);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, 1);
+  cfg.blockDim = dim3(MT * 128);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_sparse_gqa<MT, F8>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  for (Entry& e : cache[dev])
+    if (e.splits == 0) {
+      e = Entry{splits, smem, n};
+      break;
+    }
+  return n;
 }
 
 template <int MT, bool F8>
@@ -673,7 +692,8 @@ static cudaError_t launch_mt(GqaParams p, int rows, int max_pos, int num_sms, in
     // cluster that finds no GPC with room for all its CTAs waits a whole CTA lifetime for one
     const int tiles = ceil_div(max(max_pos, 1), GQ_TILE);
     while (p.splits >= 2 &&
-           (int64_t)rows * 100 > (int64_t)active_clusters<MT, F8>(p.splits) * (100 - QSA_GQA_CLUSTER_SLACK)) {
+           (int64_t)rows * 100 > (int64_t)active_clusters<MT, F8>(p.splits, gqa_smem_bytes<MT, F8>(p.tiles_per_split)) *
+                                     (100 - QSA_GQA_CLUSTER_SLACK)) {
       --p.splits;
       p.tiles_per_split = ceil_div(tiles, p.splits);
     }

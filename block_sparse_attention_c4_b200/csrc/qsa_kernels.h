@@ -136,6 +136,16 @@ cudaError_t launch_gqa(const GqaParams& p, int rows, int max_pos, int num_sms, i
 constexpr int PF_QCAP = 512;            // candidates kept per (query, TMEM quadrant) list
 constexpr int PF_EMIT_ALL = 4 * PF_QCAP - 128;  // queries with at most this many blocks emit every block
 constexpr int PF_NO_BASE = -(1 << 30);  // a query whose scores are all <= 0 (no histogram range)
+constexpr int PF_DENSE_MAX = 8192;      // work tiles whose queries see at most this many blocks write every
+                                        // score key instead of filtered candidates
+// 8-byte words of one query row's area: its 4 candidate lists, or its dense score keys (4 bytes each)
+constexpr int PF_ROW_WORDS = 4 * PF_QCAP > PF_DENSE_MAX / 2 ? 4 * PF_QCAP : PF_DENSE_MAX / 2;
+// A work tile of 64 consecutive queries of a segment (first position pos0, T queries), tile qt: its
+// queries see at most this many blocks; the tile is dense when that is at most PF_DENSE_MAX.
+__host__ __device__ inline int pf_tile_nbv_hi(int pos0, int T, int qt) {
+  const int last = (qt + 1) * 64 < T ? (qt + 1) * 64 : T;
+  return (pos0 + last) >> 2;
+}
 
 // One sequence of a (ragged) prefill call: request req, queries at positions pos0 .. pos0+T-1, stored
 // at rows q_off .. q_off+T-1 of the call's query arrays.  The segments are listed in the order their
@@ -154,7 +164,8 @@ struct PrefillParams {
   const float* w;          // [T][4] head weights (16-byte aligned)
   __nv_bfloat16* qrot;     // [T*4][128] rotated index queries (written by the rotation kernel)
   int32_t* qbase;          // [T] histogram base of each query (rotation kernel), or PF_NO_BASE
-  unsigned long long* cand;  // [T][4][PF_QCAP] candidates (key << 32 | ~block) per TMEM quadrant
+  unsigned long long* cand;  // [T][PF_ROW_WORDS] per query row: 4 lists of PF_QCAP candidates (key << 32 | ~block),
+                             // one per TMEM quadrant; or, in a dense tile, the score key of every block (uint32)
   int32_t* cand_n;         // [T][4] candidates emitted per list (may exceed PF_QCAP: overflow)
   int32_t* sel;            // [T][512] out
   int32_t* sel_n;          // [T] out

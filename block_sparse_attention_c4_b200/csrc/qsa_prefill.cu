@@ -21,8 +21,14 @@
 // issues the MMAs, 16 epilogue warps read the accumulators.  Work tiles are
 // ordered longest first (causal imbalance) and dealt to CTAs in a snake.
 //
-// Scores never go to memory as a whole.  Per work tile the M-tiles run in two
-// phases:
+// Short contexts: a work tile whose queries see at most PF_DENSE_MAX (8192)
+// blocks writes every score key (4 bytes per pair, 128 coalesced bytes per
+// warp and query) and k_prefill_select reads them all: there a threshold would
+// pass a quarter or more of each query's blocks, and emitting candidates costs
+// the epilogue more instructions than the keys cost bytes.
+//
+// Longer contexts: scores never go to memory as a whole.  Per work tile the
+// M-tiles run in two phases:
 //   (1) sample: every 8th M-tile of the tile's visible range (a stratified
 //       sample, 1/8 of the blocks) fills, per query, a log-scale histogram of
 //       its score keys in shared memory (1/16 octave per bin, the range fixed
@@ -48,6 +54,7 @@
 namespace qsa {
 
 constexpr int PF_QT = 64;              // queries per work tile
+static_assert(PF_QT == 64, "pf_tile_nbv_hi counts 64 queries per work tile");
 constexpr int PF_N = PF_QT * HI;       // 256 MMA columns
 constexpr int PF_M = 128;              // compressed keys per M-tile
 constexpr int PF_STAGES = 3;           // A ring depth
@@ -71,7 +78,7 @@ struct __align__(1024) PfSmem {
   uint8_t b[2][PF_B_BYTES / 2];              // [K half][256 rows x 128 B]
   float4 w[PF_QT];                           // halved head weights of the work tile's queries
   uint32_t hist[PF_QT * PF_HIST_STRIDE];     // sample histograms of the work tile's queries
-  float tau[PF_QT];                          // emission thresholds (scores; -inf: every block)
+  alignas(16) float tau[PF_QT];              // emission thresholds (scores; -inf: every block)
   int32_t base[PF_QT];                       // histogram bases (bin 0 = key >> 19 at or below base)
   uint64_t full_a[PF_STAGES], empty_a[PF_STAGES], full_b, empty_b, tfull[2], tempty[2];
   uint32_t tmem_base;
@@ -165,7 +172,9 @@ __host__ __device__ constexpr uint32_t pf_idesc() {
 struct PfTile {
   int req, pos0, T, q_off, qt;
   __device__ int nbv_of(int t) const { return (pos0 + t + 1) >> 2; }
-  __device__ int nbv_hi() const { return nbv_of(min(T, (qt + 1) * PF_QT) - 1); }
+  __device__ int nbv_hi() const { return pf_tile_nbv_hi(pos0, T, qt); }
+  // every score key of the tile is written (no sample, no threshold)
+  __device__ bool dense() const { return nbv_hi() <= PF_DENSE_MAX; }
   // M-tiles of the main phase (0: every query keeps all its blocks, nothing to score)
   __device__ int mtiles() const {
     const int nb = nbv_hi();
@@ -174,7 +183,7 @@ struct PfTile {
   // M-tiles of the sample phase (0: every query of the tile emits all its blocks)
   __device__ int stiles() const {
     const int nb = nbv_hi();
-    return nb <= PF_EMIT_ALL ? 0 : ceil_div(ceil_div(nb, PF_M), PF_SAMPLE);
+    return nb <= PF_EMIT_ALL || nb <= PF_DENSE_MAX ? 0 : ceil_div(ceil_div(nb, PF_M), PF_SAMPLE);
   }
 };
 
@@ -417,8 +426,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       int cntq[PF_QPW];                    // every lane: candidates of query q0 + j in this quadrant's list
 #pragma unroll
       for (int j2 = 0; j2 < PF_QPW; ++j2) cntq[j2] = 0;
-      // this quadrant's list of the warp's first query; query q0 + jl's list is 4 * PF_QCAP further on
-      unsigned long long* list0 = p.cand + ((int64_t)(tl.q_off + t0) * 4 + quad) * PF_QCAP;
+      // this quadrant's list of the warp's first query; query q0 + jl's list is PF_ROW_WORDS further on
+      unsigned long long* list0 = p.cand + (int64_t)(tl.q_off + t0) * PF_ROW_WORDS + quad * PF_QCAP;
+      // dense tile: the score keys of the warp's first query's row; query q0 + jl's are 2 * PF_ROW_WORDS on
+      uint32_t* dkeys0 = reinterpret_cast<uint32_t*>(p.cand + (int64_t)(tl.q_off + t0) * PF_ROW_WORDS);
+      const bool dense = tl.dense();
 
       for (int k = 0; k < nk; ++k, ++m_it) {
         const int mt = pf_mt_of(k, ns);
@@ -466,15 +478,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
               sc[jj] = fmaf(w4.w, x3 + fabsf(x3), a) + 0.f;
             }
             const uint32_t vis8 = (vmask >> (8 * half)) & 0xFFu;
-            if (k < ns) {
+            if (dense) {  // every visible key, coalesced: the warp's 32 blocks of one query are 128 bytes
+#pragma unroll
+              for (int jj = 0; jj < 8; ++jj)
+                if ((vis8 >> jj) & 1u) dkeys0[(int64_t)(half * 8 + jj) * (2 * PF_ROW_WORDS) + b] = to_key(sc[jj]);
+            } else if (k < ns) {
 #pragma unroll
               for (int jj = 0; jj < 8; ++jj)
                 if ((vis8 >> jj) & 1u)
                   atomicAdd(&S.hist[(q0 + half * 8 + jj) * PF_HIST_STRIDE + pf_bin(to_key(sc[jj]), S.base[q0 + half * 8 + jj])], 1u);
             } else {
               uint32_t em = 0u;  // queries this thread's block is a candidate of
+              const float4 ta = *reinterpret_cast<const float4*>(&S.tau[q0 + half * 8]);
+              const float4 tb = *reinterpret_cast<const float4*>(&S.tau[q0 + half * 8 + 4]);
+              const float tq[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
-              for (int jj = 0; jj < 8; ++jj) em |= (sc[jj] >= S.tau[q0 + half * 8 + jj] ? 1u : 0u) << jj;
+              for (int jj = 0; jj < 8; ++jj) em |= (sc[jj] >= tq[jj] ? 1u : 0u) << jj;
               em &= vis8;
               const uint32_t qm = __reduce_or_sync(0xffffffffu, em);  // queries with a candidate in this warp
               if (qm) {
@@ -486,7 +505,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     const unsigned m = __ballot_sync(0xffffffffu, e);
                     const int slot = cntq[jl] + __popc(m & lt);
                     if (e && slot < PF_QCAP)
-                      list0[(int64_t)jl * 4 * PF_QCAP + slot] = ((unsigned long long)to_key(sc[jj]) << 32) | nb_word;
+                      list0[(int64_t)jl * PF_ROW_WORDS + slot] = ((unsigned long long)to_key(sc[jj]) << 32) | nb_word;
                     cntq[jl] += __popc(m);
                   }
                 }
@@ -520,24 +539,36 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Selection from the candidates: one warp per query row, longest rows first.
-// (1) a histogram of the candidates' bins (the scorer's log-scale bins of the
-//     query) gives the bin D holding the 512th candidate;
-// (2) one pass marks the blocks of every candidate above bin D in a block
-//     bitmap and gathers bin D's candidates;
-// (3) bin D's candidates are ranked by their whole word (key, then lower
-//     block first; words are distinct), the best `need` marked;
+// Selection: one warp per query row, longest rows first, from the row's
+// candidates (long contexts) or from all its score keys (dense tiles).
+// (1) a histogram of the keys' log-scale bins (the scorer's bins of the
+//     query; 4 times finer for a dense row) gives the bin D holding the
+//     512th key;
+// (2) one pass marks the blocks of every key above bin D in a block bitmap
+//     (a dense row: one ballot per 32 blocks) and gathers bin D's keys; when
+//     bin D holds more than the warp can gather, a second pass splits it by
+//     the next 8 key bits first;
+// (3) when many were gathered, they are split by the next 8 key bits in
+//     shared memory: the sub-bins above the cut are marked, the cut sub-bin's
+//     kept; what remains is ranked by whole word (key, then lower block
+//     first; words are distinct), the best `need` marked;
 // (4) the bitmap is written out in ascending block order.
-// Rows with fewer than 512 candidates, an overflowed list, or more ties in
-// bin D than the warp holds go to the re-scoring list.
+// Rows with fewer than 512 candidates, an overflowed list, more ties in bin D
+// than the warp holds (after the split; bin 0, which also holds the keys below
+// the histogram's range, is never split) or no score bound go to the
+// re-scoring list.
 // ----------------------------------------------------------------------------
 constexpr int PS_MAX_WARPS = 8;
 constexpr int PS_TIE_CAP = 256;
 constexpr int PS_SUB_BINS = 256;   // second level: the 8 key bits below a first-level bin
-constexpr int PS_SUB_SHIFT = 11;
+constexpr int PS_TIE_RANK = 48;    // more gathered ties than this are split by sub-bin before ranking
+constexpr int PS_U = 8;            // loads in flight per lane
+constexpr int PS_DBINS = 512;      // dense rows: bins of 1/64 octave (key >> 17), the same 8 octaves
+constexpr int PS_HIST_WORDS = PS_DBINS > PS_SUB_BINS ? PS_DBINS : PS_SUB_BINS;
+static_assert(PS_DBINS == 4 * PF_BINS && PF_BIN_SHIFT == 19, "dense bins split each candidate bin in 4");
 
 __host__ __device__ constexpr int ps_warp_bytes(int bm_words) {
-  return PS_SUB_BINS * 4 + PS_TIE_CAP * 8 + ((bm_words + 3) / 4) * 16;
+  return PS_HIST_WORDS * 4 + PS_TIE_CAP * 8 + ((bm_words + 3) / 4) * 16;
 }
 
 // Bin D of hist[0 .. NB) counted from the top: count(> D) < k <= count(>= D); `above` = count(> D).
@@ -573,14 +604,170 @@ __device__ __forceinline__ void ps_top_bin(const uint32_t* hist, int k, int& D, 
   above = c;
 }
 
+// The two row forms.  A candidate row: 4 lists (one per TMEM quadrant) of words key << 32 | ~block,
+// binned like the scorer's sample (1/16 octave).  A dense row: the score key of every block, binned
+// 4 times finer (a bin then holds a few dozen keys of a few thousand), the block being the key's index.
+template <bool DENSE>
+struct PsForm {
+  static constexpr int BINS = DENSE ? PS_DBINS : PF_BINS;
+  static constexpr int SHIFT = DENSE ? PF_BIN_SHIFT - 2 : PF_BIN_SHIFT;
+  static constexpr int SUB_SHIFT = SHIFT - 8;  // the 8 key bits below a bin's
+  int base;  // bin 0 = key >> SHIFT at or below base
+  __device__ int bin(unsigned long long e) const {
+    return min(BINS - 1, max(0, (int)((uint32_t)(e >> 32) >> SHIFT) - base));
+  }
+  __device__ static int sub(unsigned long long e) {
+    return (int)((uint32_t)(e >> 32) >> SUB_SHIFT) & (PS_SUB_BINS - 1);
+  }
+};
+
+// Exact top-512 of one row (n > 512 visible blocks) by one warp, written to sel in ascending block order.
+// Returns false when the row must be re-scored in full instead (more ties in the cut bin than the warp
+// holds, or a query without a score bound whose keys all fall in one clamped bin).
+// for_each(f) calls f(word, valid) for every entry of the row, all lanes together, PS_U loads in flight
+// per lane; for a dense row the entries come in block order, 32 consecutive blocks per call.
+template <bool DENSE, class ForEach>
+__device__ bool ps_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsigned long long* tie,
+                       uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
+  using F = PsForm<DENSE>;
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (qbase == PF_NO_BASE) return false;
+  const F f{DENSE ? 4 * qbase : qbase};
+  // ---- (1) histogram ----
+  for (int i = lane; i < F::BINS; i += 32) hist[i] = 0u;
+  __syncwarp();
+  for_each([&](unsigned long long e, bool valid, int) {
+    if (valid) atomicAdd(&hist[f.bin(e)], 1u);
+  });
+  __syncwarp();
+  int D, above;
+  ps_top_bin<F::BINS>(hist, TOPK, D, above);
+  int need = TOPK - above;  // taken from bin D, >= 1
+  // ---- (2) bitmap of the blocks above bin D; bin D gathered ----
+  const int words = (n + 31) >> 5;
+  for (int i = lane; i < words; i += 32) bitmap[i] = 0u;
+  __syncwarp();
+  auto sweep = [&](auto in_above, auto in_tie) {  // one pass: bits for in_above, in_tie gathered
+    int cnt_t = 0;
+    for_each([&](unsigned long long e, bool valid, int v0) {
+      const bool up = valid && in_above(e);
+      const bool tie_e = valid && in_tie(e);
+      if constexpr (DENSE) {  // lanes hold 32 consecutive blocks from v0: one bitmap word per ballot
+        const unsigned bw = __ballot_sync(0xffffffffu, up);
+        if (lane == 0 && bw) bitmap[v0 >> 5] |= bw;
+      } else if (up) {
+        const uint32_t blk = ~(uint32_t)e;
+        atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
+      }
+      const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
+      if (tie_e) {
+        const int slot = cnt_t + __popc(tm & lt);
+        if (slot < PS_TIE_CAP) tie[slot] = e;
+      }
+      cnt_t += __popc(tm);
+    });
+    return cnt_t;
+  };
+  int nt = sweep([&](unsigned long long e) { return f.bin(e) > D; }, [&](unsigned long long e) { return f.bin(e) == D; });
+  __syncwarp();
+  // the sub-bits order the keys of one bin only when it is not clamped: bin 0 also holds every key below
+  // the range, so it is never split
+  const bool splittable = D > 0;
+  if (nt > PS_TIE_CAP) {
+    if (!splittable) return false;
+    // a crowded cut bin: split it by the next 8 key bits and keep only the cut sub-bin's ties
+    for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
+    __syncwarp();
+    for_each([&](unsigned long long e, bool valid, int) {
+      if (valid && f.bin(e) == D) atomicAdd(&hist[F::sub(e)], 1u);
+    });
+    __syncwarp();
+    int D2, above2;
+    ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
+    need -= above2;
+    nt = sweep([&](unsigned long long e) { return f.bin(e) == D && F::sub(e) > D2; },
+               [&](unsigned long long e) { return f.bin(e) == D && F::sub(e) == D2; });
+    __syncwarp();
+  } else if (nt > PS_TIE_RANK && splittable) {
+    // many ties gathered: split them by the next 8 key bits in shared memory, so that only the cut
+    // sub-bin's are ranked pairwise (the ranking costs nt^2 / 32 steps per lane)
+    for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
+    __syncwarp();
+    for (int j = lane; j < nt; j += 32) atomicAdd(&hist[F::sub(tie[j])], 1u);
+    __syncwarp();
+    int D2, above2;
+    ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
+    need -= above2;
+    // sub-bins above D2 are kept; D2's ties are packed to the front (each chunk of 32 is read into
+    // registers before the ballot, and written only at or below its own indices)
+    int nt2 = 0;
+    for (int j0 = 0; j0 < nt; j0 += 32) {
+      const int j = j0 + lane;
+      unsigned long long e = 0ull;
+      int sb = -1;
+      if (j < nt) {
+        e = tie[j];
+        sb = F::sub(e);
+      }
+      if (sb > D2) {
+        const uint32_t blk = ~(uint32_t)e;
+        atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, sb == D2);
+      if (sb == D2) tie[nt2 + __popc(m & lt)] = e;
+      nt2 += __popc(m);
+    }
+    __syncwarp();
+    nt = nt2;
+  }
+  if (nt > PS_TIE_CAP || need > nt) return false;
+  // ---- (3) the best `need` of the cut bin's ties, by whole word (words are distinct) ----
+  for (int j = lane; j < nt; j += 32) {
+    const unsigned long long ej = tie[j];
+    int rank = 0;
+    for (int m = 0; m < nt; ++m) rank += tie[m] > ej;
+    if (rank < need) {
+      const uint32_t blk = ~(uint32_t)ej;
+      atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
+    }
+  }
+  __syncwarp();
+  // ---- (4) ascending output ----
+  int out = 0;
+  for (int w0 = 0; w0 < words; w0 += 32) {
+    const int wi = w0 + lane;
+    uint32_t bits = wi < words ? bitmap[wi] : 0u;
+    const int cn = __popc(bits);
+    int xx = cn;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, xx, o);
+      if (lane >= o) xx += y;
+    }
+    int o = out + xx - cn;
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (o < TOPK) sel[o] = wi * 32 + bit;
+      ++o;
+    }
+    out += __shfl_sync(0xffffffffu, xx, 31);
+  }
+  if (lane == 0) {
+    if (out != TOPK) set_error(err, QSA_DEVERR_SELECTION);
+    *sel_n = min(out, TOPK);
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillParams p, int bm_words) {
   extern __shared__ __align__(16) uint8_t ps_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* mine = ps_raw + warp * ps_warp_bytes(bm_words);
   uint32_t* hist = reinterpret_cast<uint32_t*>(mine);
-  unsigned long long* tie = reinterpret_cast<unsigned long long*>(mine + PS_SUB_BINS * 4);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(mine + PS_SUB_BINS * 4 + PS_TIE_CAP * 8);
-  const uint32_t lt = (1u << lane) - 1u;
+  unsigned long long* tie = reinterpret_cast<unsigned long long*>(mine + PS_HIST_WORDS * 4);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(mine + PS_HIST_WORDS * 4 + PS_TIE_CAP * 8);
   const int wpb = blockDim.x >> 5;
   const int gw = blockIdx.x * wpb + warp, nw = gridDim.x * wpb;
   for (int k = gw; k < p.T; k += nw) {
@@ -597,120 +784,54 @@ __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillPar
       if (lane == 0) p.sel_n[t] = n;
       continue;
     }
-    const int cl = lane < 4 ? p.cand_n[(int64_t)t * 4 + lane] : 0;
-    const int total = __reduce_add_sync(0xffffffffu, (unsigned)cl);
-    bool rescore = __reduce_max_sync(0xffffffffu, (unsigned)cl) > (unsigned)PF_QCAP || total < TOPK;
-    if (!rescore) {
-      const int base = p.qbase[t];
-      const unsigned long long* lists = p.cand + (int64_t)t * 4 * PF_QCAP;
-      // ---- (1) histogram ----
-      for (int i = lane; i < PF_BINS; i += 32) hist[i] = 0u;
-      __syncwarp();
-      for (int q = 0; q < 4; ++q) {
-        const int cn = __shfl_sync(0xffffffffu, cl, q);
-        for (int i = lane; i < cn; i += 32)
-          atomicAdd(&hist[pf_bin((uint32_t)(__ldcg(lists + q * PF_QCAP + i) >> 32), base)], 1u);
-      }
-      __syncwarp();
-      int D, above;
-      ps_top_bin<PF_BINS>(hist, TOPK, D, above);
-      int need = TOPK - above;  // taken from bin D, >= 1
-      // ---- (2) bitmap of the blocks above bin D; bin D gathered ----
-      const int words = (n + 31) >> 5;
-      for (int i = lane; i < words; i += 32) bitmap[i] = 0u;
-      __syncwarp();
-      auto sweep = [&](auto in_above, auto in_tie) {  // one pass: bits for in_above, in_tie gathered
-        int cnt_t = 0;
-        for (int q = 0; q < 4; ++q) {
-          const int cn = __shfl_sync(0xffffffffu, cl, q);
-          for (int i0 = 0; i0 < cn; i0 += 32) {
-            const int i = i0 + lane;
-            unsigned long long e = 0ull;
-            bool up = false, tie_e = false;
-            if (i < cn) {
-              e = __ldcg(lists + q * PF_QCAP + i);
-              up = in_above(e);
-              tie_e = in_tie(e);
-            }
-            if (up) {
-              const uint32_t blk = ~(uint32_t)e;
-              atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
-            }
-            const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
-            if (tie_e) {
-              const int slot = cnt_t + __popc(tm & lt);
-              if (slot < PS_TIE_CAP) tie[slot] = e;
-            }
-            cnt_t += __popc(tm);
-          }
-        }
-        return cnt_t;
-      };
-      auto bin1 = [&](unsigned long long e) { return pf_bin((uint32_t)(e >> 32), base); };
-      int nt = sweep([&](unsigned long long e) { return bin1(e) > D; },
-                     [&](unsigned long long e) { return bin1(e) == D; });
-      __syncwarp();
-      if (nt > PS_TIE_CAP) {
-        // a crowded cut bin: split it by the next 8 key bits and keep only the cut sub-bin's ties
-        for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
-        __syncwarp();
-        auto sub = [](unsigned long long e) { return (int)((uint32_t)(e >> 32) >> PS_SUB_SHIFT) & (PS_SUB_BINS - 1); };
-        for (int q = 0; q < 4; ++q) {
-          const int cn = __shfl_sync(0xffffffffu, cl, q);
-          for (int i = lane; i < cn; i += 32) {
-            const unsigned long long e = __ldcg(lists + q * PF_QCAP + i);
-            if (bin1(e) == D) atomicAdd(&hist[sub(e)], 1u);
-          }
-        }
-        __syncwarp();
-        int D2, above2;
-        ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
-        need -= above2;
-        nt = sweep([&](unsigned long long e) { return bin1(e) == D && sub(e) > D2; },
-                   [&](unsigned long long e) { return bin1(e) == D && sub(e) == D2; });
-        __syncwarp();
-      }
-      rescore = nt > PS_TIE_CAP || need > nt;
-      if (!rescore) {
-        // ---- (3) the best `need` of bin D ----
-        for (int j = lane; j < nt; j += 32) {
-          const unsigned long long ej = tie[j];
-          int rank = 0;
-          for (int m = 0; m < nt; ++m) rank += tie[m] > ej;
-          if (rank < need) {
-            const uint32_t blk = ~(uint32_t)ej;
-            atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
-          }
-        }
-        __syncwarp();
-        // ---- (4) ascending output ----
-        int out = 0;
-        for (int w0 = 0; w0 < words; w0 += 32) {
-          const int wi = w0 + lane;
-          uint32_t bits = wi < words ? bitmap[wi] : 0u;
-          const int cn = __popc(bits);
-          int xx = cn;
+    const unsigned long long* row = p.cand + (int64_t)t * PF_ROW_WORDS;
+    const int qbase = p.qbase[t];
+    bool done;
+    if (pf_tile_nbv_hi(sg.pos0, sg.T, (t - sg.q_off) / PF_QT) <= PF_DENSE_MAX) {
+      // a dense tile's row: the score key of every block, in block order
+      const uint32_t* keys = reinterpret_cast<const uint32_t*>(row);
+      auto for_each = [&](auto fn) {
+        for (int v0 = 0; v0 < n; v0 += 32 * PS_U) {
+          uint32_t kk[PS_U];
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, xx, o);
-            if (lane >= o) xx += y;
+          for (int u = 0; u < PS_U; ++u) {
+            const int v = v0 + u * 32 + lane;
+            kk[u] = v < n ? __ldcg(keys + v) : 0u;
           }
-          int o = out + xx - cn;
-          while (bits) {
-            const int bit = __ffs(bits) - 1;
-            bits &= bits - 1u;
-            if (o < TOPK) sel[o] = wi * 32 + bit;
-            ++o;
+#pragma unroll
+          for (int u = 0; u < PS_U; ++u) {
+            const int v = v0 + u * 32 + lane;
+            fn(((unsigned long long)kk[u] << 32) | (uint32_t)~(uint32_t)v, v < n, v0 + u * 32);
           }
-          out += __shfl_sync(0xffffffffu, xx, 31);
         }
-        if (lane == 0) {
-          if (out != TOPK) set_error(p.err, QSA_DEVERR_SELECTION);
-          p.sel_n[t] = min(out, TOPK);
-        }
+      };
+      done = ps_row<true>(for_each, n, qbase, hist, tie, bitmap, sel, p.err, p.sel_n + t);
+    } else {
+      // a candidate row: its four lists, re-scored in full when they overflowed or hold fewer than 512
+      const int cl = lane < 4 ? p.cand_n[(int64_t)t * 4 + lane] : 0;
+      const int total = (int)__reduce_add_sync(0xffffffffu, (unsigned)cl);
+      done = false;
+      if (__reduce_max_sync(0xffffffffu, (unsigned)cl) <= (unsigned)PF_QCAP && total >= TOPK) {
+        auto for_each = [&](auto fn) {
+          for (int q = 0; q < 4; ++q) {
+            const int cn = __shfl_sync(0xffffffffu, cl, q);
+            const unsigned long long* list = row + q * PF_QCAP;
+            for (int i0 = 0; i0 < cn; i0 += 32 * PS_U) {
+              unsigned long long e[PS_U];
+#pragma unroll
+              for (int u = 0; u < PS_U; ++u) {
+                const int i = i0 + u * 32 + lane;
+                e[u] = i < cn ? __ldcg(list + i) : 0ull;
+              }
+#pragma unroll
+              for (int u = 0; u < PS_U; ++u) fn(e[u], i0 + u * 32 + lane < cn, 0);
+            }
+          }
+        };
+        done = ps_row<false>(for_each, n, qbase, hist, tie, bitmap, sel, p.err, p.sel_n + t);
       }
     }
-    if (rescore && lane == 0) p.fb_list[atomicAdd(p.fb_n, 1)] = t;
+    if (!done && lane == 0) p.fb_list[atomicAdd(p.fb_n, 1)] = t;
   }
 }
 

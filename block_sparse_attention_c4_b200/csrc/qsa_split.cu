@@ -146,7 +146,9 @@ __global__ void __launch_bounds__(SP_THREADS) k_split_score(SplitParams p) {
 // Best min(512, total) of `lists` ordered lists of (key, id) candidates, emitted in list order (the
 // lists are in block order end to end, so the output is ascending and ties keep the lower block).
 // One CTA per row; list j of row r holds n[j] entries at keys/ids + (r * lists + j) * 512 when
-// row_major, else at + (j * rows + r) * 512 (the ranks' exchanged arrays).
+// row_major, else at + (j * rows + r) * 512 (the ranks' exchanged arrays).  The row's keys are first
+// packed end to end into shared memory (one coalesced pass per list), so the selection's passes read
+// shared memory; only the <= 512 emitted entries look their list up again (binary search).
 struct MergeArgs {
   const uint32_t* keys;
   const int32_t* ids;
@@ -156,11 +158,14 @@ struct MergeArgs {
   int32_t* out_id;    // [rows][512]
   int32_t* out_n;     // [rows]
 };
+constexpr int SM_THREADS = 512;
+inline size_t split_merge_smem(int lists) { return (size_t)lists * TOPK * sizeof(uint32_t); }
 
-__global__ void __launch_bounds__(256) k_split_merge(MergeArgs a) {
+__global__ void __launch_bounds__(SM_THREADS) k_split_merge(MergeArgs a) {
+  extern __shared__ uint32_t mkeys[];  // [total] the row's keys, list after list
   __shared__ FastTopScratch fs;
   __shared__ int off[SPLIT_MAX_LISTS + 1];
-  using All = Group<256, 0>;
+  using All = Group<SM_THREADS, 0>;
   const int r = blockIdx.x;
   auto idx = [&](int j) { return a.row_major ? (int64_t)r * a.lists + j : (int64_t)j * a.rows + r; };
   if (threadIdx.x == 0) {
@@ -173,24 +178,47 @@ __global__ void __launch_bounds__(256) k_split_merge(MergeArgs a) {
   }
   __syncthreads();
   const int total = off[a.lists];
-  auto locate = [&](int i) {  // virtual index -> (list, entry)
-    int j = 0;
-    while (j + 1 < a.lists && off[j + 1] <= i) ++j;
-    return idx(j) * TOPK + (i - off[j]);
-  };
   const int k = min(TOPK, total);
   if (k == 0) {
     if (threadIdx.x == 0) a.out_n[r] = 0;
     return;
   }
-  fast_topk<All>([&](int i) { return __ldg(a.keys + locate(i)); }, total, k,
+  for (int j = 0; j < a.lists; ++j) {
+    const uint32_t* src = a.keys + idx(j) * TOPK;
+    const int o = off[j], cnt = off[j + 1] - o;
+    for (int e = threadIdx.x; e < cnt; e += SM_THREADS) mkeys[o + e] = __ldg(src + e);
+  }
+  __syncthreads();
+  auto locate = [&](int i) {  // packed index -> (list, entry): the last list starting at or before i
+    int lo = 0, hi = a.lists - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    return idx(lo) * TOPK + (i - off[lo]);
+  };
+  fast_topk<All>([&](int i) { return mkeys[i]; }, total, k,
                  [&](int i, int o) {
-                   const int64_t e = locate(i);
-                   a.out_id[(int64_t)r * TOPK + o] = __ldg(a.ids + e);
-                   if (a.out_key) a.out_key[(int64_t)r * TOPK + o] = __ldg(a.keys + e);
+                   a.out_id[(int64_t)r * TOPK + o] = __ldg(a.ids + locate(i));
+                   if (a.out_key) a.out_key[(int64_t)r * TOPK + o] = mkeys[i];
                  },
                  &fs);
   if (threadIdx.x == 0) a.out_n[r] = k;
+}
+
+static cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st) {
+  static int attr_bytes[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const size_t smem = split_merge_smem(a.lists);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (attr_bytes[dev] < (int)smem) {
+    const cudaError_t e = cudaFuncSetAttribute(k_split_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_bytes[dev] = (int)smem;
+  }
+  k_split_merge<<<a.rows, SM_THREADS, smem, st>>>(a);
+  return cudaGetLastError();
 }
 
 // Positions of row r this rank attends to: the kept blocks it holds (4 positions each) and, if it
@@ -270,15 +298,13 @@ cudaError_t launch_split_score(const SplitParams& p, int rows, cudaStream_t st) 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   MergeArgs a{p.cand_key, p.cand_id, p.cand_n, p.nchunks, rows, 1, p.out_key, p.out_id, p.out_n};
-  k_split_merge<<<rows, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_merge(a, st);
 }
 
 cudaError_t launch_split_merge(const uint32_t* keys, const int32_t* ids, const int32_t* n, int world, int rows,
                                int32_t* blocks, int32_t* nblocks, cudaStream_t st) {
   MergeArgs a{keys, ids, n, world, rows, 0, nullptr, blocks, nblocks};
-  k_split_merge<<<rows, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_merge(a, st);
 }
 
 cudaError_t launch_split_positions(const SplitParams& p, const int32_t* blocks, const int32_t* nblocks, int rows,

@@ -180,10 +180,12 @@ qsa_status qsa_index_score_topk(const qsa_cache* cache, const void* idx_q, const
  * positions pos0 .. pos0+T-1 of request `req` each score their complete
  * blocks b < floor((pos+1)/4) and keep the top 512.  Same result as
  * qsa_index_score_topk on those queries; built for long chunks, where the
- * chunk's queries share every compressed-key tile.  Scores do not go to
- * memory: a sampled threshold per query lets only likely members of its top
- * 512 through as candidates, the exact top 512 is taken among them, and a row
- * the candidates cannot settle is re-scored in full (exact either way).
+ * chunk's queries share every compressed-key tile.  For queries that see
+ * more than 8192 blocks scores do not go to memory: a sampled threshold per
+ * query lets only likely members of its top 512 through as candidates, the
+ * exact top 512 is taken among them, and a row the candidates cannot settle is
+ * re-scored in full (exact either way); queries of shorter contexts write all
+ * their score keys to the workspace and select from those.
  * Blog section "Qwen Sparse Attention: Retrieve Coarsely, Attend Precisely"
  * (prefill: a GPU kernel computes the index scores, a fast top-k selects).
  *   idx_q     bf16 [T][4][128] unrotated index queries

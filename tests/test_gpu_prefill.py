@@ -28,12 +28,12 @@ def W():
     return W
 
 
-def _run(Q, W, wl, pos0, T, rows=None):
+def _run(Q, W, wl, pos0, T, rows=None, w=None):
     """Append the first pos0+T index keys, score the chunk pos0 .. pos0+T-1 on the tensor cores, and check
-    rows (default: all) against the oracle."""
+    rows (default: all) against the oracle (head weights: the workload's, or `w`)."""
     cache = W.build_cache(wl, prefix_tokens=[pos0 + T])
     idx_q = wl.idx_q(0, q0=pos0, n=T)
-    w = wl.w(0, q0=pos0, n=T)
+    w = wl.w(0, q0=pos0, n=T) if w is None else w
     ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, pos0 + T))
     blocks, nblocks = Q.prefill_score_topk(cache, W.bits_to_bf16(idx_q, "cuda"), torch.from_numpy(w).cuda(), 0,
                                            pos0, ws)
@@ -53,10 +53,26 @@ def _run(Q, W, wl, pos0, T, rows=None):
 
 
 @pytest.mark.parametrize("pos0,T", [(0, 3000), (0, 64), (0, 2100), (5000, 2000), (4097, 777), (9000, 33),
-                                    (40000, 300)])
+                                    (40000, 300), (32568, 400)])
 def test_prefill_scorer_matches_oracle_every_row(Q, W, pos0, T):
+    """(32568, 400): the chunk's first work tiles see at most 8192 blocks and write every score key, the
+    later ones filter candidates."""
     wl = G.custom_decode(41 + T, [pos0 + T])
     _run(Q, W, wl, pos0, T)
+
+
+@pytest.mark.parametrize("pos0,T", [(4000, 130), (40000, 130)])
+def test_prefill_nonpositive_and_mixed_weights(Q, W, pos0, T):
+    """Head weights of both signs (the projected weights can be negative): queries whose 4 weights are
+    all <= 0 have no positive score bound, their scores are <= 0 and their best blocks are the least
+    negative; queries with mixed signs keep a bound from their positive weights.  Every row against the
+    oracle, for short (every key written) and long (filtered candidates) contexts."""
+    wl = G.custom_decode(43 + pos0, [pos0 + T])
+    rng = np.random.default_rng(pos0 + 7)
+    w = rng.uniform(-1.0, 1.0, size=(T, 4)).astype(np.float32)
+    w[::2] = -np.abs(w[::2])  # every other query: all weights <= 0
+    w[4, :] = 0.0             # one query: every score exactly 0, all blocks tied
+    _run(Q, W, wl, pos0, T, w=w)
 
 
 def test_prefill_scorer_agrees_with_streaming_scorer(Q, W):
@@ -143,8 +159,9 @@ def test_prefill_heavy_ties(Q, W):
 def test_prefill_rows_the_candidates_cannot_settle(Q, W):
     """Blocks of the sampled M-tiles (every 8th run of 128 blocks) score high and every other block
     low, so each query's sampled threshold lets far fewer than 512 blocks through: every such row is
-    re-scored in full, and the result is still the exact top 512."""
-    nb = 8192
+    re-scored in full, and the result is still the exact top 512.  (Contexts above 8192 blocks: shorter
+    ones write every score key and never need the re-scoring.)"""
+    nb = 12288
     L = 4 * nb
     T = 96
     wl = G.custom_decode(33, [L])
