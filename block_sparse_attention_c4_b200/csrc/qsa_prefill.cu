@@ -613,94 +613,35 @@ struct PsForm {
   static constexpr int SHIFT = DENSE ? PF_BIN_SHIFT - 2 : PF_BIN_SHIFT;
   static constexpr int SUB_SHIFT = SHIFT - 8;  // the 8 key bits below a bin's
   int base;  // bin 0 = key >> SHIFT at or below base
-  __device__ int bin(unsigned long long e) const {
-    return min(BINS - 1, max(0, (int)((uint32_t)(e >> 32) >> SHIFT) - base));
-  }
+  __device__ int bin_of_key(uint32_t key) const { return min(BINS - 1, max(0, (int)(key >> SHIFT) - base)); }
+  __device__ int bin(unsigned long long e) const { return bin_of_key((uint32_t)(e >> 32)); }
   __device__ static int sub(unsigned long long e) {
     return (int)((uint32_t)(e >> 32) >> SUB_SHIFT) & (PS_SUB_BINS - 1);
   }
 };
 
-// Exact top-512 of one row (n > 512 visible blocks) by one warp, written to sel in ascending block order.
-// Returns false when the row must be re-scored in full instead (more ties in the cut bin than the warp
-// holds, or a query without a score bound whose keys all fall in one clamped bin).
-// for_each(f) calls f(word, valid) for every entry of the row, all lanes together, PS_U loads in flight
-// per lane; for a dense row the entries come in block order, 32 consecutive blocks per call.
-template <bool DENSE, class ForEach>
-__device__ bool ps_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsigned long long* tie,
-                       uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
-  using F = PsForm<DENSE>;
+// The end of a row's selection, one warp: the blocks above the cut bin are marked in the bitmap, the
+// cut bin's nt entries (words key << 32 | ~block) are in tie[], `need` of them to take.  Many ties are
+// first split by their next 8 key bits in shared memory (when the cut bin is not clamped), the rest
+// ranked pairwise; then the bitmap is written out in ascending block order.  False: the row must be
+// re-scored in full (more ties than the warp holds).
+template <class Sub>
+__device__ bool ps_finish(int nt, int need, bool splittable, Sub sub, int words, uint32_t* hist,
+                          unsigned long long* tie, uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
-  if (qbase == PF_NO_BASE) return false;
-  const F f{DENSE ? 4 * qbase : qbase};
-  // ---- (1) histogram ----
-  for (int i = lane; i < F::BINS; i += 32) hist[i] = 0u;
-  __syncwarp();
-  for_each([&](unsigned long long e, bool valid, int) {
-    if (valid) atomicAdd(&hist[f.bin(e)], 1u);
-  });
-  __syncwarp();
-  int D, above;
-  ps_top_bin<F::BINS>(hist, TOPK, D, above);
-  int need = TOPK - above;  // taken from bin D, >= 1
-  // ---- (2) bitmap of the blocks above bin D; bin D gathered ----
-  const int words = (n + 31) >> 5;
-  for (int i = lane; i < words; i += 32) bitmap[i] = 0u;
-  __syncwarp();
-  auto sweep = [&](auto in_above, auto in_tie) {  // one pass: bits for in_above, in_tie gathered
-    int cnt_t = 0;
-    for_each([&](unsigned long long e, bool valid, int v0) {
-      const bool up = valid && in_above(e);
-      const bool tie_e = valid && in_tie(e);
-      if constexpr (DENSE) {  // lanes hold 32 consecutive blocks from v0: one bitmap word per ballot
-        const unsigned bw = __ballot_sync(0xffffffffu, up);
-        if (lane == 0 && bw) bitmap[v0 >> 5] |= bw;
-      } else if (up) {
-        const uint32_t blk = ~(uint32_t)e;
-        atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
-      }
-      const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
-      if (tie_e) {
-        const int slot = cnt_t + __popc(tm & lt);
-        if (slot < PS_TIE_CAP) tie[slot] = e;
-      }
-      cnt_t += __popc(tm);
-    });
-    return cnt_t;
-  };
-  int nt = sweep([&](unsigned long long e) { return f.bin(e) > D; }, [&](unsigned long long e) { return f.bin(e) == D; });
-  __syncwarp();
-  // the sub-bits order the keys of one bin only when it is not clamped: bin 0 also holds every key below
-  // the range, so it is never split
-  const bool splittable = D > 0;
-  if (nt > PS_TIE_CAP) {
-    if (!splittable) return false;
-    // a crowded cut bin: split it by the next 8 key bits and keep only the cut sub-bin's ties
+  if (nt > PS_TIE_CAP || need > nt) return false;
+  if (nt > PS_TIE_RANK && splittable) {
+    // sub-bins above the cut sub-bin D2 are kept; D2's ties are packed to the front (each chunk of 32 is
+    // read into registers before the ballot, and written only at or below its own indices); the pairwise
+    // ranking costs nt^2 / 32 steps per lane, so it only sees D2's
     for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
     __syncwarp();
-    for_each([&](unsigned long long e, bool valid, int) {
-      if (valid && f.bin(e) == D) atomicAdd(&hist[F::sub(e)], 1u);
-    });
+    for (int j = lane; j < nt; j += 32) atomicAdd(&hist[sub(tie[j])], 1u);
     __syncwarp();
     int D2, above2;
     ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
     need -= above2;
-    nt = sweep([&](unsigned long long e) { return f.bin(e) == D && F::sub(e) > D2; },
-               [&](unsigned long long e) { return f.bin(e) == D && F::sub(e) == D2; });
-    __syncwarp();
-  } else if (nt > PS_TIE_RANK && splittable) {
-    // many ties gathered: split them by the next 8 key bits in shared memory, so that only the cut
-    // sub-bin's are ranked pairwise (the ranking costs nt^2 / 32 steps per lane)
-    for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
-    __syncwarp();
-    for (int j = lane; j < nt; j += 32) atomicAdd(&hist[F::sub(tie[j])], 1u);
-    __syncwarp();
-    int D2, above2;
-    ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
-    need -= above2;
-    // sub-bins above D2 are kept; D2's ties are packed to the front (each chunk of 32 is read into
-    // registers before the ballot, and written only at or below its own indices)
     int nt2 = 0;
     for (int j0 = 0; j0 < nt; j0 += 32) {
       const int j = j0 + lane;
@@ -708,7 +649,7 @@ __device__ bool ps_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsig
       int sb = -1;
       if (j < nt) {
         e = tie[j];
-        sb = F::sub(e);
+        sb = sub(e);
       }
       if (sb > D2) {
         const uint32_t blk = ~(uint32_t)e;
@@ -721,8 +662,7 @@ __device__ bool ps_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsig
     __syncwarp();
     nt = nt2;
   }
-  if (nt > PS_TIE_CAP || need > nt) return false;
-  // ---- (3) the best `need` of the cut bin's ties, by whole word (words are distinct) ----
+  // ---- the best `need` of the cut bin's ties, by whole word (words are distinct) ----
   for (int j = lane; j < nt; j += 32) {
     const unsigned long long ej = tie[j];
     int rank = 0;
@@ -733,7 +673,7 @@ __device__ bool ps_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsig
     }
   }
   __syncwarp();
-  // ---- (4) ascending output ----
+  // ---- ascending output ----
   int out = 0;
   for (int w0 = 0; w0 < words; w0 += 32) {
     const int wi = w0 + lane;
@@ -759,6 +699,156 @@ __device__ bool ps_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsig
     *sel_n = min(out, TOPK);
   }
   return true;
+}
+
+// Exact top-512 of a candidate row (n > 512 visible blocks) by one warp.  for_each(f) calls
+// f(word, valid) for every candidate, all lanes together, PS_U loads in flight per lane.  False: the
+// row must be re-scored in full.
+template <class ForEach>
+__device__ bool ps_candidate_row(ForEach for_each, int n, int qbase, uint32_t* hist, unsigned long long* tie,
+                                 uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
+  using F = PsForm<false>;
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (qbase == PF_NO_BASE) return false;  // no score bound: every key would fall in one clamped bin
+  const F f{qbase};
+  // ---- (1) histogram ----
+  for (int i = lane; i < F::BINS; i += 32) hist[i] = 0u;
+  __syncwarp();
+  for_each([&](unsigned long long e, bool valid) {
+    if (valid) atomicAdd(&hist[f.bin(e)], 1u);
+  });
+  __syncwarp();
+  int D, above;
+  ps_top_bin<F::BINS>(hist, TOPK, D, above);
+  int need = TOPK - above;  // taken from bin D, >= 1
+  // ---- (2) bitmap of the blocks above bin D; bin D gathered ----
+  const int words = (n + 31) >> 5;
+  for (int i = lane; i < words; i += 32) bitmap[i] = 0u;
+  __syncwarp();
+  auto sweep = [&](auto in_above, auto in_tie) {  // one pass: bits for in_above, in_tie gathered
+    int cnt_t = 0;
+    for_each([&](unsigned long long e, bool valid) {
+      const bool up = valid && in_above(e);
+      const bool tie_e = valid && in_tie(e);
+      if (up) {
+        const uint32_t blk = ~(uint32_t)e;
+        atomicOr(&bitmap[blk >> 5], 1u << (blk & 31));
+      }
+      const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
+      if (tie_e) {
+        const int slot = cnt_t + __popc(tm & lt);
+        if (slot < PS_TIE_CAP) tie[slot] = e;
+      }
+      cnt_t += __popc(tm);
+    });
+    return cnt_t;
+  };
+  int nt = sweep([&](unsigned long long e) { return f.bin(e) > D; }, [&](unsigned long long e) { return f.bin(e) == D; });
+  __syncwarp();
+  // the sub-bits order the keys of one bin only when it is not clamped: bin 0 also holds every key below
+  // the range, so it is never split
+  const bool splittable = D > 0;
+  if (nt > PS_TIE_CAP && splittable) {
+    // a crowded cut bin: split it by the next 8 key bits and keep only the cut sub-bin's ties
+    for (int i = lane; i < PS_SUB_BINS; i += 32) hist[i] = 0u;
+    __syncwarp();
+    for_each([&](unsigned long long e, bool valid) {
+      if (valid && f.bin(e) == D) atomicAdd(&hist[F::sub(e)], 1u);
+    });
+    __syncwarp();
+    int D2, above2;
+    ps_top_bin<PS_SUB_BINS>(hist, need, D2, above2);
+    need -= above2;
+    nt = sweep([&](unsigned long long e) { return f.bin(e) == D && F::sub(e) > D2; },
+               [&](unsigned long long e) { return f.bin(e) == D && F::sub(e) == D2; });
+    __syncwarp();
+  }
+  return ps_finish(nt, need, splittable, F::sub, words, hist, tie, bitmap, sel, err, sel_n);
+}
+
+// Exact top-512 of a dense row (n > 512 visible blocks, the score key of block b at keys[b]) by one
+// warp, in two passes over the keys read 4 per 16-byte load: (1) the histogram; (2) the cut as key
+// thresholds (the bins are monotone in the key): the bitmap words of the blocks above the cut bin are
+// built from lane masks (a 128-key chunk is 8 lanes per 32-block word), the cut bin's keys gathered.
+// False: the row must be re-scored in full (no score bound, or more keys in the cut bin than the warp
+// holds).
+__device__ bool ps_dense_row(const uint32_t* keys, int n, int qbase, uint32_t* hist, unsigned long long* tie,
+                             uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
+  using F = PsForm<true>;
+  constexpr int U = PS_U / 2;  // 16-byte loads in flight per lane
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (qbase == PF_NO_BASE) return false;
+  const F f{4 * qbase};
+  const uint4* k4 = reinterpret_cast<const uint4*>(keys);  // the row area is 16-byte aligned and holds
+  const int n4 = (n + 3) >> 2;                              // at least 4 * n4 keys
+  auto load = [&](int c0, uint4 (&r)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * 32 + lane;
+      r[u] = c < n4 ? __ldcg(k4 + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  // ---- (1) histogram ----
+  for (int i = lane; i < F::BINS; i += 32) hist[i] = 0u;
+  __syncwarp();
+  for (int c0 = 0; c0 < n4; c0 += 32 * U) {
+    uint4 r[U];
+    load(c0, r);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = 4 * (c0 + u * 32 + lane);
+      const uint32_t kk[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (v + j < n) atomicAdd(&hist[f.bin_of_key(kk[j])], 1u);
+    }
+  }
+  __syncwarp();
+  int D, above;
+  ps_top_bin<F::BINS>(hist, TOPK, D, above);
+  const int need = TOPK - above;  // taken from bin D, >= 1
+  // bin D as keys: [klo, khi); bin 0 also holds every key below the range, the top bin every key above
+  const uint32_t klo = D == 0 ? 0u : (uint32_t)(f.base + D) << F::SHIFT;
+  const bool top = D == F::BINS - 1;
+  const uint32_t khi = top ? 0xFFFFFFFFu : (uint32_t)(f.base + D + 1) << F::SHIFT;
+  // ---- (2) bitmap words of the blocks above bin D; bin D gathered ----
+  const int words = (n + 31) >> 5;
+  int nt = 0;
+  for (int c0 = 0; c0 < n4; c0 += 32 * U) {
+    uint4 r[U];
+    load(c0, r);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int cb = c0 + u * 32;  // this step's first 4-key group: blocks 4 cb .. 4 cb + 127
+      const int v = 4 * (cb + lane);
+      const uint32_t kk[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+      uint32_t m4 = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool valid = v + j < n;
+        const bool up = valid && !top && kk[j] >= khi;
+        const bool tie_e = valid && kk[j] >= klo && (top || kk[j] < khi);
+        m4 |= (up ? 1u : 0u) << j;
+        const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
+        if (tie_e) {
+          const int slot = nt + __popc(tm & lt);
+          if (slot < PS_TIE_CAP) tie[slot] = ((unsigned long long)kk[j] << 32) | (uint32_t)~(uint32_t)(v + j);
+        }
+        nt += __popc(tm);
+      }
+      // lanes 8 w .. 8 w + 7 hold the 32 blocks of word cb / 8 + w
+      uint32_t wd = m4 << (4 * (lane & 7));
+      wd |= __shfl_xor_sync(0xffffffffu, wd, 1);
+      wd |= __shfl_xor_sync(0xffffffffu, wd, 2);
+      wd |= __shfl_xor_sync(0xffffffffu, wd, 4);
+      const int wi = cb / 8 + (lane >> 3);
+      if ((lane & 7) == 0 && wi < words) bitmap[wi] = wd;
+    }
+  }
+  __syncwarp();
+  return ps_finish(nt, need, D > 0 && !top, F::sub, words, hist, tie, bitmap, sel, err, sel_n);
 }
 
 __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillParams p, int bm_words) {
@@ -789,23 +879,8 @@ __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillPar
     bool done;
     if (pf_tile_nbv_hi(sg.pos0, sg.T, (t - sg.q_off) / PF_QT) <= PF_DENSE_MAX) {
       // a dense tile's row: the score key of every block, in block order
-      const uint32_t* keys = reinterpret_cast<const uint32_t*>(row);
-      auto for_each = [&](auto fn) {
-        for (int v0 = 0; v0 < n; v0 += 32 * PS_U) {
-          uint32_t kk[PS_U];
-#pragma unroll
-          for (int u = 0; u < PS_U; ++u) {
-            const int v = v0 + u * 32 + lane;
-            kk[u] = v < n ? __ldcg(keys + v) : 0u;
-          }
-#pragma unroll
-          for (int u = 0; u < PS_U; ++u) {
-            const int v = v0 + u * 32 + lane;
-            fn(((unsigned long long)kk[u] << 32) | (uint32_t)~(uint32_t)v, v < n, v0 + u * 32);
-          }
-        }
-      };
-      done = ps_row<true>(for_each, n, qbase, hist, tie, bitmap, sel, p.err, p.sel_n + t);
+      done = ps_dense_row(reinterpret_cast<const uint32_t*>(row), n, qbase, hist, tie, bitmap, sel, p.err,
+                          p.sel_n + t);
     } else {
       // a candidate row: its four lists, re-scored in full when they overflowed or hold fewer than 512
       const int cl = lane < 4 ? p.cand_n[(int64_t)t * 4 + lane] : 0;
@@ -824,11 +899,11 @@ __global__ void __launch_bounds__(PS_MAX_WARPS * 32) k_prefill_select(PrefillPar
                 e[u] = i < cn ? __ldcg(list + i) : 0ull;
               }
 #pragma unroll
-              for (int u = 0; u < PS_U; ++u) fn(e[u], i0 + u * 32 + lane < cn, 0);
+              for (int u = 0; u < PS_U; ++u) fn(e[u], i0 + u * 32 + lane < cn);
             }
           }
         };
-        done = ps_row<false>(for_each, n, qbase, hist, tie, bitmap, sel, p.err, p.sel_n + t);
+        done = ps_candidate_row(for_each, n, qbase, hist, tie, bitmap, sel, p.err, p.sel_n + t);
       }
     }
     if (!done && lane == 0) p.fb_list[atomicAdd(p.fb_n, 1)] = t;
