@@ -718,7 +718,8 @@ def run_prefill_scorer(dev, reps: int = 20, long_context: bool = True):
                      "algorithmic_flops_per_launch": flops},
         "roofline_mma_kernel": {"kernel": "k_prefill_score", "bound": "tensor", "achieved": round(mma_ach, 1),
                                 "peak": peak, "unit": "TFLOP/s", "frac": round(mma_ach / peak, 4),
-                                "note": "includes the sample pass (1/8 extra MMA, not in the algorithmic FLOPs)"},
+                                "note": "work tiles whose queries see more than 8192 blocks also score a 1/8 sample first (MMA not in "
+                                        "the algorithmic FLOPs); at L = 32768 every tile writes all its keys"},
     }
     del cache, ws, blocks, nblocks, idx_q, w
     torch.cuda.empty_cache()
