@@ -45,23 +45,26 @@ constexpr int GQ_MAX_TILES = (QSA_MAX_SEL + QSA_MAX_DRAFT + GQ_TILE - 1) / GQ_TI
 
 // The queries (both KV groups, MT*16 rows each) are staged in shared memory only until they are
 // in registers; when they fit one tile's bf16 area they pass through the last ring stage (bf16 K/V)
-// or the second conversion buffer (fp8 K/V), which the pipeline first writes after every warp has
-// read them.  Less shared memory leaves more L1 for the loads.
+// or the V buffers (fp8 K/V), which the pipeline first writes after every warp has read them.  Less
+// shared memory leaves more L1 for the loads.
 //
 // FP8 K/V (E4M3, one scale for K and one for V): a tile is gathered as 512 B per position into a
-// half-size ring stage, then converted (exactly: every E4M3 value is a bf16 value) into one of two
-// bf16 tile buffers laid out like a bf16 stage, which the MMAs read.  The ring, then the conversion
-// buffers, are one contiguous area that the split merge reuses.
+// half-size ring stage (K rows with their 16-byte chunks swizzled).  Every E4M3 value is a bf16 value,
+// so the conversions are exact.  K is read from the stage straight into the B fragments of Q K^T
+// (4 consecutive dims per 32-bit load, the same dim order in the query's A fragments); each warp
+// converts only the half of its KV group's V that it multiplies into a bf16 buffer of its own, so no
+// CTA-wide pass or barrier sits on a tile's path.  The ring, then the V buffers, are one contiguous
+// area that the split merge reuses.
 template <int MT, bool F8>
 struct GqaSmem {
   static constexpr int STAGE = F8 ? GQ_STAGE_BYTES / 2 : GQ_STAGE_BYTES;  // a tile's K and V as gathered
   static constexpr int STAGES = F8 ? GQ_STAGES_F8 : GQ_STAGES;
-  static constexpr int CVT = F8 ? GQ_STAGE_BYTES : 128;
+  static constexpr int VBUF = GQ_TILE * (GQ_ROW_BYTES / 2);  // fp8: one warp's V half, bf16 [16 pos][64 dims]
+  static constexpr int CVT = F8 ? MT * 4 * VBUF : 128;
   static constexpr int QBYTES = HKV * MT * 16 * GQ_ROW_BYTES;
-  static constexpr bool Q_IN_RING = QBYTES <= GQ_STAGE_BYTES;
-  alignas(128) uint8_t kv[STAGES][STAGE];  // [K|V][group][pos][row], bf16 rows swizzled
-  alignas(128) uint8_t cvt[1][CVT];           // fp8: the converted tile (bf16 stage layout); one buffer is
-                                              // enough, the loop's first barrier ends the previous tile's reads
+  static constexpr bool Q_IN_RING = QBYTES <= (F8 ? CVT : GQ_STAGE_BYTES);
+  alignas(128) uint8_t kv[STAGES][STAGE];  // [K|V][group][pos][row], bf16 rows swizzled; fp8: K rows swizzled
+  alignas(128) uint8_t cvt[CVT];           // fp8: the warps' V buffers (warp w at w * VBUF), rows swizzled
   alignas(128) uint8_t qsep[Q_IN_RING ? 16 : QBYTES];
   int is_last;
   alignas(16) int32_t slot[4];  // [p.tiles_per_split * 16] physical slot of each position of this CTA (-1: none)
@@ -73,7 +76,7 @@ struct GqaSmem {
       PO_BYTES <= AREA && (ML_IN_RING || (Q_IN_RING ? 16 : QBYTES) >= PML_BYTES);
   __device__ __forceinline__ uint8_t* area() { return kv[0]; }
   __device__ __forceinline__ uint8_t* qrow(int g, int rho) {
-    uint8_t* q = Q_IN_RING ? (F8 ? cvt[0] : kv[STAGES - 1]) : qsep;
+    uint8_t* q = Q_IN_RING ? (F8 ? cvt : kv[STAGES - 1]) : qsep;
     return q + (g * MT * 16 + rho) * GQ_ROW_BYTES;
   }
 };
@@ -243,7 +246,9 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
         const int64_t sl = tslot[j];
         const uint8_t* base = reinterpret_cast<const uint8_t*>(kvsel ? p.c.v : p.c.k);
         const uint8_t* src = sl >= 0 ? base + sl * p.c.kv_stride + g * D + ch * 16 : base;
-        uint8_t* dst = dst0 + kvsel * (GQ_KV_BYTES / 2) + g * (GQ_TILE * D) + j * D + ch * 16;
+        // K rows: chunk ch of position j at chunk ch ^ (j & 7), so that the fragment loads of 8 positions
+        // at one dim offset hit 8 different bank groups
+        uint8_t* dst = dst0 + kvsel * (GQ_KV_BYTES / 2) + g * (GQ_TILE * D) + j * D + ((kvsel ? ch : ch ^ (j & 7)) << 4);
         cp_async_16(dst, src, sl >= 0 ? 16 : 0);
       }
     }
@@ -262,12 +267,24 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
   const int g = warp & 1, dh = (warp >> 1) & 1, mt = warp >> 2;
   const int gq = lane >> 2, cq = lane & 3;
   uint32_t qa[8][4];
-  {
+  if constexpr (!F8) {
     const int mtx = lane >> 3;
     const int rho = mt * 16 + (lane & 7) + ((mtx & 1) << 3);
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       ldmatrix_x4(qa[j][0], qa[j][1], qa[j][2], qa[j][3], smem_u32(S.qrow(g, rho) + swz(rho, 2 * j + (mtx >> 1))));
+  } else {
+    // k-step j, lane (gq, cq): MMA k = 2cq, 2cq+1 are dims 16j + 4cq + {0, 1}, k = 2cq+8, 2cq+9 are
+    // dims 16j + 4cq + {2, 3} (the order the K fragments are read in below)
+    const int r0 = mt * 16 + gq, r1 = r0 + 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int ch = 2 * j + (cq >> 1), off = (cq & 1) * 8;
+      qa[j][0] = *reinterpret_cast<const uint32_t*>(S.qrow(g, r0) + swz(r0, ch) + off);
+      qa[j][1] = *reinterpret_cast<const uint32_t*>(S.qrow(g, r1) + swz(r1, ch) + off);
+      qa[j][2] = *reinterpret_cast<const uint32_t*>(S.qrow(g, r0) + swz(r0, ch) + off + 4);
+      qa[j][3] = *reinterpret_cast<const uint32_t*>(S.qrow(g, r1) + swz(r1, ch) + off + 4);
+    }
   }
   const int qi0 = (mt * 16 + gq) >> 3, qi1 = (mt * 16 + gq + 8) >> 3;  // query of rows gq, gq+8
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -284,27 +301,15 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
     const int stage = it % NST;
     const int t = t_begin + it;
     const uint8_t* tile = S.kv[stage];
-    if constexpr (F8) {  // the gathered fp8 tile -> bf16, laid out like a bf16 stage
-      uint8_t* dst0 = S.cvt[0];
-      constexpr int PER = 1024 / THREADS;
-#pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        const int c = tid + k * THREADS;
-        const int kvsel = c >> 9, j = (c >> 5) & 15, gg = (c >> 4) & 1, ch = c & 15;
-        const uint2 v8 = *reinterpret_cast<const uint2*>(tile + kvsel * (GQ_KV_BYTES / 2) + gg * (GQ_TILE * D) +
-                                                         j * D + ch * 8);
-        *reinterpret_cast<uint4*>(dst0 + kvsel * GQ_KV_BYTES + gg * (GQ_TILE * GQ_ROW_BYTES) + j * GQ_ROW_BYTES +
-                                  swz(j, ch)) = e4m3x8_to_bf16x8(v8);
-      }
-      __syncthreads();
-      tile = dst0;
-    }
-    const uint8_t* kbase = tile + g * (GQ_TILE * GQ_ROW_BYTES);
-    const uint8_t* vbase = tile + GQ_KV_BYTES + g * (GQ_TILE * GQ_ROW_BYTES);
-
     // S = Q K^T : 16 rows x 16 positions
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    {
+    const uint8_t* vbase;  // this warp's V rows (bf16, rows swizzled), and the row size and chunk base
+    int vrow, vch0;
+    if constexpr (!F8) {
+      const uint8_t* kbase = tile + g * (GQ_TILE * GQ_ROW_BYTES);
+      vbase = tile + GQ_KV_BYTES + g * (GQ_TILE * GQ_ROW_BYTES);
+      vrow = GQ_ROW_BYTES;
+      vch0 = dh * 8;
       const int mtx = lane >> 3;
       const int pj = (lane & 7) + ((mtx >> 1) << 3);
 #pragma unroll
@@ -314,6 +319,36 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
         mma_bf16_16816(s[0], qa[j], b0, b1);
         mma_bf16_16816(s[1], qa[j], b2, b3);
       }
+    } else {
+      // this warp's half of its group's V (dims dh*64 .. +63) -> bf16 in its own buffer: lane l converts
+      // the 32 values of position l/2, dims dh*64 + 32 (l&1) .. +31
+      uint8_t* vb = S.cvt + warp * Smem::VBUF;
+      {
+        const int pos = lane >> 1, hf = lane & 1;
+        const uint4* src = reinterpret_cast<const uint4*>(tile + GQ_KV_BYTES / 2 + g * (GQ_TILE * D) + pos * D +
+                                                          dh * 64 + hf * 32);
+        const uint4 a = src[0], b = src[1];
+        uint8_t* dst = vb + pos * (GQ_ROW_BYTES / 2);
+        *reinterpret_cast<uint4*>(dst + swz(pos, 4 * hf + 0)) = e4m3x8_to_bf16x8(make_uint2(a.x, a.y));
+        *reinterpret_cast<uint4*>(dst + swz(pos, 4 * hf + 1)) = e4m3x8_to_bf16x8(make_uint2(a.z, a.w));
+        *reinterpret_cast<uint4*>(dst + swz(pos, 4 * hf + 2)) = e4m3x8_to_bf16x8(make_uint2(b.x, b.y));
+        *reinterpret_cast<uint4*>(dst + swz(pos, 4 * hf + 3)) = e4m3x8_to_bf16x8(make_uint2(b.z, b.w));
+      }
+      vbase = vb;
+      vrow = GQ_ROW_BYTES / 2;
+      vch0 = 0;
+      // K fragments straight from the fp8 rows: lane (gq, cq) reads dims 16j + 4cq .. +3 of positions gq
+      // and gq + 8 (chunk j of a row sits at chunk j ^ (pos & 7))
+      const uint8_t* k0 = tile + g * (GQ_TILE * D) + gq * D + 4 * cq;
+      const uint8_t* k1 = k0 + 8 * D;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(k0 + ((j ^ (gq & 7)) << 4));
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(k1 + ((j ^ (gq & 7)) << 4));
+        mma_bf16_16816(s[0], qa[j], e4m3x2_to_bf16x2((uint16_t)(w0 & 0xFFFFu)), e4m3x2_to_bf16x2((uint16_t)(w0 >> 16)));
+        mma_bf16_16816(s[1], qa[j], e4m3x2_to_bf16x2((uint16_t)(w1 & 0xFFFFu)), e4m3x2_to_bf16x2((uint16_t)(w1 >> 16)));
+      }
+      __syncwarp();  // the warp's V buffer is written
     }
     // mask, scale (log2 domain), online softmax
     float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -367,9 +402,9 @@ __global__ void __launch_bounds__(MT * 128) k_sparse_gqa(GqaParams p) {
       const int pj = (lane & 7) + ((mtx & 1) << 3);
 #pragma unroll
       for (int pp = 0; pp < 4; ++pp) {
-        const int ch = (dh * 64 + pp * 16) / 8 + (mtx >> 1);
+        const int ch = vch0 + pp * 2 + (mtx >> 1);
         uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(vbase + pj * GQ_ROW_BYTES + swz(pj, ch)));
+        ldmatrix_x4_trans(b0, b1, b2, b3, smem_u32(vbase + pj * vrow + swz(pj, ch)));
         mma_bf16_16816(o[2 * pp], pa, b0, b1);
         mma_bf16_16816(o[2 * pp + 1], pa, b2, b3);
       }
