@@ -625,14 +625,17 @@ def run_split_decode(dev, reps: int = 50):
         parts = [rk.attend(q, seq_len, blocks, nblocks) for rk in ranks]
         outs, lses = torch.stack([p[0] for p in parts]), torch.stack([p[1] for p in parts])
         torch.cuda.synchronize()
-        per_rank = []
+        per_rank, parts_us = [], []
         for rk in ranks:
-            per_rank.append(time_calls(lambda: rk.score(idx_q, w, seq_len), reps) +
-                            time_calls(lambda: SP.merge(*stack), reps) +
-                            time_calls(lambda: rk.attend(q, seq_len, blocks, nblocks), reps) +
-                            time_calls(lambda: SP.combine(outs, lses), reps))
+            parts = [time_calls(lambda: rk.score(idx_q, w, seq_len), reps),
+                     time_calls(lambda: SP.merge(*stack), reps),
+                     time_calls(lambda: rk.attend(q, seq_len, blocks, nblocks), reps),
+                     time_calls(lambda: SP.combine(outs, lses), reps)]
+            per_rank.append(sum(parts))
+            parts_us.append([round(x * 1e3, 2) for x in parts])
         res[f"world{world}"] = {"per_rank_compute_us_max": round(max(per_rank) * 1e3, 2),
                                 "per_rank_compute_us": [round(x * 1e3, 2) for x in per_rank],
+                                "rank0_score_merge_attend_combine_us": parts_us[0],
                                 "exchange_bytes_per_rank": {"candidates": 512 * 8 + 4, "attention": 16 * 128 * 2 + 16 * 4}}
     res["note"] = ("virtual ranks on one GPU sharing one pool (each rank's page table maps only its pages); "
                    "per-rank time = its kernels timed separately; the two all-gathers are not timed")

@@ -174,8 +174,9 @@ def test_long_context_262k(Q, W):
 # ---------------------------------------------------------------------------------------------
 
 def _prefill_chain(Q, W, wl, cache, pos0, T, check_rows, L_keys, comp=None):
-    """qsa_prefill_score_topk over the causal chunk pos0 .. pos0+T-1 of request 0, then
-    qsa_expand_indices and qsa_sparse_gqa over every query of the chunk.  Every row is validated;
+    """qsa_prefill_score_topk over the causal chunk pos0 .. pos0+T-1 of request 0 (twice: bitwise the
+    same kept blocks), then qsa_expand_indices and qsa_sparse_gqa over every query of the chunk.  Every
+    row is validated;
     the rows in `check_rows` (positions) are checked against the oracle: kept blocks under the
     near-tie rule, attention against the oracle run on the GPU's own selection."""
     dev = "cuda"
@@ -184,6 +185,14 @@ def _prefill_chain(Q, W, wl, cache, pos0, T, check_rows, L_keys, comp=None):
     q = W.bits_to_bf16(wl.q(0, q0=pos0, n=T), dev)
     ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, pos0 + T))
     blocks, nblocks = Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws)
+    # the same call again: the kept blocks are bitwise the same (the candidates' order in their lists
+    # varies with scheduling, the selection does not)
+    blocks2, nblocks2 = Q.prefill_score_topk(cache, idx_q, w, 0, pos0, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(nblocks, nblocks2)
+    keep = torch.arange(512, device=dev)[None, :] < nblocks[:, None]
+    assert torch.equal(torch.where(keep, blocks, -1), torch.where(keep, blocks2, -1))
+    del blocks2, nblocks2
     q_pos = torch.arange(pos0, pos0 + T, dtype=torch.int32, device=dev)
     pos, npos = Q.expand_indices(blocks, nblocks, q_pos)
     ws2 = Q.Workspace(Q.workspace_bytes(Q.OP_SPARSE_GQA, T, 2051))
