@@ -193,7 +193,7 @@ cudaError_t launch_index_proj(const ProjParams& p, cudaStream_t st);
 // ---- split-context decode (qsa_split.cu) ----
 constexpr int SPLIT_MAX_LISTS = 64;  // candidate lists a merge takes: ranks, or chunks of one rank
 constexpr int SPLIT_CHUNK_BLOCKS = 8192;  // most blocks one CTA of the split scorer takes
-constexpr int SPLIT_CHUNK_MIN = 1024;     // fewest
+constexpr int SPLIT_CHUNK_MIN = 2048;     // fewest (fewer, longer chunks: a row's merge has fewer lists)
 // Blocks per CTA of the split scorer for contexts up to max_len: the smallest multiple of 16 (at least
 // SPLIT_CHUNK_MIN) that keeps a row's chunks within SPLIT_MAX_LISTS, so a rank's blocks spread over
 // many CTAs; 0 when even SPLIT_CHUNK_BLOCKS per CTA leaves too many chunks.

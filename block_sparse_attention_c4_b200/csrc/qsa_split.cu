@@ -31,6 +31,7 @@ using SpCta = Group<SP_THREADS, 0>;
 
 struct SpSmem {
   uint32_t keys[SP_CHUNK];
+  int32_t pid[SP_CHUNK / PAGE_BLOCKS];  // physical pages of the chunk
   alignas(16) uint32_t hist[HT_WORDS];
   HistTopScratch ht;
   double cs[D / 2], sn[D / 2];
@@ -110,19 +111,21 @@ __global__ void __launch_bounds__(SP_THREADS) k_split_score(SplitParams p) {
   const int32_t* pt = p.c.page_table + (int64_t)r * p.c.max_pages;
   const uint4* cidx = reinterpret_cast<const uint4*>(p.c.cidx);
   const int np = ceil_div(n, PAGE_BLOCKS), lp0 = b0 / PAGE_BLOCKS;
-  for (int k = warp; k < np; k += SP_WARPS) {
+  // the chunk's physical pages, looked up together (-1: outside the table or the pool, flagged)
+  for (int k = tid; k < np; k += SP_THREADS) {
     const int lp = lp0 + k;
     int phys = lp < p.c.max_pages ? __ldg(pt + lp) : -1;
     if (phys < 0 || phys >= p.c.num_pages) {
-      if (lane == 0) set_error(p.err, QSA_DEVERR_PAGE);
+      set_error(p.err, QSA_DEVERR_PAGE);
       phys = -1;
     }
-    PageRegs pr;
+    S.pid[k] = phys;
+  }
+  __syncthreads();
+  // each warp scores its pages two at a time (both loads in flight before either is used)
+  auto finish = [&](int k, const PageRegs& pr, bool ok) {
     float lo = 0.f, hi = 0.f;
-    if (phys >= 0) {
-      load_page(pr, cidx + (int64_t)phys * (PAGE_BLOCKS * D / 8), g8, cq);
-      score_page(pr, bq, wa, wb, lo, hi);
-    }
+    if (ok) score_page(pr, bq, wa, wb, lo, hi);
     if (cq < 2) {
       const int local = k * PAGE_BLOCKS + g8 + 8 * cq;
       if (local < n) {
@@ -131,6 +134,15 @@ __global__ void __launch_bounds__(SP_THREADS) k_split_score(SplitParams p) {
         ht_count(S.hist, key);
       }
     }
+  };
+  for (int k = warp; k < np; k += 2 * SP_WARPS) {
+    const int k2 = k + SP_WARPS;
+    const int ph1 = S.pid[k], ph2 = k2 < np ? S.pid[k2] : -1;
+    PageRegs pr1, pr2;
+    if (ph1 >= 0) load_page(pr1, cidx + (int64_t)ph1 * (PAGE_BLOCKS * D / 8), g8, cq);
+    if (ph2 >= 0) load_page(pr2, cidx + (int64_t)ph2 * (PAGE_BLOCKS * D / 8), g8, cq);
+    finish(k, pr1, ph1 >= 0);
+    if (k2 < np) finish(k2, pr2, ph2 >= 0);
   }
   __syncthreads();
   const int k_keep = min(TOPK, n);
@@ -147,8 +159,8 @@ __global__ void __launch_bounds__(SP_THREADS) k_split_score(SplitParams p) {
 // lists are in block order end to end, so the output is ascending and ties keep the lower block).
 // One CTA per row; list j of row r holds n[j] entries at keys/ids + (r * lists + j) * 512 when
 // row_major, else at + (j * rows + r) * 512 (the ranks' exchanged arrays).  The row's keys are first
-// packed end to end into shared memory (one coalesced pass per list), so the selection's passes read
-// shared memory; only the <= 512 emitted entries look their list up again (binary search).
+// packed end to end into shared memory (all of a thread's loads in flight at once), so the selection's
+// passes read shared memory; only the <= 512 emitted entries look their list up again (binary search).
 struct MergeArgs {
   const uint32_t* keys;
   const int32_t* ids;
@@ -183,12 +195,6 @@ __global__ void __launch_bounds__(SM_THREADS) k_split_merge(MergeArgs a) {
     if (threadIdx.x == 0) a.out_n[r] = 0;
     return;
   }
-  for (int j = 0; j < a.lists; ++j) {
-    const uint32_t* src = a.keys + idx(j) * TOPK;
-    const int o = off[j], cnt = off[j + 1] - o;
-    for (int e = threadIdx.x; e < cnt; e += SM_THREADS) mkeys[o + e] = __ldg(src + e);
-  }
-  __syncthreads();
   auto locate = [&](int i) {  // packed index -> (list, entry): the last list starting at or before i
     int lo = 0, hi = a.lists - 1;
     while (lo < hi) {
@@ -197,6 +203,26 @@ __global__ void __launch_bounds__(SM_THREADS) k_split_merge(MergeArgs a) {
     }
     return idx(lo) * TOPK + (i - off[lo]);
   };
+  // one list per warp at a time, a lane's 16 loads issued before any is stored (in flight together)
+  {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int j = warp; j < a.lists; j += SM_THREADS / 32) {
+      const uint32_t* src = a.keys + idx(j) * TOPK;
+      const int o = off[j], cnt = off[j + 1] - o;
+      uint32_t kv[TOPK / 32];
+#pragma unroll
+      for (int u = 0; u < TOPK / 32; ++u) {
+        const int e = lane + 32 * u;
+        kv[u] = e < cnt ? __ldg(src + e) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < TOPK / 32; ++u) {
+        const int e = lane + 32 * u;
+        if (e < cnt) mkeys[o + e] = kv[u];
+      }
+    }
+  }
+  __syncthreads();
   fast_topk<All>([&](int i) { return mkeys[i]; }, total, k,
                  [&](int i, int o) {
                    a.out_id[(int64_t)r * TOPK + o] = __ldg(a.ids + locate(i));
