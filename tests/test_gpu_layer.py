@@ -265,6 +265,29 @@ def test_decode_edge_lengths(Q, W):
         assert len(o["pos"]) == 4 * min(lens[r] // 4, 512) + lens[r] % 4
 
 
+def test_decode_many_rows_front_end_kernel(Q, W):
+    """More rows than the scorer keeps page offsets for in shared memory (> 512): the step runs the
+    separate front-end kernel (append, rotation, page counts and their prefix) before the scorer and
+    the sparse GQA.  Every row's selection is validated; edge and seeded rows against the oracle,
+    including the appended key."""
+    rng = np.random.default_rng(29)
+    lens = rng.integers(1, 5000, 600)
+    lens[:6] = [1, 4, 2051, 2052, 2055, 4999]
+    wl = G.custom_decode(29, [int(x) for x in lens])
+    assert Q.decode_kernel_count(wl.batch) == 3
+    res = _run_decode(Q, W, wl, keep_cache=True)
+    bl, nbl = res["blocks"], res["nblocks"]
+    for r, L in enumerate(lens):
+        nb = int(L) // 4
+        assert nbl[r] == min(nb, 512), f"row {r}"
+        if nbl[r]:
+            b = bl[r, :nbl[r]]
+            assert np.all(np.diff(b) > 0) and b[0] >= 0 and b[-1] < nb, f"row {r}"
+    assert np.all(np.isfinite(res["out"]))
+    for r in sorted({0, 1, 2, 3, 4, 5, 599} | set(rng.choice(600, 8, replace=False).tolist())):
+        _check_decode_request(wl, r, res, cache=res["cache"])
+
+
 def test_decode_is_idempotent(Q, W):
     wl = G.custom_decode(27, [4097, 9000])
     res = _run_decode(Q, W, wl, keep_cache=True)
