@@ -47,6 +47,7 @@
 // k_prefill_rescore (mma.sync over its pages, exact radix top-k).  Queries
 // with at most PF_EMIT_ALL blocks skip the sample and emit every block.
 #include <mutex>
+#include <type_traits>
 
 #include "qsa_common.cuh"
 #include "qsa_kernels.h"
@@ -563,9 +564,11 @@ constexpr int PS_TIE_CAP = 256;
 constexpr int PS_SUB_BINS = 256;   // second level: the 8 key bits below a first-level bin
 constexpr int PS_TIE_RANK = 48;    // more gathered ties than this are split by sub-bin before ranking
 constexpr int PS_U = 8;            // loads in flight per lane
-constexpr int PS_DBINS = 512;      // dense rows: bins of 1/64 octave (key >> 17), the same 8 octaves
+constexpr int PS_DSPLIT_LOG = 2;                 // dense rows: 4 bins per candidate bin, i.e. 512 bins
+constexpr int PS_DSPLIT = 1 << PS_DSPLIT_LOG;     // of 1/64 octave (key >> 17) over the same 8 octaves
+constexpr int PS_DBINS = PF_BINS * PS_DSPLIT;
 constexpr int PS_HIST_WORDS = PS_DBINS > PS_SUB_BINS ? PS_DBINS : PS_SUB_BINS;
-static_assert(PS_DBINS == 4 * PF_BINS && PF_BIN_SHIFT == 19, "dense bins split each candidate bin in 4");
+static_assert(PF_BIN_SHIFT - PS_DSPLIT_LOG >= 8, "a dense bin keeps 8 key bits below it for the tie split");
 
 __host__ __device__ constexpr int ps_warp_bytes(int bm_words) {
   return PS_HIST_WORDS * 4 + PS_TIE_CAP * 8 + ((bm_words + 3) / 4) * 16;
@@ -610,10 +613,10 @@ __device__ __forceinline__ void ps_top_bin(const uint32_t* hist, int k, int& D, 
 template <bool DENSE>
 struct PsForm {
   static constexpr int BINS = DENSE ? PS_DBINS : PF_BINS;
-  static constexpr int SHIFT = DENSE ? PF_BIN_SHIFT - 2 : PF_BIN_SHIFT;
+  static constexpr int SHIFT = DENSE ? PF_BIN_SHIFT - PS_DSPLIT_LOG : PF_BIN_SHIFT;
   static constexpr int SUB_SHIFT = SHIFT - 8;  // the 8 key bits below a bin's
   int base;  // bin 0 = key >> SHIFT at or below base
-  __device__ int bin_of_key(uint32_t key) const { return min(BINS - 1, max(0, (int)(key >> SHIFT) - base)); }
+  __device__ int bin_of_key(uint32_t key) const { return __vimin_s32_relu((int)(key >> SHIFT) - base, BINS - 1); }
   __device__ int bin(unsigned long long e) const { return bin_of_key((uint32_t)(e >> 32)); }
   __device__ static int sub(unsigned long long e) {
     return (int)((uint32_t)(e >> 32) >> SUB_SHIFT) & (PS_SUB_BINS - 1);
@@ -771,16 +774,15 @@ __device__ bool ps_candidate_row(ForEach for_each, int n, int qbase, uint32_t* h
 // warp, in two passes over the keys read 4 per 16-byte load: (1) the histogram; (2) the cut as key
 // thresholds (the bins are monotone in the key): the bitmap words of the blocks above the cut bin are
 // built from lane masks (a 128-key chunk is 8 lanes per 32-block word), the cut bin's keys gathered.
-// False: the row must be re-scored in full (no score bound, or more keys in the cut bin than the warp
-// holds).
+// A step whose U x 128 keys all lie below n skips the per-key bound test.  False: the row must be
+// re-scored in full (no score bound, or more keys in the cut bin than the warp holds).
 __device__ bool ps_dense_row(const uint32_t* keys, int n, int qbase, uint32_t* hist, unsigned long long* tie,
                              uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
   using F = PsForm<true>;
   constexpr int U = PS_U / 2;  // 16-byte loads in flight per lane
   const int lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;
   if (qbase == PF_NO_BASE) return false;
-  const F f{4 * qbase};
+  const F f{qbase * PS_DSPLIT};
   const uint4* k4 = reinterpret_cast<const uint4*>(keys);  // the row area is 16-byte aligned and holds
   const int n4 = (n + 3) >> 2;                              // at least 4 * n4 keys
   auto load = [&](int c0, uint4 (&r)[U]) {
@@ -796,47 +798,67 @@ __device__ bool ps_dense_row(const uint32_t* keys, int n, int qbase, uint32_t* h
   for (int c0 = 0; c0 < n4; c0 += 32 * U) {
     uint4 r[U];
     load(c0, r);
+    if (4 * (c0 + 32 * U) <= n) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int v = 4 * (c0 + u * 32 + lane);
-      const uint32_t kk[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+      for (int u = 0; u < U; ++u) {
+        const uint32_t kk[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (v + j < n) atomicAdd(&hist[f.bin_of_key(kk[j])], 1u);
+        for (int j = 0; j < 4; ++j) atomicAdd(&hist[f.bin_of_key(kk[j])], 1u);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = 4 * (c0 + u * 32 + lane);
+        const uint32_t kk[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (v + j < n) atomicAdd(&hist[f.bin_of_key(kk[j])], 1u);
+      }
     }
   }
   __syncwarp();
   int D, above;
   ps_top_bin<F::BINS>(hist, TOPK, D, above);
   const int need = TOPK - above;  // taken from bin D, >= 1
-  // bin D as keys: [klo, khi); bin 0 also holds every key below the range, the top bin every key above
-  const uint32_t klo = D == 0 ? 0u : (uint32_t)(f.base + D) << F::SHIFT;
+  // bin D as keys klo .. khm1; above it: keys > khm1 (none when D is the top bin, which holds every key
+  // above the range); bin 0 also holds every key below the range
   const bool top = D == F::BINS - 1;
-  const uint32_t khi = top ? 0xFFFFFFFFu : (uint32_t)(f.base + D + 1) << F::SHIFT;
-  // ---- (2) bitmap words of the blocks above bin D; bin D gathered ----
+  const uint32_t klo = D == 0 ? 0u : (uint32_t)(f.base + D) << F::SHIFT;
+  const uint32_t khm1 = top ? 0xFFFFFFFFu : ((uint32_t)(f.base + D + 1) << F::SHIFT) - 1u;
+  const uint32_t span = khm1 - klo;  // key in bin D  <=>  key - klo <= span (unsigned)
+  // ---- (2) bitmap words of the blocks above bin D; bin D gathered (slots from a shared counter: the
+  // order of the gathered keys does not matter, the finishing step ranks them by whole word) ----
   const int words = (n + 31) >> 5;
-  int nt = 0;
-  for (int c0 = 0; c0 < n4; c0 += 32 * U) {
-    uint4 r[U];
-    load(c0, r);
+  unsigned* tie_count = hist;  // the histogram is no longer read
+  __syncwarp();
+  if (lane == 0) *tie_count = 0u;
+  __syncwarp();
+  auto step = [&](const uint4 (&r)[U], int c0, auto full) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int cb = c0 + u * 32;  // this step's first 4-key group: blocks 4 cb .. 4 cb + 127
       const int v = 4 * (cb + lane);
       const uint32_t kk[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
-      uint32_t m4 = 0u;
+      uint32_t m4 = 0u, t4 = 0u;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const bool valid = v + j < n;
-        const bool up = valid && !top && kk[j] >= khi;
-        const bool tie_e = valid && kk[j] >= klo && (top || kk[j] < khi);
-        m4 |= (up ? 1u : 0u) << j;
-        const unsigned tm = __ballot_sync(0xffffffffu, tie_e);
-        if (tie_e) {
-          const int slot = nt + __popc(tm & lt);
-          if (slot < PS_TIE_CAP) tie[slot] = ((unsigned long long)kk[j] << 32) | (uint32_t)~(uint32_t)(v + j);
-        }
-        nt += __popc(tm);
+        m4 |= (kk[j] > khm1 ? 1u : 0u) << j;
+        t4 |= (kk[j] - klo <= span ? 1u : 0u) << j;
+      }
+      if constexpr (!decltype(full)::value) {
+        const int rem = n - v;  // keys of this lane's group below n
+        const uint32_t vm = rem >= 4 ? 0xFu : rem <= 0 ? 0u : (1u << rem) - 1u;
+        m4 &= vm;
+        t4 &= vm;
+      }
+      if (t4 != 0u) {
+        int slot = (int)atomicAdd(tie_count, (unsigned)__popc(t4));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((t4 >> j) & 1u) {
+            if (slot < PS_TIE_CAP) tie[slot] = ((unsigned long long)kk[j] << 32) | (uint32_t)~(uint32_t)(v + j);
+            ++slot;
+          }
       }
       // lanes 8 w .. 8 w + 7 hold the 32 blocks of word cb / 8 + w
       uint32_t wd = m4 << (4 * (lane & 7));
@@ -846,8 +868,18 @@ __device__ bool ps_dense_row(const uint32_t* keys, int n, int qbase, uint32_t* h
       const int wi = cb / 8 + (lane >> 3);
       if ((lane & 7) == 0 && wi < words) bitmap[wi] = wd;
     }
+  };
+  for (int c0 = 0; c0 < n4; c0 += 32 * U) {
+    uint4 r[U];
+    load(c0, r);
+    if (4 * (c0 + 32 * U) <= n)
+      step(r, c0, std::true_type{});
+    else
+      step(r, c0, std::false_type{});
   }
   __syncwarp();
+  const int nt = (int)*tie_count;
+  __syncwarp();  // every lane has read the count before the finishing step reuses the histogram
   return ps_finish(nt, need, D > 0 && !top, F::sub, words, hist, tie, bitmap, sel, err, sel_n);
 }
 
