@@ -59,9 +59,14 @@ static_assert(PF_QT == 64, "pf_tile_nbv_hi counts 64 queries per work tile");
 constexpr int PF_N = PF_QT * HI;       // 256 MMA columns
 constexpr int PF_M = 128;              // compressed keys per M-tile
 constexpr int PF_STAGES = 3;           // A ring depth
-constexpr int PF_EPI_WARPS = 16;
-constexpr int PF_THREADS = (2 + PF_EPI_WARPS) * 32;
-constexpr int PF_QPW = PF_QT * 4 / PF_EPI_WARPS;  // queries per epilogue warp (16)
+// Epilogue warps: 16 (576 threads; two of the SM's four register-file quarters hold five warps, so
+// at most 96 registers per thread) for calls with candidate tiles, 8 (320 threads, up to 168
+// registers) when every work tile writes dense keys: there the wider warps carry 32 queries each
+// without spilling and the 32K chunk scores faster, while candidate emission needs the 16.
+constexpr int PF_EPI_WARPS_CAND = 16;
+constexpr int PF_EPI_WARPS_DENSE = 8;
+template <int EW>
+constexpr int pf_threads() { return (2 + EW) * 32; }
 constexpr int PF_A_BYTES = PF_M * D * 2;  // 32 KiB
 constexpr int PF_B_BYTES = PF_N * D * 2;  // 64 KiB
 constexpr uint32_t PF_TMEM_COLS = 512;
@@ -71,8 +76,6 @@ constexpr float PF_SAMPLE_KEEP = 0.5f;    // tau passes about 512 / PF_SAMPLE_KE
 constexpr int PF_BINS = 128;              // histogram bins per query: 8 octaves below the bound
 constexpr int PF_BIN_SHIFT = 19;          // key >> 19 = sign, exponent, 4 mantissa bits (1/16 octave)
 constexpr int PF_HIST_STRIDE = PF_BINS + 1;  // padded rows: conflict-free per-query scans
-static_assert(PF_EPI_WARPS % 4 == 0 && PF_QPW % 8 == 0, "epilogue warps cover the four TMEM quadrants evenly");
-static_assert(PF_QPW <= 32, "one lane per query of an epilogue warp holds its list counter");
 
 struct __align__(1024) PfSmem {
   uint8_t a[PF_STAGES][2][PF_A_BYTES / 2];  // [stage][K half][128 rows x 128 B], 128B-swizzled
@@ -237,10 +240,14 @@ __device__ __forceinline__ uint32_t pf_threshold(const uint32_t* hist_row, int b
   return 0u;
 }
 
-// 576 threads (18 warps), one CTA per SM: two of the SM's four register-file quarters hold five warps,
-// so the kernel gets at most 96 registers per thread
-__global__ void __launch_bounds__(PF_THREADS, 1)
+// One CTA per SM: a TMA producer warp, an MMA warp and EW epilogue warps.
+template <int EW>
+__global__ void __launch_bounds__(pf_threads<EW>(), 1)
     k_prefill_score(PrefillParams p, const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap) {
+  constexpr int PF_EPI_WARPS = EW;
+  constexpr int PF_QPW = PF_QT * 4 / EW;  // queries per epilogue warp
+  static_assert(EW % 4 == 0 && PF_QPW % 8 == 0, "epilogue warps cover the four TMEM quadrants evenly");
+  static_assert(PF_QPW <= 32, "one lane per query of an epilogue warp holds its list counter");
   extern __shared__ uint8_t smem_raw[];
   PfSmem& S = *reinterpret_cast<PfSmem*>(smem_aligned<1024>(smem_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -445,7 +452,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           const uint32_t nb_word = ~(uint32_t)b;       // low word of its candidates: lower block ranks first
           // which of the warp's 16 queries see this thread's block (all of them except in a tile's last
           // M-tiles), as a mask computed once per M-tile
-          uint32_t vmask = 0xFFFFu;
+          uint32_t vmask = PF_QPW == 32 ? 0xFFFFFFFFu : (1u << PF_QPW) - 1u;
           if (!((mt + 1) * PF_M <= tl.nbv_of(t0) && t0 + PF_QPW <= tl.T)) {
             vmask = 0u;
 #pragma unroll
@@ -480,6 +487,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             }
             const uint32_t vis8 = (vmask >> (8 * half)) & 0xFFu;
             if (dense) {  // every visible key, coalesced: the warp's 32 blocks of one query are 128 bytes
+              if (vis8 == 0xFFu) {  // no per-query test in the M-tiles every query sees
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) dkeys0[(int64_t)(half * 8 + jj) * (2 * PF_ROW_WORDS) + b] = to_key(sc[jj]);
+              } else
 #pragma unroll
               for (int jj = 0; jj < 8; ++jj)
                 if ((vis8 >> jj) & 1u) dkeys0[(int64_t)(half * 8 + jj) * (2 * PF_ROW_WORDS) + b] = to_key(sc[jj]);
@@ -1096,7 +1107,11 @@ cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, c
   cudaGetDevice(&dev);
   const size_t smem = sizeof(PfSmem) + 1024;
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k_prefill_score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_prefill_score<PF_EPI_WARPS_CAND>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_prefill_score<PF_EPI_WARPS_DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_prefill_select, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
@@ -1115,7 +1130,14 @@ cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, c
   if (e != cudaSuccess) return e;
   const int tiles = p.ntiles;
   mark(2);
-  k_prefill_score<<<std::min(num_sms, tiles), PF_THREADS, smem, st>>>(p, kmap, qmap);
+  bool all_dense = true;  // every work tile of the call writes dense keys
+  for (int i = 0; i < p.nseg; ++i)
+    all_dense = all_dense && pf_tile_nbv_hi(p.seg[i].pos0, p.seg[i].T, (p.seg[i].T - 1) / PF_QT) <= PF_DENSE_MAX;
+  if (all_dense)
+    k_prefill_score<PF_EPI_WARPS_DENSE>
+        <<<std::min(num_sms, tiles), pf_threads<PF_EPI_WARPS_DENSE>(), smem, st>>>(p, kmap, qmap);
+  else
+    k_prefill_score<PF_EPI_WARPS_CAND><<<std::min(num_sms, tiles), pf_threads<PF_EPI_WARPS_CAND>(), smem, st>>>(p, kmap, qmap);
   mark(3);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   mark(4);
