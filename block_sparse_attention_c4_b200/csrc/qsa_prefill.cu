@@ -80,7 +80,7 @@ constexpr int PF_HIST_STRIDE = PF_BINS + 1;  // padded rows: conflict-free per-q
 struct __align__(1024) PfSmem {
   uint8_t a[PF_STAGES][2][PF_A_BYTES / 2];  // [stage][K half][128 rows x 128 B], 128B-swizzled
   uint8_t b[2][PF_B_BYTES / 2];              // [K half][256 rows x 128 B]
-  float4 w[PF_QT];                           // halved head weights of the work tile's queries
+  float4 w[PF_QT];                           // halved head weights, query pairs interleaved by head
   uint32_t hist[PF_QT * PF_HIST_STRIDE];     // sample histograms of the work tile's queries
   alignas(16) float tau[PF_QT];              // emission thresholds (scores; -inf: every block)
   int32_t base[PF_QT];                       // histogram bases (bin 0 = key >> 19 at or below base)
@@ -88,6 +88,16 @@ struct __align__(1024) PfSmem {
   uint32_t tmem_base;
   int abort;  // set by the first role whose wait gives up: every role then stops issuing work
 };
+
+// Two lanes of fma.rn.f32x2: each is fmaf(a, b, c) of its lane (round to nearest, subnormals kept).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n.reg .b64 ra, rb, rc, rd;\nmov.b64 ra, {%2, %3};\nmov.b64 rb, {%4, %5};\nmov.b64 rc, {%6, %7};\n"
+      "fma.rn.f32x2 rd, ra, rb, rc;\nmov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
 
 // Histogram bin of a score key for a query whose bins start at `base` (monotone in the key).
 __device__ __forceinline__ int pf_bin(uint32_t key, int base) {
@@ -422,7 +432,14 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
           w4 = __ldg(reinterpret_cast<const float4*>(p.w) + tl.q_off + t);
           bs = __ldg(p.qbase + tl.q_off + t);
         }
-        S.w[etid] = make_float4(0.5f * w4.x, 0.5f * w4.y, 0.5f * w4.z, 0.5f * w4.w);
+        {  // query pairs interleaved: S.w[2i] = (x, x', y, y'), S.w[2i+1] = (z, z', w, w') of queries 2i, 2i+1
+          float* wf = reinterpret_cast<float*>(S.w) + (etid >> 1) * 8 + (etid & 1);
+          wf[0] = 0.5f * w4.x;
+          wf[2] = 0.5f * w4.y;
+          wf[4] = 0.5f * w4.z;
+          wf[6] = 0.5f * w4.w;
+        }
+
         S.base[etid] = bs;
         S.tau[etid] = -INFINITY;
       }
@@ -459,8 +476,8 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
             for (int jl = 0; jl < PF_QPW; ++jl)
               vmask |= (t0 + jl < tl.T && b < tl.nbv_of(t0 + jl)) ? (1u << jl) : 0u;
           }
-          // the 16 queries' 4 heads in two loads of 8 queries (32 columns each); the TMEM buffer goes back
-          // to the MMA warp once both are in registers
+          // the warp's queries' 4 heads in loads of 8 queries (32 columns each); the TMEM buffer goes back
+          // to the MMA warp once the last is in registers
 #pragma unroll
           for (int half = 0; half < PF_QPW / 8; ++half) {
             uint32_t r[32];
@@ -476,14 +493,22 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
             // and halving are exact), which keeps the ReLU on the FMA pipe; + 0 turns an underflowed -0 into +0
             float sc[8];
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const float4 w4 = S.w[q0 + half * 8 + jj];
-              const float x0 = __uint_as_float(r[4 * jj]), x1 = __uint_as_float(r[4 * jj + 1]);
-              const float x2 = __uint_as_float(r[4 * jj + 2]), x3 = __uint_as_float(r[4 * jj + 3]);
-              float a = fmaf(w4.x, x0 + fabsf(x0), 0.f);
-              a = fmaf(w4.y, x1 + fabsf(x1), a);
-              a = fmaf(w4.z, x2 + fabsf(x2), a);
-              sc[jj] = fmaf(w4.w, x3 + fabsf(x3), a) + 0.f;
+            for (int jj = 0; jj < 8; jj += 2) {  // two queries per packed FMA, heads in order from +0
+              const float4 wa = S.w[q0 + half * 8 + jj], wb = S.w[q0 + half * 8 + jj + 1];
+              float y[2][4];
+#pragma unroll
+              for (int o = 0; o < 2; ++o)
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const float x = __uint_as_float(r[4 * (jj + o) + h]);
+                  y[o][h] = x + fabsf(x);
+                }
+              float2 acc = fma2(make_float2(wa.x, wa.y), make_float2(y[0][0], y[1][0]), make_float2(0.f, 0.f));
+              acc = fma2(make_float2(wa.z, wa.w), make_float2(y[0][1], y[1][1]), acc);
+              acc = fma2(make_float2(wb.x, wb.y), make_float2(y[0][2], y[1][2]), acc);
+              acc = fma2(make_float2(wb.z, wb.w), make_float2(y[0][3], y[1][3]), acc);
+              sc[jj] = acc.x + 0.f;
+              sc[jj + 1] = acc.y + 0.f;
             }
             const uint32_t vis8 = (vmask >> (8 * half)) & 0xFFu;
             if (dense) {  // every visible key, coalesced: the warp's 32 blocks of one query are 128 bytes
