@@ -54,6 +54,7 @@ EXPORTS = [
     "qsa_set_profile_events", "qsa_decode_kernel_count", "qsa_status_string", "qsa_version",
     "qsa_prefill_score_topk", "qsa_sparse_gqa_noalloc", "qsa_check_bounded_wait", "qsa_last_error_string",
     "qsa_index_project", "qsa_decode_indexer", "qsa_decode_attend", "qsa_prefill_rescored_rows",
+    "qsa_prefill_rotated_queries",
 ]
 
 
@@ -99,6 +100,8 @@ def lib():
     L.qsa_decode_fp8.restype = ctypes.c_int
     L.qsa_prefill_rescored_rows.argtypes = [vp, i32, i32, vp]
     L.qsa_prefill_rescored_rows.restype = i32
+    L.qsa_prefill_rotated_queries.argtypes = [vp, i32, i32, vp, vp]
+    L.qsa_prefill_rotated_queries.restype = ctypes.c_int
     L.qsa_check_bounded_wait.argtypes = [cp, vp, vp, ctypes.c_uint64, vp, sz, vp]
     L.qsa_check_bounded_wait.restype = ctypes.c_int
     L.qsa_device_error.argtypes = [vp, i32, vp]
@@ -295,6 +298,17 @@ def prefill_score_topk_varlen(cache: LayerCache, idx_q, w, seg_req, seg_pos0, cu
 def prefill_rescored_rows(ws: Workspace, T: int, max_len: int, stream=None) -> int:
     """Rows of the last prefill_score_topk call on `ws` that were re-scored in full (synchronises)."""
     return int(lib().qsa_prefill_rescored_rows(ws.ptr, int(T), int(max_len), _stream(stream)))
+
+
+def prefill_rotated_queries(ws: Workspace, T: int, max_len: int, stream=None):
+    """The rotated index queries of the last prefill_score_topk call on `ws`: uint16 bf16 bits [T][4][128]
+    (synchronises)."""
+    import numpy as np
+
+    out = np.empty((int(T), 4, 128), dtype=np.uint16)
+    _check(lib().qsa_prefill_rotated_queries(ws.ptr, int(T), int(max_len), out.ctypes.data, _stream(stream)),
+           "qsa_prefill_rotated_queries")
+    return out
 
 
 def expand_indices(blocks, nblocks, q_pos, pos=None, npos=None, stream=None):

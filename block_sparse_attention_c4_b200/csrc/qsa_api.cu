@@ -316,6 +316,16 @@ int32_t qsa_prefill_rescored_rows(void* ws, int32_t T, int32_t max_len, void* st
   return v;
 }
 
+qsa_status qsa_prefill_rotated_queries(const void* ws, int32_t T, int32_t max_len, void* out, void* stream) {
+  WsLayout L;
+  if (!ws || !out || T < 1 || !layout(QSA_OP_PREFILL_SCORE_TOPK, T, max_len, L)) return QSA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(out, static_cast<const uint8_t*>(ws) + L.qrot, (size_t)T * HI * D * 2, cudaMemcpyDeviceToHost,
+                      st) != cudaSuccess)
+    return cuda_status(cudaGetLastError());
+  return cuda_status(cudaStreamSynchronize(st));
+}
+
 int32_t qsa_decode_kernel_count(int32_t batch) { return batch <= SC_ROWS_SMEM ? 2 : 3; }
 
 qsa_status qsa_compress_append(const qsa_cache* cache, const void* idx_k_new, const int32_t* cu_new,

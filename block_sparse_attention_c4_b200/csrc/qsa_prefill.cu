@@ -1039,9 +1039,31 @@ __global__ void __launch_bounds__(PB_WARPS * 32) k_prefill_rescore(PrefillParams
 // taken with 2% of slack, sets the top bin; the 127 bins below it cover
 // eight octaves at 1/16 octave each.
 // ----------------------------------------------------------------------------
-// One warp per query: lane i owns the rotation pairs (i, i+64) and (i+32, i+96)
-// of all four heads; the angles pos * inv_freq_i are taken once per query in
-// FP64 and each rotated value is rounded once to bf16.
+// One warp per query: lane i owns the rotation pairs (2i, 2i+64) and (2i+1, 2i+65) of all four heads,
+// read and written as 32-bit words of two bf16 dims; the angles pos * inv_freq_j are taken once per
+// query in FP64.
+//
+// Each rotated value is rounded once to bf16 (nearest even) from its exact value x0 c - x1 s (or
+// x0 s + x1 c) with the FP64 terms c, s.  FP32 first: with cf, sf the FP32 roundings of c and s (|c|,
+// |s| <= 1) and two more FP32 roundings, the FP32 result y lies within 2^-23 (|x0| + |x1| + |y|) +
+// 2^-149 of the exact value (each rounding at most 2^-24 relative, or 2^-150 below the normal range).
+// Rounding to bf16 is monotone, so when y minus and plus twice that bound round to the same bf16
+// value, y rounds to the exact value's; otherwise (a value that close to a rounding boundary, about
+// one in 10^4) that component is redone in FP64.
+__device__ __forceinline__ uint32_t rope_pair_bf16(float x0, float x1, float cf, float sf, double c, double s) {
+  const float y0 = fmaf(x0, cf, -(x1 * sf));
+  const float y1 = fmaf(x0, sf, x1 * cf);
+  const float m = fmaf(fabsf(x0) + fabsf(x1), 0x1p-22f, 0x1p-126f);
+  const float e0 = fmaf(fabsf(y0), 0x1p-22f, m), e1 = fmaf(fabsf(y1), 0x1p-22f, m);
+  const uint32_t b0 = pack_bf16x2(y0 - e0, y0 + e0), b1 = pack_bf16x2(y1 - e1, y1 + e1);
+  uint32_t r = pack_bf16x2(y0, y1);  // low half: the first component
+  if ((b0 >> 16) != (b0 & 0xFFFFu))
+    r = (r & 0xFFFF0000u) | f64_to_bf16_bits((double)x0 * c - (double)x1 * s);
+  if ((b1 >> 16) != (b1 & 0xFFFFu))
+    r = (r & 0x0000FFFFu) | ((uint32_t)f64_to_bf16_bits((double)x0 * s + (double)x1 * c) << 16);
+  return r;
+}
+
 constexpr int PR_WARPS = 8;
 
 __global__ void __launch_bounds__(PR_WARPS * 32) k_prefill_rotate(PrefillParams p, const __nv_bfloat16* __restrict__ idx_q,
@@ -1052,27 +1074,36 @@ __global__ void __launch_bounds__(PR_WARPS * 32) k_prefill_rotate(PrefillParams 
   if (t >= p.T) return;
   const PfSeg& sg = pf_seg_of_row(p, t);
   const double pos = (double)(sg.pos0 + (t - sg.q_off));
-  double sn[2], cs[2];
+  const uint32_t* qin = reinterpret_cast<const uint32_t*>(idx_q + (int64_t)t * HI * D) + lane;
+  uint32_t x[HI][2];  // [head][dims 2i, 2i+1 | dims 2i+64, 2i+65]
 #pragma unroll
-  for (int e = 0; e < 2; ++e) sincos(pos * fr.f[lane + 32 * e], &sn[e], &cs[e]);
-  const uint16_t* qin = reinterpret_cast<const uint16_t*>(idx_q + (int64_t)t * HI * D);
-  uint16_t* qo = reinterpret_cast<uint16_t*>(p.qrot + (int64_t)t * HI * D);
+  for (int h = 0; h < HI; ++h) {
+    x[h][0] = __ldg(qin + h * (D / 2));
+    x[h][1] = __ldg(qin + h * (D / 2) + D / 4);
+  }
+  double sn[2], cs[2];
+  float sf[2], cf[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    sincos(pos * fr.f[2 * lane + j], &sn[j], &cs[j]);
+    sf[j] = (float)sn[j];
+    cf[j] = (float)cs[j];
+  }
+  uint32_t* qo = reinterpret_cast<uint32_t*>(p.qrot + (int64_t)t * HI * D) + lane;
   float nrm2[HI];
 #pragma unroll
   for (int h = 0; h < HI; ++h) {
-    nrm2[h] = 0.f;
+    uint32_t rp[2];  // pair j: low half dim 2i+j rotated, high half dim 2i+64+j rotated
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int i = h * D + lane + 32 * e;
-      const double x0 = (double)bf16_bits_to_f32(__ldg(qin + i));
-      const double x1 = (double)bf16_bits_to_f32(__ldg(qin + i + D / 2));
-      const uint16_t y0 = f64_to_bf16_bits(x0 * cs[e] - x1 * sn[e]);
-      const uint16_t y1 = f64_to_bf16_bits(x0 * sn[e] + x1 * cs[e]);
-      qo[i] = y0;
-      qo[i + D / 2] = y1;
-      const float f0 = bf16_bits_to_f32(y0), f1 = bf16_bits_to_f32(y1);
-      nrm2[h] = fmaf(f0, f0, fmaf(f1, f1, nrm2[h]));
-    }
+    for (int j = 0; j < 2; ++j)
+      rp[j] = rope_pair_bf16(__uint_as_float(x[h][0] << (16 - 16 * j) & 0xFFFF0000u),
+                             __uint_as_float(x[h][1] << (16 - 16 * j) & 0xFFFF0000u), cf[j], sf[j], cs[j], sn[j]);
+    const uint32_t lo = __byte_perm(rp[0], rp[1], 0x5410), hi = __byte_perm(rp[0], rp[1], 0x7632);
+    qo[h * (D / 2)] = lo;
+    qo[h * (D / 2) + D / 4] = hi;
+    const float a0 = __uint_as_float(lo << 16), a1 = __uint_as_float(lo & 0xFFFF0000u);
+    const float b0 = __uint_as_float(hi << 16), b1 = __uint_as_float(hi & 0xFFFF0000u);
+    nrm2[h] = fmaf(a0, a0, fmaf(b0, b0, fmaf(a1, a1, b1 * b1)));
   }
 #pragma unroll
   for (int h = 0; h < HI; ++h)

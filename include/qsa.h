@@ -491,6 +491,18 @@ void qsa_set_profile_events(void* const* events, int32_t n_pairs);
  */
 int32_t qsa_prefill_rescored_rows(void* ws, int32_t T, int32_t max_len, void* stream);
 
+/*
+ * Measurement hook of qsa_prefill_score_topk: copies the rotated index queries
+ * of the last call made with workspace `ws` (sized for T queries and contexts
+ * up to max_len), bf16 [T][4][128] as uint16 bit patterns, into `out`, a HOST
+ * buffer of T*4*128*2 bytes owned by the caller, so that the rotation can be
+ * checked against its plain definition (blog section "Qwen Sparse Attention:
+ * Retrieve Coarsely, Attend Precisely": the index query is rotated at its own
+ * position).  Synchronises `stream`.  QSA_ERR_INVALID_ARG for a null pointer or
+ * sizes no workspace layout has; QSA_ERR_CUDA when the copy fails.
+ */
+qsa_status qsa_prefill_rotated_queries(const void* ws, int32_t T, int32_t max_len, void* out, void* stream);
+
 /* Number of kernels qsa_decode launches per call for `batch` requests: 2 up to
  * 512 requests (the scorer runs the indexer front end itself, then the sparse
  * GQA), 3 above (a separate front-end kernel first). */

@@ -104,6 +104,24 @@ def test_prefill_scorer_agrees_with_streaming_scorer(Q, W):
     assert clear > 20
 
 
+@pytest.mark.parametrize("pos0,T", [(0, 3000), (200000, 64)])
+def test_prefill_rotation_is_the_rounded_rope(Q, W, pos0, T):
+    """Every rotated index query of the call is the oracle's rotation at the query's position (pinned to
+    the complex-multiply definition), rounded once to bf16: bit for bit, at short and long positions."""
+    wl = G.custom_decode(77 + T, [pos0 + T])
+    cache = W.build_cache(wl, prefix_tokens=[pos0 + T])
+    idx_q = wl.idx_q(0, q0=pos0, n=T)
+    w = wl.w(0, q0=pos0, n=T)
+    ws = Q.Workspace(Q.workspace_bytes(Q.OP_PREFILL_SCORE_TOPK, T, pos0 + T))
+    Q.prefill_score_topk(cache, W.bits_to_bf16(idx_q, "cuda"), torch.from_numpy(w).cuda(), 0, pos0, ws)
+    torch.cuda.synchronize()
+    assert ws.device_error() == 0
+    got = Q.prefill_rotated_queries(ws, T, pos0 + T)
+    for i in range(T):
+        ref = O.rotate_query(idx_q[i], pos0 + i, wl.rope_theta)
+        np.testing.assert_array_equal(got[i].reshape(-1), ref.reshape(-1), err_msg=f"row {pos0 + i}")
+
+
 def test_prefill_scorer_32k(Q, W):
     """The 32768-token prefill: every row's kept set is valid; sampled rows match the oracle."""
     wl = G.prefill_32k()
