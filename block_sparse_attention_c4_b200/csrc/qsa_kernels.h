@@ -177,6 +177,7 @@ struct PrefillParams {
   int* err;
   uint64_t wait_ns;        // limit of each mbarrier wait (0: WAIT_LIMIT_NS)
   int* stats;              // nullable [4]: rows selected from candidates, rows re-scored, candidates, -
+  int sel_r0, sel_pivot;   // one segment, sel_pivot > 0: the selection's row order (see k_prefill_select)
 };
 
 // ---- index projection (qsa_proj.cu) ----
@@ -232,7 +233,7 @@ cudaError_t launch_split_combine(const __nv_bfloat16* outs, const float* lses, i
                                  __nv_bfloat16* out, cudaStream_t st);
 
 // ev (nullable): n_ev event pairs recorded around the rotation, scoring and finalize kernels.
-cudaError_t launch_prefill(const PrefillParams& p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,
+cudaError_t launch_prefill(PrefillParams p, const __nv_bfloat16* idx_q, const RopeFreqs& fr, int num_sms,
                            cudaStream_t st, const cudaEvent_t* ev, int n_ev);
 
 }  // namespace qsa
