@@ -257,6 +257,8 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
     k_prefill_score(PrefillParams p, const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap) {
   constexpr int PF_EPI_WARPS = EW;
   constexpr int PF_QPW = PF_QT * 4 / EW;  // queries per epilogue warp
+  // the 8-warp form runs only calls whose tiles all write dense keys: no sample, no candidate code
+  constexpr bool DENSE_ONLY = EW == PF_EPI_WARPS_DENSE;
   static_assert(EW % 4 == 0 && PF_QPW % 8 == 0, "epilogue warps cover the four TMEM quadrants evenly");
   static_assert(PF_QPW <= 32, "one lane per query of an epilogue warp holds its list counter");
   extern __shared__ uint8_t smem_raw[];
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
       unsigned long long* list0 = p.cand + (int64_t)(tl.q_off + t0) * PF_ROW_WORDS + quad * PF_QCAP;
       // dense tile: the score keys of the warp's first query's row; query q0 + jl's are 2 * PF_ROW_WORDS on
       uint32_t* dkeys0 = reinterpret_cast<uint32_t*>(p.cand + (int64_t)(tl.q_off + t0) * PF_ROW_WORDS);
-      const bool dense = tl.dense();
+      const bool dense = DENSE_ONLY || tl.dense();
 
       for (int k = 0; k < nk; ++k, ++m_it) {
         const int mt = pf_mt_of(k, ns);
@@ -520,12 +522,13 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
 #pragma unroll
               for (int jj = 0; jj < 8; ++jj)
                 if ((vis8 >> jj) & 1u) dkeys0[(int64_t)(half * 8 + jj) * (2 * PF_ROW_WORDS) + b] = to_key(sc[jj]);
-            } else if (k < ns) {
+            } else if constexpr (!DENSE_ONLY) {
+              if (k < ns) {
 #pragma unroll
-              for (int jj = 0; jj < 8; ++jj)
-                if ((vis8 >> jj) & 1u)
-                  atomicAdd(&S.hist[(q0 + half * 8 + jj) * PF_HIST_STRIDE + pf_bin(to_key(sc[jj]), S.base[q0 + half * 8 + jj])], 1u);
-            } else {
+                for (int jj = 0; jj < 8; ++jj)
+                  if ((vis8 >> jj) & 1u)
+                    atomicAdd(&S.hist[(q0 + half * 8 + jj) * PF_HIST_STRIDE + pf_bin(to_key(sc[jj]), S.base[q0 + half * 8 + jj])], 1u);
+              } else {
               uint32_t em = 0u;  // queries this thread's block is a candidate of
               const float4 ta = *reinterpret_cast<const float4*>(&S.tau[q0 + half * 8]);
               const float4 tb = *reinterpret_cast<const float4*>(&S.tau[q0 + half * 8 + 4]);
@@ -548,10 +551,11 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
                   }
                 }
               }
+              }
             }
           }
         }
-        if (k == ns - 1) {  // the sample is complete: each query's threshold
+        if (!DENSE_ONLY && k == ns - 1) {  // the sample is complete: each query's threshold
           asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
           if (etid < PF_QT) {
             const int t = tl.qt * PF_QT + etid;
@@ -562,10 +566,12 @@ __global__ void __launch_bounds__(pf_threads<EW>(), 1)
           asm volatile("bar.sync 1, %0;" ::"n"(PF_EPI_WARPS * 32) : "memory");
         }
       }
-      int mine = 0;
+      if constexpr (!DENSE_ONLY) {  // dense rows' lists are never read
+        int mine = 0;
 #pragma unroll
-      for (int j2 = 0; j2 < PF_QPW; ++j2) mine = lane == j2 ? cntq[j2] : mine;
-      if (lane < PF_QPW && t0 + lane < tl.T) p.cand_n[(int64_t)(tl.q_off + t0 + lane) * 4 + quad] = mine;
+        for (int j2 = 0; j2 < PF_QPW; ++j2) mine = lane == j2 ? cntq[j2] : mine;
+        if (lane < PF_QPW && t0 + lane < tl.T) p.cand_n[(int64_t)(tl.q_off + t0 + lane) * 4 + quad] = mine;
+      }
     }
   }
   tc_fence_before();
