@@ -612,6 +612,7 @@ constexpr int PS_TIE_CAP = 256;
 constexpr int PS_SUB_BINS = 256;   // second level: the 8 key bits below a first-level bin
 constexpr int PS_TIE_RANK = 48;    // more gathered ties than this are split by sub-bin before ranking
 constexpr int PS_U = 8;            // loads in flight per lane
+constexpr int PS_DENSE_U = 6;      // dense rows: 16-byte loads in flight per lane (4: +8 us, 8: +18 us at L = 32768)
 constexpr int PS_DSPLIT_LOG = 2;                 // dense rows: 4 bins per candidate bin, i.e. 512 bins
 constexpr int PS_DSPLIT = 1 << PS_DSPLIT_LOG;     // of 1/64 octave (key >> 17) over the same 8 octaves
 constexpr int PS_DBINS = PF_BINS * PS_DSPLIT;
@@ -827,7 +828,7 @@ __device__ bool ps_candidate_row(ForEach for_each, int n, int qbase, uint32_t* h
 __device__ bool ps_dense_row(const uint32_t* keys, int n, int qbase, uint32_t* hist, unsigned long long* tie,
                              uint32_t* bitmap, int32_t* sel, int* err, int* sel_n) {
   using F = PsForm<true>;
-  constexpr int U = PS_U / 2;  // 16-byte loads in flight per lane
+  constexpr int U = PS_DENSE_U;  // 16-byte loads in flight per lane
   const int lane = threadIdx.x & 31;
   if (qbase == PF_NO_BASE) return false;
   const F f{qbase * PS_DSPLIT};
