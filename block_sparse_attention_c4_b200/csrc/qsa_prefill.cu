@@ -611,7 +611,7 @@ constexpr double PS_L2_FIRST_BYTES = 64.0 * 1048576.0;
 constexpr int PS_TIE_CAP = 256;
 constexpr int PS_SUB_BINS = 256;   // second level: the 8 key bits below a first-level bin
 constexpr int PS_TIE_RANK = 48;    // more gathered ties than this are split by sub-bin before ranking
-constexpr int PS_U = 8;            // loads in flight per lane
+constexpr int PS_U = 8;            // candidate rows: 8-byte loads in flight per lane
 constexpr int PS_DENSE_U = 6;      // dense rows: 16-byte loads in flight per lane (4: +8 us, 8: +18 us at L = 32768)
 constexpr int PS_DSPLIT_LOG = 2;                 // dense rows: 4 bins per candidate bin, i.e. 512 bins
 constexpr int PS_DSPLIT = 1 << PS_DSPLIT_LOG;     // of 1/64 octave (key >> 17) over the same 8 octaves
